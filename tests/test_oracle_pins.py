@@ -1,0 +1,344 @@
+"""Pins of the float64 oracle to facts that do not come from the oracle.
+
+Each test ties one oracle function to a closed form, an invariant of the
+mathematics, a value printed on the pages (tests/golden/), or an
+independent pure-Python loop, so that a dropped term, a wrong sign or index
+or a transposed operand fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import bruteforce as bf
+from oracle import lrkv_oracle as orc
+from rank_kv_cache_lrkv_b200 import workloads as wk
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+D = 128
+
+
+def _orth(rng, n, r):
+    q, rr = np.linalg.qr(rng.standard_normal((n, r)))
+    return q * np.sign(np.diag(rr))[None, :]
+
+
+# ------------------------------------------------------------ attention
+
+def test_full_rank_orthonormal_basis_reproduces_dense_attention():
+    """Half the Memory, section 04: routing the uncompressed cache through
+    the path reproduces the model's output.  r = 128 with an orthonormal
+    basis is that case: latent attention must equal dense attention."""
+    rng = np.random.default_rng(1)
+    Pk, Pv = _orth(rng, D, D), _orth(rng, D, D)
+    K, V = rng.standard_normal((40, D)), rng.standard_normal((40, D))
+    q = rng.standard_normal(D)
+    o_lat = orc.latent_attention(q, Pk, Pv, orc.project(Pk, K), orc.project(Pv, V),
+                                 np.zeros((0, D)), np.zeros((0, D)), 0.3)
+    o_dense = orc.dense_attention(q, K, V, 0.3)
+    assert np.max(np.abs(o_lat - o_dense)) < 1e-12 * np.max(np.abs(o_dense)) + 1e-13
+
+
+def test_latent_equals_reconstructed_for_any_basis():
+    """Section 08: attending on the codes is algebraically equal to
+    attending over reconstructed tensors; true for any (non-orthonormal) P."""
+    rng = np.random.default_rng(2)
+    Pk = rng.standard_normal((D, 24)) * 0.2
+    Pv = rng.standard_normal((D, 16)) * 0.2
+    Ck, Cv = rng.standard_normal((30, 24)), rng.standard_normal((30, 16))
+    Ka, Va = rng.standard_normal((5, D)), rng.standard_normal((5, D))
+    q = rng.standard_normal(D)
+    a = orc.latent_attention(q, Pk, Pv, Ck, Cv, Ka, Va, 0.2)
+    b = orc.reconstructed_attention(q, Pk, Pv, Ck, Cv, Ka, Va, 0.2)
+    assert np.max(np.abs(a - b)) < 1e-12 * np.max(np.abs(b))
+
+
+def test_bruteforce_loops_match_vectorised_oracle():
+    """Independent pure-Python loops on tiny inputs (T <= 16, r <= 8)."""
+    rng = np.random.default_rng(3)
+    for trial in range(3):
+        rk, rv, n, na = 8, 4 + trial, 9 + 3 * trial, trial
+        Pk, Pv = rng.standard_normal((D, rk)), rng.standard_normal((D, rv))
+        Xk, Xv = rng.standard_normal((n, D)), rng.standard_normal((n, D))
+        Ck, Cv = orc.project(Pk, Xk), orc.project(Pv, Xv)
+        assert np.max(np.abs(Ck - np.array(bf.codes(Pk.tolist(), Xk.tolist())))) < 1e-12
+        Ka, Va = rng.standard_normal((na, D)), rng.standard_normal((na, D))
+        q = rng.standard_normal(D)
+        o = orc.latent_attention(q, Pk, Pv, Ck, Cv, Ka, Va, 0.125)
+        ob = bf.attention(q.tolist(), Pk.tolist(), Pv.tolist(), Ck.tolist(),
+                          Cv.tolist(), Ka.tolist(), Va.tolist(), 0.125)
+        assert np.max(np.abs(o - np.array(ob))) < 1e-13 * max(1.0, np.max(np.abs(o)))
+
+
+def test_softmax_rows_sum_to_one_and_survive_huge_scores():
+    rng = np.random.default_rng(4)
+    for scale in [1.0, 1e3, 1e6]:
+        p = orc.softmax(rng.standard_normal(1000) * scale)
+        assert abs(p.sum() - 1.0) < 1e-15 * 1000
+        assert np.all(np.isfinite(p)) and np.all(p >= 0)
+
+
+def test_single_token_returns_its_reconstructed_value():
+    rng = np.random.default_rng(5)
+    Pk, Pv = rng.standard_normal((D, 8)), rng.standard_normal((D, 8))
+    ck, cv = rng.standard_normal((1, 8)), rng.standard_normal((1, 8))
+    o = orc.latent_attention(rng.standard_normal(D), Pk, Pv, ck, cv,
+                             np.zeros((0, D)), np.zeros((0, D)), 1.0)
+    assert np.max(np.abs(o - Pv @ cv[0])) < 1e-14 * np.max(np.abs(o))
+    va = rng.standard_normal((1, D))
+    o2 = orc.latent_attention(rng.standard_normal(D), Pk, Pv, np.zeros((0, 8)),
+                              np.zeros((0, 8)), rng.standard_normal((1, D)), va, 1.0)
+    assert np.array_equal(o2, va[0])
+
+
+def test_zero_query_gives_mean_of_values():
+    """q = 0 makes every score 0, so softmax is uniform."""
+    rng = np.random.default_rng(6)
+    Pk, Pv = rng.standard_normal((D, 8)), rng.standard_normal((D, 6))
+    Ck, Cv = rng.standard_normal((7, 8)), rng.standard_normal((7, 6))
+    Ka, Va = rng.standard_normal((3, D)), rng.standard_normal((3, D))
+    o = orc.latent_attention(np.zeros(D), Pk, Pv, Ck, Cv, Ka, Va, 1.0)
+    mean = (np.sum(Cv @ Pv.T, 0) + np.sum(Va, 0)) / 10.0
+    assert np.max(np.abs(o - mean)) < 1e-14 * np.max(np.abs(mean))
+
+
+def test_token_permutation_does_not_change_output():
+    rng = np.random.default_rng(7)
+    Pk, Pv = rng.standard_normal((D, 16)), rng.standard_normal((D, 8))
+    Ck, Cv = rng.standard_normal((50, 16)), rng.standard_normal((50, 8))
+    q = rng.standard_normal(D)
+    z = np.zeros((0, D))
+    a = orc.latent_attention(q, Pk, Pv, Ck, Cv, z, z, 0.1)
+    perm = rng.permutation(50)
+    b = orc.latent_attention(q, Pk, Pv, Ck[perm], Cv[perm], z, z, 0.1)
+    assert np.max(np.abs(a - b)) < 1e-14 * np.max(np.abs(a))
+
+
+def test_gqa_head_h_reads_kv_head_h_over_G():
+    rng = np.random.default_rng(8)
+    B, Hkv, G = 2, 3, 2
+    c = orc.LatentCacheOracle(B, Hkv, 8, 8)
+    Pk = rng.standard_normal((1, Hkv, D, 8))
+    Pv = rng.standard_normal((1, Hkv, D, 8))
+    k, v = rng.standard_normal((B, Hkv, 6, D)), rng.standard_normal((B, Hkv, 6, D))
+    c.append(k, v, Pk, Pv)
+    q = rng.standard_normal((B, Hkv * G, D))
+    o = c.attend(q, Pk, Pv, 0.1)
+    for b in range(B):
+        for h in range(Hkv * G):
+            g = h // G
+            ref = orc.dense_attention(q[b, h], orc.reconstruct(Pk[0, g], orc.project(Pk[0, g], k[b, g])),
+                                      orc.reconstruct(Pv[0, g], orc.project(Pv[0, g], v[b, g])), 0.1)
+            assert np.max(np.abs(o[b, h] - ref)) < 1e-12 * np.max(np.abs(ref))
+
+
+# ------------------------------------------------------------ cache / anchors
+
+def test_all_anchor_cache_is_dense_attention_and_stores_inputs_bitwise():
+    """OjaKV anchors are kept full-rank: a cache whose tokens are all anchors
+    must be ordinary attention, with the anchor rows equal to the inputs."""
+    rng = np.random.default_rng(9)
+    T = 20
+    c = orc.LatentCacheOracle(1, 1, 8, 8, n_sink=1, window=T)
+    k, v = rng.standard_normal((1, 1, T, D)), rng.standard_normal((1, 1, T, D))
+    P = rng.standard_normal((1, 1, D, 8))
+    c.append(k, v, P, P)
+    Ka, Va = c.anchors(0, 0)
+    assert np.array_equal(Ka, k[0, 0]) and np.array_equal(Va, v[0, 0])
+    assert c.codes_k[0][0].shape[0] == 0
+    q = rng.standard_normal((1, 1, D))
+    o = c.attend(q, P, P, 0.2)
+    assert np.max(np.abs(o[0, 0] - orc.dense_attention(q[0, 0], k[0, 0], v[0, 0], 0.2))) < 1e-13
+
+
+@pytest.mark.parametrize("n_sink,W", [(0, 0), (1, 0), (0, 5), (1, 5), (1, 64)])
+def test_partition_and_chunked_appends(n_sink, W):
+    """First token (sink) and the W most recent tokens full-rank, the rest
+    compressed in order; appending in any chunking gives the same state."""
+    rng = np.random.default_rng(10 + W)
+    B, Hkv, T = 2, 2, 37
+    k, v = rng.standard_normal((B, Hkv, T, D)), rng.standard_normal((B, Hkv, T, D))
+    P = rng.standard_normal((1, Hkv, D, 8))
+    one = orc.LatentCacheOracle(B, Hkv, 8, 8, n_sink, W)
+    one.append(k, v, P, P)
+    chunked = orc.LatentCacheOracle(B, Hkv, 8, 8, n_sink, W)
+    pos = 0
+    for n in [1, 3, 0, 10, 2, 21]:
+        chunked.append(k[:, :, pos:pos + n], v[:, :, pos:pos + n], P, P)
+        pos += n
+    assert pos == T
+    sink, lat, win = orc.partition(T, n_sink, W)
+    assert len(sink) + len(lat) + len(win) == T
+    for b in range(B):
+        for h in range(Hkv):
+            for c in (one, chunked):
+                assert np.allclose(c.codes_k[b][h], k[b, h, lat] @ P[0, h], rtol=0, atol=1e-12)
+                Ka, Va = c.anchors(b, h)
+                assert np.array_equal(Ka, k[b, h, sink + win])
+                assert np.array_equal(Va, v[b, h, sink + win])
+
+
+def test_evicted_tokens_use_the_basis_current_at_eviction():
+    rng = np.random.default_rng(11)
+    k, v = rng.standard_normal((1, 1, 6, D)), rng.standard_normal((1, 1, 6, D))
+    P1, P2 = rng.standard_normal((1, 1, D, 4)), rng.standard_normal((1, 1, D, 4))
+    c = orc.LatentCacheOracle(1, 1, 4, 4, 0, 2)
+    c.append(k[:, :, :4], v[:, :, :4], P1, P1)   # tokens 0,1 evicted with P1
+    c.append(k[:, :, 4:], v[:, :, 4:], P2, P2)   # tokens 2,3 evicted with P2
+    exp = np.concatenate([k[0, 0, :2] @ P1[0, 0], k[0, 0, 2:4] @ P2[0, 0]])
+    assert np.allclose(c.codes_k[0][0], exp, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ basis
+
+def test_eckart_young_tail_energy_with_planted_spectrum():
+    """Rank-r reconstruction error of the top-r SVD basis equals the sum of
+    the squared tail singular values, which are planted here (not computed)."""
+    rng = np.random.default_rng(12)
+    n = 300
+    U = _orth(rng, n, D)
+    Vt = _orth(rng, D, D).T
+    sig = np.exp(-np.arange(D) / 10.0) * 3.0
+    X = (U * sig[None, :]) @ Vt
+    for r in [8, 32, 64, 127]:
+        P = orc.svd_basis(X, r)
+        err = np.sum((X - orc.reconstruct(P, orc.project(P, X))) ** 2)
+        tail = np.sum(sig[r:] ** 2)
+        assert abs(err - tail) <= 1e-10 * tail + 1e-13 * np.sum(sig ** 2)
+        assert np.max(np.abs(P.T @ P - np.eye(r))) < 1e-12
+
+
+def test_generator_tail_energy_matches_its_spectrum():
+    """The seeded generator's decaying spectrum: relative tail energy of a
+    rank-r SVD basis is sum_{i>=r} s_i^2 / sum s_i^2 (statistically)."""
+    wl = wk.TINY_SINGLE_HEAD
+    for kind, r in [("k", 64), ("v", 32), ("k", 16)]:
+        s2 = wk.spectrum(kind) ** 2
+        expect = s2[r:].sum() / s2.sum()
+        X = wk.stream(wl, kind, 0, 0, 0, n=2048)
+        P = wk.basis(wl.with_(r_k=r, r_v=r), kind, 0, 0).astype(np.float64)
+        rel = np.sum((X - orc.reconstruct(P, orc.project(P, X))) ** 2) / np.sum(X ** 2)
+        assert 0.8 * expect < rel < 1.25 * expect, (kind, r, rel, expect)
+
+
+# ------------------------------------------------------------ Oja
+
+def test_oja_single_step_closed_form():
+    """P = e1 (r = 1), x = a e1 + b e2: y = a, x - P y = b e2, so the new
+    basis is e1 + eta a b e2 (worked by hand)."""
+    a, b, eta = 2.0, 3.0, 0.1
+    P = np.zeros((D, 1))
+    P[0, 0] = 1.0
+    x = np.zeros(D)
+    x[0], x[1] = a, b
+    out = orc.oja_update(P, x[None, :], eta, 0)
+    exp = P.copy()
+    exp[1, 0] = eta * a * b
+    assert np.array_equal(out, exp)
+    out_c = orc.oja_update_streams(P[None], x[None, None, :], eta, 0)[0]
+    assert np.array_equal(out_c, exp)
+
+
+def test_oja_in_span_is_a_fixed_point():
+    rng = np.random.default_rng(13)
+    P = _orth(rng, D, 6)
+    X = rng.standard_normal((20, 6)) @ P.T
+    out = orc.oja_update(P, X, 0.05, 0)
+    assert np.max(np.abs(out - P)) < 1e-14
+
+
+def test_oja_step_matches_bruteforce_loops():
+    rng = np.random.default_rng(14)
+    P = rng.standard_normal((D, 5)) * 0.1
+    x = rng.standard_normal(D)
+    a = orc.oja_update(P, x[None], 0.01, 0)
+    b = np.array(bf.oja_step(P.tolist(), x.tolist(), 0.01))
+    assert np.max(np.abs(a - b)) < 1e-14
+
+
+def test_oja_qr_orthonormal_with_positive_diagonal():
+    rng = np.random.default_rng(15)
+    P = rng.standard_normal((D, 12))
+    Q = orc.qr_positive(P)
+    assert np.max(np.abs(Q.T @ Q - np.eye(12))) < 1e-13
+    R = Q.T @ P
+    assert np.max(np.abs(np.tril(R, -1))) < 1e-12 and np.all(np.diag(R) > 0)
+    assert np.max(np.abs(Q @ R - P)) < 1e-12
+
+
+def test_oja_c_loop_matches_numpy_loop_with_qr():
+    rng = np.random.default_rng(16)
+    S, r, n = 3, 8, 70
+    P0 = np.stack([_orth(rng, D, r) for _ in range(S)])
+    X = rng.standard_normal((S, n, D)).astype(np.float32)
+    Pc = orc.oja_update_streams(P0, X, 0.02, 16, tokens_seen=5)
+    for s in range(S):
+        Pn = orc.oja_update(P0[s], X[s].astype(np.float64), 0.02, 16, tokens_seen=5)
+        assert np.max(np.abs(Pc[s] - Pn)) < 1e-12
+
+
+def test_oja_two_half_calls_equal_one_call():
+    rng = np.random.default_rng(17)
+    P0 = _orth(rng, D, 8)
+    X = rng.standard_normal((100, D))
+    one = orc.oja_update(P0, X, 0.01, 32)
+    two = orc.oja_update(orc.oja_update(P0, X[:50], 0.01, 32), X[50:], 0.01, 32,
+                         tokens_seen=50)
+    assert np.max(np.abs(one - two)) < 1e-12
+
+
+def test_oja_is_rotation_equivariant():
+    """P -> P R (R orthogonal) maps the trajectory to P_t R without QR; with
+    QR the projector P P^T is unchanged."""
+    rng = np.random.default_rng(18)
+    P0 = _orth(rng, D, 6)
+    R = _orth(rng, 6, 6)
+    X = rng.standard_normal((60, D))
+    a = orc.oja_update(P0, X, 0.01, 0)
+    b = orc.oja_update(P0 @ R, X, 0.01, 0)
+    assert np.max(np.abs(a @ R - b)) < 1e-12
+    a = orc.oja_update(P0, X, 0.01, 20)
+    b = orc.oja_update(P0 @ R, X, 0.01, 20)
+    assert np.max(np.abs(a @ a.T - b @ b.T)) < 1e-12
+
+
+def test_oja_tracks_a_planted_subspace():
+    """On data drawn from a planted r-dim subspace plus small noise the
+    projector distance to the planted subspace shrinks while it is far above
+    the noise floor, and ends near that floor."""
+    rng = np.random.default_rng(19)
+    r = 4
+    U = _orth(rng, D, r)
+    P = _orth(rng, D, r)
+    X = rng.standard_normal((3000, r)) @ (U.T * 3.0) + 0.01 * rng.standard_normal((3000, D))
+    dist = [np.linalg.norm(P @ P.T - U @ U.T)]
+    for c in range(6):
+        P = orc.oja_update(P, X[c * 100:(c + 1) * 100], 0.001, 50, tokens_seen=c * 100)
+        dist.append(np.linalg.norm(P @ P.T - U @ U.T))
+    assert all(dist[i + 1] < dist[i] for i in range(len(dist) - 1)), dist
+    P = orc.oja_update(P, X[600:], 0.01, 50, tokens_seen=600)
+    assert np.linalg.norm(P @ P.T - U @ U.T) < 0.05 * dist[0]
+
+
+# ------------------------------------------------------------ sizes
+
+def test_llama_kv_cache_is_16_gib():
+    g = json.load(open(os.path.join(GOLDEN, "kv_cache_sizes.json")))["llama31_8b_dense_32k_b4"]
+    n = orc.kv_cache_bytes(g["layers"], g["kv_heads"], g["head_dim"], g["tokens"],
+                           g["batch"], g["bytes_per_elem"])
+    assert n == g["exact_gib"] * 2 ** 30
+    assert abs(n / 1e9 - g["stated_gb_approx"]) / g["stated_gb_approx"] < 0.1
+
+
+def test_two_x_compression_halves_the_cache_and_values_at_quarter():
+    g = json.load(open(os.path.join(GOLDEN, "kv_cache_sizes.json")))
+    h = g["halved_at_2x"]
+    assert orc.compression_ratio(h["r_k_plus_r_v"] // 2, h["r_k_plus_r_v"] // 2) == h["ratio"]
+    dense = orc.kv_cache_bytes(1, 8, 128, 4096, 2)
+    lat = orc.latent_cache_bytes(1, 8, 64, 64, 4096, 2)
+    assert dense == 2 * lat
+    q = g["values_at_quarter"]
+    assert q["r_v"] / q["head_dim"] == q["fraction"]
+    assert math.isclose(orc.compression_ratio(64, 32), 256 / 96)
