@@ -1,0 +1,425 @@
+"""Decode benchmark of the latent-KV cache (one process per GPU).
+
+Workload (default): the Llama-3.1-8B-shaped layer with hybrid anchors,
+B=4, H_q=32, H_kv=8, d=128, 32K-token prompt, token 0 and the 128 most
+recent tokens full-rank bf16, all other tokens r_k=64 / r_v=32 bf16 codes.
+A step is one decode step of every sequence: lrkv_compress of the new token
+(window append + eviction of the oldest window token into codes) and
+lrkv_decode_attn (q-fold, split-K over the codes and anchors, merge with the
+value up-projection).
+
+Prints one JSON line (rank 0).  `value` is decode tokens/s over all ranks
+(B * steps * N / max-over-ranks time, device time with CUDA events around a
+CUDA graph of the timed steps).  Extra keys: the lrkv_decode_attn roofline
+(algorithmic bytes: codes + anchors + q + o), the dense bf16 decode baseline
+measured in the same run, an end-to-end number through the Python API with
+host buffers, the oracle on the host cores, and SM clocks sampled during the
+timed region.
+
+--impl reference runs the float64 oracle (the only reference this method
+has) on the host cores instead.
+"""
+import argparse
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEAD_DIM = 128
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=256)
+    p.add_argument("--warmup", type=int, default=8)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="llama32k", choices=["llama32k", "qwen8k"])
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    return p.parse_args()
+
+
+def workload(name):
+    from rank_kv_cache_lrkv_b200 import workloads as wk
+    return {"llama32k": wk.LLAMA31_LAYER_32K_ANCHORS, "qwen8k": wk.QWEN3_LAYER_8K}[name]
+
+
+def config_of(wl):
+    return {"workload": wl.name, "B": wl.B, "H_q": wl.H_q, "H_kv": wl.H_kv, "head_dim": HEAD_DIM,
+            "T": wl.T, "r_k": wl.r_k, "r_v": wl.r_v, "n_sink": wl.n_sink, "window": wl.window,
+            "codes": wl.dtype, "accumulate": "fp32",
+            "l2": "no flush: every decode step streams the whole code cache, larger than L2"}
+
+
+def step_bytes(wl, L):
+    """Algorithmic bytes of one decode-attention call at sequence length L:
+    latent codes + full-rank anchors + q + o (bf16)."""
+    es = 2 if wl.dtype == "bf16" else 4
+    sink = min(L, wl.n_sink)
+    win = min(L - sink, wl.window)
+    lat = L - sink - win
+    units = wl.B * wl.H_kv
+    return (units * lat * (wl.r_k + wl.r_v) * es + units * (sink + win) * 2 * HEAD_DIM * es
+            + 2 * wl.B * wl.H_q * HEAD_DIM * es)
+
+
+def dense_step_bytes(wl, L):
+    es = 2 if wl.dtype == "bf16" else 4
+    return wl.B * wl.H_kv * L * 2 * HEAD_DIM * es + 2 * wl.B * wl.H_q * HEAD_DIM * es
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls NVML (the library nvidia-smi reads) for SM clock and throttle
+    reasons while the timed region runs."""
+
+    def __init__(self, index=0, period=0.002):
+        self.samples, self.period, self.index = [], period, index
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        nv = self.nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        mhz = sorted(s[0] for s in self.samples)
+        seen = set()
+        for _, rs in self.samples:
+            for n, bit in names.items():
+                if rs & bit and n != "gpu_idle":
+                    seen.add(n)
+        return {"sm_mhz": mhz[len(mhz) // 2] if mhz else None, "sm_max_mhz": self.max_mhz,
+                "samples": len(mhz), "reasons": sorted(seen)}
+
+
+# ------------------------------------------------------------------ oracle
+class OracleUnit:
+    """The float64 oracle on one (sequence, KV head) unit of the workload:
+    its prompt is compressed once; a decode step appends one token and
+    attends with the unit's G query heads."""
+
+    def __init__(self, wl, inp):
+        import numpy as np
+        from oracle import lrkv_oracle as orc
+        self.np, self.wl = np, wl
+        self.Pk = inp["P_k"][0:1].double().numpy()[None]
+        self.Pv = inp["P_v"][0:1].double().numpy()[None]
+        self.K = inp["K"][0:1, 0:1].double().numpy()
+        self.V = inp["V"][0:1, 0:1].double().numpy()
+        self.oc = orc.LatentCacheOracle(1, 1, wl.r_k, wl.r_v, wl.n_sink, wl.window)
+        self.oc.append(self.K[:, :, :wl.T], self.V[:, :, :wl.T], self.Pk, self.Pv)
+        self.rng = np.random.default_rng(0)
+        self.n = 0
+
+    def run(self, seconds):
+        """Decode steps for about `seconds`; returns (steps, seconds per step)."""
+        wl, np = self.wl, self.np
+        n, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < seconds or n == 0:
+            t = wl.T + (self.n % (self.K.shape[2] - wl.T))
+            self.oc.append(self.K[:, :, t:t + 1], self.V[:, :, t:t + 1], self.Pk, self.Pv)
+            q = self.rng.standard_normal((1, wl.G, HEAD_DIM)) / np.sqrt(HEAD_DIM)
+            self.oc.attend(q, self.Pk, self.Pv, wl.scale)
+            n += 1
+            self.n += 1
+        return n, (time.perf_counter() - t0) / n
+
+
+def host_cores():
+    try:
+        import threadpoolctl
+        return max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_text(wl, n):
+    units = wl.B * wl.H_kv
+    return (f"{n} float64 oracle decode steps (append + attend) of 1 of the {units} "
+            f"(sequence, KV head) units at {wl.T}-token context; a full step is taken "
+            f"as {units} x the unit time")
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    from rank_kv_cache_lrkv_b200 import lrkv
+    from rank_kv_cache_lrkv_b200 import workloads as wk
+
+    base = workload(args.workload)
+    W, K = args.warmup, args.steps
+    E = 0 if args.no_e2e else min(K, 64)
+    wl = base.with_(n_decode=W + K + E + 2)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = wk.layer_inputs(wl)
+    qs = wk.layer_queries(wl).to(dev)
+    Kd, Vd = inp["K"].to(dev), inp["V"].to(dev)
+    Pk, Pv = inp["P_k"].to(dev), inp["P_v"].to(dev)
+    cap = wl.T + wl.n_decode
+    cache = lrkv.LatentCache(wl.B, wl.H_kv, wl.r_k, wl.r_v, cap, wl.n_sink, wl.window,
+                             dtype=Kd.dtype, device=dev)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    lrkv.compress(cache, Kd[:, :, :wl.T], Vd[:, :, :wl.T], Pk, Pv)
+    e1.record()
+    torch.cuda.synchronize()
+    prefill_ms = e0.elapsed_time(e1)
+    ws = lrkv.decode_workspace(cache, wl.H_q, device=dev)
+    o = torch.empty_like(qs[0])
+
+    def step(s):
+        t = wl.T + s
+        lrkv.compress(cache, Kd[:, :, t:t + 1], Vd[:, :, t:t + 1], Pk, Pv)
+        lrkv.decode_attn(cache, qs[s], Pk, Pv, wl.scale, o, ws)
+
+    for s in range(W):
+        step(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        for s in range(W, W + K):
+            step(s)
+    torch.cuda.synchronize()
+    L_mid = wl.T + W + K // 2
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    assert lrkv.workspace_error(ws) == 0
+
+    # roofline of lrkv_decode_attn alone: the same call replayed (state fixed)
+    R = 200
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, capture_error_mode="relaxed"):
+        for _ in range(R):
+            lrkv.decode_attn(cache, qs[0], Pk, Pv, wl.scale, o, ws)
+    g2.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    g2.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    attn_ms = e0.elapsed_time(e1) / R
+    L_now = wl.T + W + K
+    abytes = step_bytes(wl, L_now)
+    pk = peaks()
+    hbm = pk["hbm_gbs"] if pk else 6650.0
+    achieved = abytes / (attn_ms * 1e-3) / 1e9
+    out = {
+        "metric": "latent-KV decode tokens/s and achieved HBM GB/s (fraction of ~8 TB/s) at 1 GPU",
+        "value": round(wl.B * K * world / (ms * 1e-3), 2),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": dict(config_of(wl), parallelism=f"replicas{world}"),
+        "gpu_launches": 4 * K,
+        "roofline": {"kernel": "lrkv_decode_attn (qfold + split + merge)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "frac_of_8TBs": round(achieved / 8000, 4),
+                     "peak_source": "MEASURED_PEAKS.json hbm_gbs" if pk else "fallback",
+                     "bytes_per_call": abytes, "us_per_call": round(attn_ms * 1e3, 3),
+                     "context": L_now, "traffic": None},
+        "prefill_compress": {"tokens": wl.T * wl.B, "ms": round(prefill_ms, 3),
+                             "tokens_per_s": round(wl.T * wl.B / (prefill_ms * 1e-3), 1)},
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_dense:
+        dc = lrkv.DenseCache(wl.B, wl.H_kv, cap, dtype=Kd.dtype, device=dev)
+        lrkv.dense_append(dc, Kd[:, :, :wl.T + W], Vd[:, :, :wl.T + W])
+        dws = lrkv.dense_decode_workspace(dc, wl.H_q, device=dev)
+        g3 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g3, capture_error_mode="relaxed"):
+            for s in range(W, W + K):
+                t = wl.T + s
+                lrkv.dense_append(dc, Kd[:, :, t:t + 1], Vd[:, :, t:t + 1])
+                lrkv.dense_decode_attn(dc, qs[s], wl.scale, o, dws)
+        torch.cuda.synchronize()
+        e0.record()
+        g3.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        dms = e0.elapsed_time(e1)
+        g4 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g4, capture_error_mode="relaxed"):
+            for _ in range(R):
+                lrkv.dense_decode_attn(dc, qs[0], wl.scale, o, dws)
+        g4.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        g4.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        dattn = e0.elapsed_time(e1) / R
+        db = dense_step_bytes(wl, L_now)
+        out["dense_baseline"] = {
+            "tokens_per_s": round(wl.B * K / (dms * 1e-3), 2), "ms_per_step": round(dms / K, 5),
+            "attn_us": round(dattn * 1e3, 3), "attn_GBs": round(db / (dattn * 1e-3) / 1e9, 1),
+            "bytes_per_call": db, "speedup_latent_over_dense": round(dms / ms, 3)}
+        del dc, g3, g4
+
+    if E:
+        # End to end through the public API with host buffers: per step the
+        # new k, v and q are copied from pinned host memory, and o read back.
+        a0 = wl.T + W + K
+        kh = inp["K"][:, :, a0:a0 + E].permute(2, 0, 1, 3).unsqueeze(3).contiguous().pin_memory()
+        vh = inp["V"][:, :, a0:a0 + E].permute(2, 0, 1, 3).unsqueeze(3).contiguous().pin_memory()
+        qh = wk.layer_queries(wl)[W + K:W + K + E].contiguous().pin_memory()
+        oh = torch.empty((E,) + tuple(o.shape), dtype=o.dtype).pin_memory()
+        kd = torch.empty((wl.B, wl.H_kv, 1, HEAD_DIM), dtype=Kd.dtype, device=dev)
+        vd = torch.empty_like(kd)
+        qd = torch.empty_like(qs[0])
+        torch.cuda.synchronize()
+        e0.record()
+        for s in range(E):
+            kd.copy_(kh[s], non_blocking=True)
+            vd.copy_(vh[s], non_blocking=True)
+            qd.copy_(qh[s], non_blocking=True)
+            lrkv.compress(cache, kd, vd, Pk, Pv)
+            lrkv.decode_attn(cache, qd, Pk, Pv, wl.scale, o, ws)
+            oh[s].copy_(o, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        es = kd.element_size()
+        out["e2e"] = {"value": round(wl.B * E * world / (ems * 1e-3), 2), "unit": "tokens/s",
+                      "h2d_bytes_per_step": 2 * kd.numel() * es + qd.numel() * es,
+                      "d2h_bytes_per_step": o.numel() * es, "steps": E}
+    if rank == 0 and world == 1 and not args.no_cpu:
+        n, per_unit = OracleUnit(wl, inp).run(args.cpu_seconds)
+        rate = wl.B / (per_unit * wl.B * wl.H_kv)
+        out["cpu_baseline"] = {"value": round(rate, 4), "unit": "tokens/s", "cores": host_cores(),
+                               "kind": "oracle", "sample": oracle_sample_text(wl, n)}
+    return out
+
+
+def run_reference(args, rank, world):
+    """The oracle arm: float64 decode steps on the host cores."""
+    from rank_kv_cache_lrkv_b200 import workloads as wk
+    base = workload(args.workload)
+    K, W = args.steps, args.warmup
+    wl = base.with_(n_decode=16)
+    # Inputs of one unit suffice for the bounded sample.
+    inp = wk.layer_inputs(wl.with_(B=1, H_kv=1, H_q=wl.G))
+    unit = OracleUnit(wl, inp)
+    per = max(0.2, min(2.0, 120.0 / max(1, K + W)))
+    rates, total = [], 0
+    for i in range(W + K):
+        n, dt = unit.run(per)
+        if i >= W:
+            rates.append(wl.B / (dt * wl.B * wl.H_kv))
+            total += n
+    rate = sorted(rates)[len(rates) // 2]
+    cores, sample = host_cores(), oracle_sample_text(wl, total)
+    step_ms = wl.B / rate * 1e3
+    return {"impl": "reference",
+            "metric": "latent-KV decode tokens/s and achieved HBM GB/s (fraction of ~8 TB/s) at 1 GPU",
+            "value": round(rate, 4), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": round(step_ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(config_of(wl), parallelism="host cores"),
+            "cpu_baseline": {"value": round(rate, 4), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(rate, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    import datetime
+    import torch
+    import torch.distributed as dist
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    try:
+        out = run_ours(args, rank, world)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,182 @@
+/* lrkv: low-rank latent KV cache with decode attention over the codes.
+ *
+ * C ABI of the CUDA library liblrkv.so (sm_100a).  Plain pointers and sizes
+ * only.  Unless a comment says "host", every pointer is DEVICE memory owned
+ * by the caller; the library keeps no state between calls and allocates no
+ * memory.  Every call is asynchronous on the given stream (a cudaStream_t
+ * passed as void*; NULL is the legacy default stream).  Arguments are
+ * checked on the host before anything is launched: a bad argument returns a
+ * negative status and launches nothing.  A failed launch returns
+ * LRKV_ERR_CUDA.  Errors inside a kernel surface at the caller's next
+ * synchronisation; kernels never trap.
+ *
+ * The method (pages: "Half the Memory, None of the Answers Lost" sections
+ * 04, 05 and 08; the OjaKV article; the Palu and LowRAM abstracts):
+ *  - each token's post-RoPE key k and value v (128 dims per KV head) are
+ *    stored as r-dim codes c_k = P_k^T k and c_v = P_v^T v under a
+ *    per-(layer, KV head) basis P in R^{128 x r};
+ *  - the first token (sink) and a window of the W most recent tokens stay
+ *    full-rank (OjaKV: first and most recent tokens kept as anchors); a
+ *    token that leaves the window is compressed with the basis passed to
+ *    the call that evicts it;
+ *  - decode attention runs on the codes: q~ = P_k^T q, s_t = q~ . c_k,t *
+ *    scale for latent tokens, s_a = q . k_a * scale for anchors, one softmax
+ *    over both, o = P_v sum_t p_t c_v,t + sum_a p_a v_a;
+ *  - the basis may be refreshed online by Oja's rule with periodic QR.
+ */
+#ifndef LRKV_H
+#define LRKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+enum {
+  LRKV_OK = 0,
+  LRKV_ERR_ARG = -1,         /* null pointer, bad size, misaligned pointer  */
+  LRKV_ERR_UNSUPPORTED = -2, /* head_dim != 128, rank not supported, ...    */
+  LRKV_ERR_CAPACITY = -3,    /* appended tokens would overflow the pages    */
+  LRKV_ERR_WORKSPACE = -4,   /* workspace smaller than the size query says  */
+  LRKV_ERR_CUDA = -5         /* a CUDA runtime call or launch failed        */
+};
+
+/* Element type of K/V inputs, codes, anchors, q and o. */
+enum { LRKV_BF16 = 0, LRKV_F32 = 1 };
+
+#define LRKV_HEAD_DIM 128
+#define LRKV_PAGE_TOKENS 64    /* tokens per latent code page */
+#define LRKV_FULL_RANK_TILE 32 /* tokens per full-rank anchor / dense tile */
+#define LRKV_MAX_BATCH 1024
+
+/* Chunk of a stored row: 16 bytes, i.e. CE = 8 bf16 or 4 fp32 elements.
+ *
+ * Latent code pool, chunk-major pages:
+ *   k_codes[num_pages][num_kv_heads][rank_k / CE][LRKV_PAGE_TOKENS][CE]
+ *   v_codes[num_pages][num_kv_heads][rank_v / CE][LRKV_PAGE_TOKENS][CE]
+ * Latent token j of sequence b (j-th token that left the window) lives in
+ * page block_table[b * max_pages_per_seq + j / 64], row j % 64.
+ *
+ * Anchors (full-rank sink + window ring), chunk-major tiles of 32 slots:
+ *   anchor_k[batch][num_kv_heads][anchor_tiles][128 / CE][32][CE]
+ * with anchor_tiles = ceil((n_sink + window) / 32).  Slot 0 holds the sink
+ * when n_sink == 1; token t >= n_sink of the window sits in slot
+ * n_sink + (t - n_sink) % window.  The valid slots of a sequence of L tokens
+ * are the first min(L, n_sink) + min(L - sink, window) slots.
+ *
+ * seq_len[b] counts the tokens appended to sequence b so far; the library
+ * advances it.  append_counter[b] is scratch the append kernels use to
+ * advance seq_len: zero it once when the cache is created; every completed
+ * lrkv_compress leaves it zero again. */
+typedef struct lrkv_cache {
+  int32_t batch;             /* B, 1..LRKV_MAX_BATCH                       */
+  int32_t num_kv_heads;      /* H_kv                                       */
+  int32_t head_dim;          /* must be 128                                */
+  int32_t rank_k, rank_v;    /* 8..128, multiples of CE                    */
+  int32_t dtype;             /* LRKV_BF16 or LRKV_F32                      */
+  int32_t n_sink;            /* 0 or 1                                     */
+  int32_t window;            /* W >= 0 full-rank recent tokens             */
+  int32_t num_pages;         /* pages in the code pools                    */
+  int32_t max_pages_per_seq; /* row length of block_table                  */
+  void *k_codes, *v_codes;   /* code pools, layout above                   */
+  const int32_t *block_table;/* [batch][max_pages_per_seq] page ids        */
+  void *anchor_k, *anchor_v; /* anchor tiles (may be NULL when n_sink+W==0)*/
+  int32_t *seq_len;          /* [batch] tokens appended so far             */
+  int32_t *append_counter;   /* [batch] zero-initialised scratch           */
+} lrkv_cache;
+
+/* Append new tokens to every sequence and compress the tokens that become
+ * latent ("store the small r-dim codes", Half the Memory, section 04;
+ * anchors and window: OjaKV article).
+ *   n_tokens : rows available per sequence in k and v.
+ *   n_new    : optional device [batch] counts; sequence b appends
+ *              min(n_new[b], n_tokens) tokens.  NULL: every sequence appends
+ *              n_tokens tokens.
+ *   k, v   : post-RoPE rows in the cache dtype; token i of (b, h) starts at
+ *            k + b*seq_stride + h*head_stride + i*128 (element strides).
+ *   P_k    : fp32 basis [Bp][H_kv][128][rank_k] (row-major 128 x r per head);
+ *            sequence b uses P_k + b*basis_batch_stride (0 = shared by all).
+ *   P_v    : the same for values with rank_v.
+ * The sink, window slots and codes of each sequence are written; seq_len is
+ * advanced by n_tokens.  Returns LRKV_ERR_CAPACITY only when the host can see
+ * the overflow (n_tokens larger than the page capacity); the kernels skip
+ * (and never write) code rows beyond max_pages_per_seq pages. */
+int lrkv_compress(const lrkv_cache *cache, const void *k, const void *v,
+                  int32_t n_tokens, const int32_t *n_new, int64_t seq_stride,
+                  int64_t head_stride,
+                  const float *P_k, const float *P_v,
+                  int64_t basis_batch_stride, void *stream);
+
+/* Bytes of workspace lrkv_decode_attn needs on the current device. */
+size_t lrkv_decode_workspace_bytes(const lrkv_cache *cache, int32_t num_q_heads);
+
+/* Decode attention of one query per q head over the latent cache plus the
+ * full-rank anchors (Half the Memory, section 08: attend directly against
+ * the codes; q folded as q~ = P_k^T q, o = P_v sum p c_v + sum p_a v_a).
+ *   q, o  : [batch][num_q_heads][128] in the cache dtype (q post-RoPE).
+ *           q head h reads KV head h / (num_q_heads / num_kv_heads).
+ *   scale : softmax scale applied to q . k (1/sqrt(128) for these models).
+ *   workspace : device scratch of at least lrkv_decode_workspace_bytes; its
+ *           first 4 bytes receive an error word (0 = ok, 1 = a bounded wait
+ *           timed out) that the caller may read after synchronising.
+ * A sequence with no tokens gets o = 0. */
+int lrkv_decode_attn(const lrkv_cache *cache, const void *q, int32_t num_q_heads,
+                     const float *P_k, const float *P_v,
+                     int64_t basis_batch_stride, float scale, void *o,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* Oja subspace update of S independent bases, in place (OjaKV article:
+ * online PCA with Oja's algorithm during prefill and periodically during
+ * decode).  For each token x of stream s in order: y = P^T x,
+ * P <- P + eta (x - P y) y^T; when (tokens_seen + i + 1) % qr_every == 0
+ * (qr_every > 0) P is replaced by the Q of its QR with diag(R) > 0.
+ *   P  : fp32 [S] bases of [128][rank], stream s at P + s*basis_stride.
+ *   x  : tokens of stream s at x + s*x_stream_stride + i*128, dtype x_dtype.
+ * tokens_seen is the host-side count of tokens this basis saw before. */
+int lrkv_oja_update(float *P, int32_t num_streams, int32_t rank,
+                    int64_t basis_stride, const void *x, int32_t x_dtype,
+                    int64_t x_stream_stride, int32_t n_tokens, float eta,
+                    int32_t qr_every, int64_t tokens_seen, void *stream);
+
+/* Replace each basis by the Q factor of its thin QR with diag(R) > 0. */
+int lrkv_qr_orthonormalize(float *P, int32_t num_streams, int32_t rank,
+                           int64_t basis_stride, void *stream);
+
+/* Dense full-rank paged KV cache: the baseline the latent cache replaces
+ * (Half the Memory, section 08 compares against the full cache).
+ *   k_pages[num_pages][num_kv_heads][128 / CE][32][CE] (chunk-major tiles),
+ *   token t of sequence b in page block_table[b*max_pages_per_seq + t/32]. */
+typedef struct lrkv_dense_cache {
+  int32_t batch, num_kv_heads, head_dim, dtype;
+  int32_t num_pages, max_pages_per_seq;
+  void *k_pages, *v_pages;
+  const int32_t *block_table;
+  int32_t *seq_len;
+  int32_t *append_counter; /* [batch] zero-initialised scratch */
+} lrkv_dense_cache;
+
+/* Append tokens to the dense cache (same k/v/n_new conventions as
+ * lrkv_compress) and advance seq_len. */
+int lrkv_dense_append(const lrkv_dense_cache *cache, const void *k,
+                      const void *v, int32_t n_tokens, const int32_t *n_new,
+                      int64_t seq_stride, int64_t head_stride, void *stream);
+size_t lrkv_dense_decode_workspace_bytes(const lrkv_dense_cache *cache,
+                                         int32_t num_q_heads);
+int lrkv_dense_decode_attn(const lrkv_dense_cache *cache, const void *q,
+                           int32_t num_q_heads, float scale, void *o,
+                           void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Static text for a status code. */
+const char *lrkv_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int lrkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LRKV_H */

@@ -1,0 +1,152 @@
+// Device helpers shared by the latent-KV kernels (sm_100a).
+//
+// Layouts (all caller-owned device memory):
+//  * Latent code pages, chunk-major: [page][kv head][r / CE][64 tokens][CE],
+//    where a chunk is 16 bytes (CE = 8 bf16 or 4 fp32 elements).  A page of
+//    one head is one contiguous slab, so one bulk copy moves it, and lane t
+//    reading chunk j of token t touches consecutive 16-byte words: no bank
+//    conflicts without a swizzle.
+//  * Full-rank tiles (anchors and the dense baseline) use the same
+//    chunk-major form with 32 tokens per tile: [tile][128 / CE][32][CE].
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lrkv.h"
+
+namespace lrkv {
+
+constexpr int kHeadDim = 128;
+constexpr int kLatPage = LRKV_PAGE_TOKENS;     // tokens per latent page
+constexpr int kFrTile = LRKV_FULL_RANK_TILE;   // tokens per full-rank tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Error word values written to the first 4 bytes of a decode workspace.
+constexpr int kErrNone = 0;
+constexpr int kErrTimeout = 1;
+constexpr int kErrBadPage = 2;
+
+template <typename T> struct Elem;
+template <> struct Elem<__nv_bfloat16> { static constexpr int CE = 8; };
+template <> struct Elem<float> { static constexpr int CE = 4; };
+
+// ------------------------------------------------------------ token split
+// Sequence of L tokens: the first min(L, n_sink) are the sink; of the rest
+// the most recent min(rest, W) form the window; the others are latent.
+struct Split {
+  int sink, win, lat;
+};
+__host__ __device__ inline Split split_tokens(int L, int n_sink, int W) {
+  Split s;
+  s.sink = L < n_sink ? L : n_sink;
+  int rest = L - s.sink;
+  s.win = rest < W ? rest : W;
+  s.lat = rest - s.win;
+  return s;
+}
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ inline uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ inline void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ inline void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ inline uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: gives up after ~timeout_ns and returns false.
+__device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                         uint64_t timeout_ns = 2000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 256; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > timeout_ns) return false;
+  }
+}
+// One bulk copy global -> shared completing on an mbarrier (no multicast).
+__device__ inline void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ------------------------------------------------------------ conversions
+// bf16 pair in one 32-bit word -> two floats (exact).
+__device__ inline float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ inline float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Unpack one 16-byte chunk into CE floats.
+template <typename T>
+__device__ inline void unpack_chunk(const uint4& c, float* f);
+template <>
+__device__ inline void unpack_chunk<__nv_bfloat16>(const uint4& c, float* f) {
+  f[0] = bf_lo(c.x); f[1] = bf_hi(c.x);
+  f[2] = bf_lo(c.y); f[3] = bf_hi(c.y);
+  f[4] = bf_lo(c.z); f[5] = bf_hi(c.z);
+  f[6] = bf_lo(c.w); f[7] = bf_hi(c.w);
+}
+template <>
+__device__ inline void unpack_chunk<float>(const uint4& c, float* f) {
+  f[0] = __uint_as_float(c.x); f[1] = __uint_as_float(c.y);
+  f[2] = __uint_as_float(c.z); f[3] = __uint_as_float(c.w);
+}
+
+template <typename T> __device__ inline float to_f(T x);
+template <> __device__ inline float to_f<float>(float x) { return x; }
+template <> __device__ inline float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T> __device__ inline T from_f(float x);
+template <> __device__ inline float from_f<float>(float x) { return x; }
+template <> __device__ inline __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ inline float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ inline float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Element offset of (chunk c, token row, elem e) inside one chunk-major slab.
+__host__ __device__ inline int64_t slab_off(int c, int row, int rows, int CE) {
+  return ((int64_t)c * rows + row) * CE;
+}
+
+}  // namespace lrkv

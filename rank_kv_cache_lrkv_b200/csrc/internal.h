@@ -1,0 +1,46 @@
+// Internal host-side launchers behind the C ABI (not exported).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lrkv.h"
+
+namespace lrkv {
+
+struct DecodeLaunch {
+  int B, H_kv, H_q, dtype;
+  const int* seq_len;
+  int n_sink, W;
+  const void *kc, *vc;
+  const int* bt_lat;
+  int maxp_lat, rk, rv, num_pages_lat;
+  const void *fk, *fv;
+  const int* bt_fr;
+  int maxp_fr, num_pages_fr;
+  const void* q;
+  const float *P_k, *P_v;
+  long long basis_bs;
+  float scale;
+  void* o;
+  void* ws;
+  size_t ws_bytes;
+};
+
+size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has_lat,
+                              bool has_fr, int dtype);
+int decode_launch(const DecodeLaunch& L, cudaStream_t st);
+
+int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, const int* n_new,
+                    long long seq_stride, long long head_stride, const float* P_k,
+                    const float* P_v, long long basis_bs, cudaStream_t st);
+int dense_append_launch(const lrkv_dense_cache& c, const void* k, const void* v, int n,
+                        const int* n_new,
+                        long long seq_stride, long long head_stride, cudaStream_t st);
+
+int oja_launch(float* P, int S, int r, long long basis_stride, const void* x, int x_dtype,
+               long long x_stride, int n, float eta, int qr_every, long long tokens_seen,
+               cudaStream_t st);
+int qr_launch(float* P, int S, int r, long long basis_stride, cudaStream_t st);
+
+}  // namespace lrkv

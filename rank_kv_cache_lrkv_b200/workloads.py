@@ -35,6 +35,7 @@ available; these seeded draws stand in for its activations.
 from __future__ import annotations
 
 import dataclasses
+import functools
 from typing import Optional
 
 import numpy as np
@@ -148,12 +149,25 @@ def spectrum(kind: str) -> np.ndarray:
     return np.exp(-i / (16.0 if kind == "k" else 8.0))
 
 
+@functools.lru_cache(maxsize=8)
+def _rope_table(n: int, theta: float):
+    half = HEAD_DIM // 2
+    inv_freq = theta ** (-np.arange(half, dtype=np.float64) * 2.0 / HEAD_DIM)
+    ang = np.arange(n, dtype=np.float64)[:, None] * inv_freq[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
 def rope_rotate(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
     """Rotate-half RoPE of rows of x [n, 128] at integer positions [n]."""
     half = HEAD_DIM // 2
-    inv_freq = theta ** (-np.arange(half, dtype=np.float64) * 2.0 / HEAD_DIM)
-    ang = positions.astype(np.float64)[:, None] * inv_freq[None, :]
-    cos, sin = np.cos(ang), np.sin(ang)
+    positions = np.asarray(positions)
+    if positions.ndim == 1 and len(positions) and np.array_equal(
+            positions, np.arange(len(positions))):
+        cos, sin = _rope_table(len(positions), float(theta))
+    else:
+        inv_freq = theta ** (-np.arange(half, dtype=np.float64) * 2.0 / HEAD_DIM)
+        ang = positions.astype(np.float64)[:, None] * inv_freq[None, :]
+        cos, sin = np.cos(ang), np.sin(ang)
     x1, x2 = x[:, :half], x[:, half:]
     return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=1)
 
@@ -238,12 +252,15 @@ def round_to(x: np.ndarray, dtype: str):
     return t, t.to(torch.float64).numpy()
 
 
-def layer_inputs(wl: Workload, layer: int = 0):
+def layer_inputs(wl: Workload, layer: int = 0, threads: Optional[int] = None):
     """All K/V streams of one layer, rounded to the workload dtype.
 
     Returns dict with torch CPU tensors K, V [B, H_kv, T + n_decode, 128] in
-    the workload dtype, and fp32 bases P_k [H_kv, 128, r_k], P_v.
+    the workload dtype, and fp32 bases P_k [H_kv, 128, r_k], P_v.  Streams are
+    drawn in parallel threads; each stream's values depend only on its seed.
     """
+    import concurrent.futures
+    import os
     import torch
     total = wl.T + wl.n_decode
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -251,13 +268,24 @@ def layer_inputs(wl: Workload, layer: int = 0):
     V = torch.empty_like(K)
     Pk = np.empty((wl.H_kv, HEAD_DIM, wl.r_k), np.float32)
     Pv = np.empty((wl.H_kv, HEAD_DIM, wl.r_v), np.float32)
-    for h in range(wl.H_kv):
-        Qk, Qv = head_q(wl, "k", layer, h), head_q(wl, "v", layer, h)
-        for b in range(wl.B):
-            K[b, h] = round_to(stream(wl, "k", layer, b, h, Q=Qk), wl.dtype)[0]
-            V[b, h] = round_to(stream(wl, "v", layer, b, h, Q=Qv), wl.dtype)[0]
+    Qs = {(kind, h): head_q(wl, kind, layer, h) for kind in "kv" for h in range(wl.H_kv)}
+    if wl.rope_theta is not None:
+        _rope_table(total, float(wl.rope_theta))
+
+    def one(job):
+        kind, b, h = job
+        dst = K if kind == "k" else V
+        dst[b, h] = round_to(stream(wl, kind, layer, b, h, Q=Qs[(kind, h)]), wl.dtype)[0]
+
+    def bases(h):
         Pk[h] = basis(wl, "k", layer, h)
         Pv[h] = basis(wl, "v", layer, h)
+
+    jobs = [(kind, b, h) for kind in "kv" for b in range(wl.B) for h in range(wl.H_kv)]
+    n = threads or min(16, os.cpu_count() or 4)
+    with concurrent.futures.ThreadPoolExecutor(n) as ex:
+        list(ex.map(one, jobs))
+        list(ex.map(bases, range(wl.H_kv)))
     return {"K": K, "V": V, "P_k": torch.from_numpy(Pk), "P_v": torch.from_numpy(Pv)}
 
 

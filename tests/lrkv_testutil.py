@@ -1,0 +1,127 @@
+"""Helpers shared by the GPU parity tests: run a workload through the C ABI
+and through the oracle on the same seeded inputs, read stored codes back
+from the page layout, and compare outputs."""
+import numpy as np
+import torch
+
+from oracle import lrkv_oracle as orc
+from rank_kv_cache_lrkv_b200 import workloads as wk
+
+D = 128
+
+
+def row_rel_err(o, ref) -> float:
+    """max over rows (b, h) of ||o - ref||_inf / ||ref||_inf."""
+    o = np.asarray(o, np.float64).reshape(-1, D)
+    ref = np.asarray(ref, np.float64).reshape(-1, D)
+    den = np.maximum(np.max(np.abs(ref), axis=1), 1e-30)
+    return float(np.max(np.max(np.abs(o - ref), axis=1) / den))
+
+
+def torch_dtype(wl):
+    return torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+
+def gather_codes(cache, b, kvh, n, kind="k"):
+    """Codes of latent tokens 0..n-1 of (b, kvh) as float64 [n, r]."""
+    pool = cache.k_codes if kind == "k" else cache.v_codes
+    r = cache.r_k if kind == "k" else cache.r_v
+    bt = cache.block_table[b].long().cpu()
+    j = torch.arange(n)
+    pages = bt[j // 64]
+    rows = j % 64
+    x = pool[pages.to(pool.device), kvh, :, rows.to(pool.device), :]  # [n, r/CE, CE]
+    return x.reshape(n, r).double().cpu().numpy()
+
+
+def gather_anchor_slots(cache, b, kvh, slots, kind="k"):
+    pool = cache.anchor_k if kind == "k" else cache.anchor_v
+    s = torch.as_tensor(slots, dtype=torch.long)
+    x = pool[b, kvh, (s // 32).to(pool.device), :, (s % 32).to(pool.device), :]
+    return x.reshape(len(slots), D).double().cpu().numpy()
+
+
+def window_slots(L, n_sink, W):
+    """GPU slots of the oracle's anchors in its order (sink, then window
+    oldest first) for a sequence of L tokens."""
+    sink, _, win = orc.partition(L, n_sink, W)
+    return list(sink) + [n_sink + (t - n_sink) % W for t in win]
+
+
+class Inputs:
+    """Rounded inputs of one layer of a workload, on CPU."""
+
+    def __init__(self, wl, layer=0):
+        d = wk.layer_inputs(wl, layer)
+        self.K, self.V = d["K"], d["V"]
+        self.Pk, self.Pv = d["P_k"], d["P_v"]
+        self.q = wk.layer_queries(wl, layer)
+
+
+def run_gpu(wl, inp, n_steps=None, page_perm=None, lrkv=None, prefill_chunks=None):
+    """Prefill + decode steps through the C ABI; returns (cache, [o per step])."""
+    n_steps = wl.n_decode if n_steps is None else n_steps
+    dt = torch_dtype(wl)
+    cache = lrkv.LatentCache(wl.B, wl.H_kv, wl.r_k, wl.r_v, wl.T + n_steps, wl.n_sink,
+                             wl.window, dtype=dt, page_perm=page_perm)
+    K, V = inp.K.cuda(), inp.V.cuda()
+    Pk, Pv = inp.Pk.cuda(), inp.Pv.cuda()
+    chunks = prefill_chunks or [wl.T]
+    pos = 0
+    for n in chunks:
+        lrkv.compress(cache, K[:, :, pos:pos + n], V[:, :, pos:pos + n], Pk, Pv)
+        pos += n
+    assert pos == wl.T
+    ws = lrkv.decode_workspace(cache, wl.H_q)
+    outs = []
+    for s in range(n_steps):
+        if wl.append_before_attend:
+            t = wl.T + s
+            lrkv.compress(cache, K[:, :, t:t + 1], V[:, :, t:t + 1], Pk, Pv)
+        q = inp.q[s].cuda().contiguous()
+        o = torch.empty_like(q)
+        lrkv.decode_attn(cache, q, Pk, Pv, wl.scale, o, ws)
+        outs.append(o.double().cpu().numpy())
+    torch.cuda.synchronize()
+    assert lrkv.workspace_error(ws) == 0
+    return cache, outs
+
+
+def run_oracle(wl, inp, n_steps=None, units=None):
+    """The same schedule in the float64 oracle.  units: optional list of
+    (b, kvh) pairs; then only those units are simulated (each as its own
+    single-sequence, single-head cache) and outputs are returned per unit as
+    {(b, kvh): [o [G, 128] per step]}."""
+    n_steps = wl.n_decode if n_steps is None else n_steps
+    G = wl.G
+    if units is None:
+        K = inp.K.double().numpy()
+        V = inp.V.double().numpy()
+        Pk = inp.Pk.double().numpy()[None]
+        Pv = inp.Pv.double().numpy()[None]
+        oc = orc.LatentCacheOracle(wl.B, wl.H_kv, wl.r_k, wl.r_v, wl.n_sink, wl.window)
+        oc.append(K[:, :, :wl.T], V[:, :, :wl.T], Pk, Pv)
+        outs = []
+        for s in range(n_steps):
+            if wl.append_before_attend:
+                t = wl.T + s
+                oc.append(K[:, :, t:t + 1], V[:, :, t:t + 1], Pk, Pv)
+            outs.append(oc.attend(inp.q[s].double().numpy(), Pk, Pv, wl.scale))
+        return oc, outs
+    res = {}
+    for (b, h) in units:
+        K = inp.K[b:b + 1, h:h + 1].double().numpy()
+        V = inp.V[b:b + 1, h:h + 1].double().numpy()
+        Pk = inp.Pk[h:h + 1].double().numpy()[None]
+        Pv = inp.Pv[h:h + 1].double().numpy()[None]
+        oc = orc.LatentCacheOracle(1, 1, wl.r_k, wl.r_v, wl.n_sink, wl.window)
+        oc.append(K[:, :, :wl.T], V[:, :, :wl.T], Pk, Pv)
+        outs = []
+        for s in range(n_steps):
+            if wl.append_before_attend:
+                t = wl.T + s
+                oc.append(K[:, :, t:t + 1], V[:, :, t:t + 1], Pk, Pv)
+            q = inp.q[s][b:b + 1, h * G:(h + 1) * G].double().numpy()
+            outs.append(oc.attend(q, Pk, Pv, wl.scale)[0])
+        res[(b, h)] = (oc, outs)
+    return res
