@@ -40,6 +40,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="llama32k", choices=["llama32k", "qwen8k"])
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--context", type=int, default=0,
+                   help="override the prompt length (small cases for profiler captures)")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
@@ -201,6 +203,8 @@ def run_ours(args, rank, world):
     from rank_kv_cache_lrkv_b200 import workloads as wk
 
     base = workload(args.workload)
+    if args.context:
+        base = base.with_(T=args.context)
     W, K = args.warmup, args.steps
     E = 0 if args.no_e2e else min(K, 64)
     wl = base.with_(n_decode=W + K + E + 2)

@@ -53,15 +53,20 @@ enum { LRKV_BF16 = 0, LRKV_F32 = 1 };
 #define LRKV_MAX_BATCH 1024
 
 /* Chunk of a stored row: 16 bytes, i.e. CE = 8 bf16 or 4 fp32 elements.
+ * Every stored block is chunk-major: for each 16-byte chunk index, the
+ * chunks of all tokens of the block follow each other, so one bulk copy
+ * moves a block and lane t reading chunk j of token t touches consecutive
+ * 16-byte words.
  *
- * Latent code pool, chunk-major pages:
- *   k_codes[num_pages][num_kv_heads][rank_k / CE][LRKV_PAGE_TOKENS][CE]
- *   v_codes[num_pages][num_kv_heads][rank_v / CE][LRKV_PAGE_TOKENS][CE]
- * Latent token j of sequence b (j-th token that left the window) lives in
- * page block_table[b * max_pages_per_seq + j / 64], row j % 64.
+ * Latent code pool, one slab per (page, KV head) holding the key codes'
+ * chunks first, then the value codes' chunks:
+ *   codes[num_pages][num_kv_heads][(rank_k + rank_v) / CE][LRKV_PAGE_TOKENS][CE]
+ * Latent token j of sequence b (the j-th token that left the window) lives
+ * in page block_table[b * max_pages_per_seq + j / 64], row j % 64.
  *
- * Anchors (full-rank sink + window ring), chunk-major tiles of 32 slots:
- *   anchor_k[batch][num_kv_heads][anchor_tiles][128 / CE][32][CE]
+ * Anchors (full-rank sink + window ring), chunk-major tiles of 32 slots with
+ * the key's 128 dims first, then the value's:
+ *   anchors[batch][num_kv_heads][anchor_tiles][256 / CE][32][CE]
  * with anchor_tiles = ceil((n_sink + window) / 32).  Slot 0 holds the sink
  * when n_sink == 1; token t >= n_sink of the window sits in slot
  * n_sink + (t - n_sink) % window.  The valid slots of a sequence of L tokens
@@ -79,11 +84,11 @@ typedef struct lrkv_cache {
   int32_t dtype;             /* LRKV_BF16 or LRKV_F32                      */
   int32_t n_sink;            /* 0 or 1                                     */
   int32_t window;            /* W >= 0 full-rank recent tokens             */
-  int32_t num_pages;         /* pages in the code pools                    */
+  int32_t num_pages;         /* pages in the code pool                     */
   int32_t max_pages_per_seq; /* row length of block_table                  */
-  void *k_codes, *v_codes;   /* code pools, layout above                   */
+  void *codes;               /* code pool, layout above                    */
   const int32_t *block_table;/* [batch][max_pages_per_seq] page ids        */
-  void *anchor_k, *anchor_v; /* anchor tiles (may be NULL when n_sink+W==0)*/
+  void *anchors;             /* anchor tiles (may be NULL when n_sink+W==0)*/
   int32_t *seq_len;          /* [batch] tokens appended so far             */
   int32_t *append_counter;   /* [batch] zero-initialised scratch           */
 } lrkv_cache;
@@ -110,18 +115,25 @@ int lrkv_compress(const lrkv_cache *cache, const void *k, const void *v,
                   const float *P_k, const float *P_v,
                   int64_t basis_batch_stride, void *stream);
 
-/* Bytes of workspace lrkv_decode_attn needs on the current device. */
+/* Bytes of workspace lrkv_decode_attn needs on the current device.  The
+ * workspace must be zero-filled once when it is allocated: it holds per-
+ * (sequence, KV head) tile counters that every completed call leaves at
+ * zero, split-K partial records, and (first 4 bytes) an error word. */
 size_t lrkv_decode_workspace_bytes(const lrkv_cache *cache, int32_t num_q_heads);
 
 /* Decode attention of one query per q head over the latent cache plus the
  * full-rank anchors (Half the Memory, section 08: attend directly against
  * the codes; q folded as q~ = P_k^T q, o = P_v sum p c_v + sum p_a v_a).
+ * One kernel launch.
  *   q, o  : [batch][num_q_heads][128] in the cache dtype (q post-RoPE).
  *           q head h reads KV head h / (num_q_heads / num_kv_heads).
  *   scale : softmax scale applied to q . k (1/sqrt(128) for these models).
- *   workspace : device scratch of at least lrkv_decode_workspace_bytes; its
- *           first 4 bytes receive an error word (0 = ok, 1 = a bounded wait
- *           timed out) that the caller may read after synchronising.
+ *   workspace : zero-filled once (see above), at least
+ *           lrkv_decode_workspace_bytes; calls sharing a workspace must be
+ *           stream-ordered.  The error word is set (1 = a bounded wait timed
+ *           out, 2 = a block-table entry out of range) and never cleared by
+ *           the library; after a nonzero error word, zero the workspace
+ *           again before reusing it.
  * A sequence with no tokens gets o = 0. */
 int lrkv_decode_attn(const lrkv_cache *cache, const void *q, int32_t num_q_heads,
                      const float *P_k, const float *P_v,
@@ -146,13 +158,14 @@ int lrkv_qr_orthonormalize(float *P, int32_t num_streams, int32_t rank,
                            int64_t basis_stride, void *stream);
 
 /* Dense full-rank paged KV cache: the baseline the latent cache replaces
- * (Half the Memory, section 08 compares against the full cache).
- *   k_pages[num_pages][num_kv_heads][128 / CE][32][CE] (chunk-major tiles),
+ * (Half the Memory, section 08 compares against the full cache).  One slab
+ * per (page, KV head), key chunks then value chunks:
+ *   kv_pages[num_pages][num_kv_heads][256 / CE][32][CE] (chunk-major),
  *   token t of sequence b in page block_table[b*max_pages_per_seq + t/32]. */
 typedef struct lrkv_dense_cache {
   int32_t batch, num_kv_heads, head_dim, dtype;
   int32_t num_pages, max_pages_per_seq;
-  void *k_pages, *v_pages;
+  void *kv_pages;
   const int32_t *block_table;
   int32_t *seq_len;
   int32_t *append_counter; /* [batch] zero-initialised scratch */
@@ -163,6 +176,7 @@ typedef struct lrkv_dense_cache {
 int lrkv_dense_append(const lrkv_dense_cache *cache, const void *k,
                       const void *v, int32_t n_tokens, const int32_t *n_new,
                       int64_t seq_stride, int64_t head_stride, void *stream);
+/* Workspace of the dense decode; the same zero-once contract as above. */
 size_t lrkv_dense_decode_workspace_bytes(const lrkv_dense_cache *cache,
                                          int32_t num_q_heads);
 int lrkv_dense_decode_attn(const lrkv_dense_cache *cache, const void *q,

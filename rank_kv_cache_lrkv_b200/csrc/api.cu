@@ -27,13 +27,9 @@ int check_cache(const lrkv_cache* c) {
   if (rc != LRKV_OK) return rc;
   if (c->n_sink < 0 || c->n_sink > 1 || c->window < 0 || c->window > (1 << 20)) return LRKV_ERR_ARG;
   if (c->num_pages < 1 || c->max_pages_per_seq < 1) return LRKV_ERR_ARG;
-  if (!c->k_codes || !c->v_codes || !c->block_table || !c->seq_len || !c->append_counter)
-    return LRKV_ERR_ARG;
-  if (!aligned16(c->k_codes) || !aligned16(c->v_codes)) return LRKV_ERR_ARG;
-  if (c->n_sink + c->window > 0) {
-    if (!c->anchor_k || !c->anchor_v) return LRKV_ERR_ARG;
-    if (!aligned16(c->anchor_k) || !aligned16(c->anchor_v)) return LRKV_ERR_ARG;
-  }
+  if (!c->codes || !c->block_table || !c->seq_len || !c->append_counter) return LRKV_ERR_ARG;
+  if (!aligned16(c->codes)) return LRKV_ERR_ARG;
+  if (c->n_sink + c->window > 0 && (!c->anchors || !aligned16(c->anchors))) return LRKV_ERR_ARG;
   return LRKV_OK;
 }
 
@@ -43,9 +39,8 @@ int check_dense(const lrkv_dense_cache* c) {
   if (c->head_dim != kHeadDim) return LRKV_ERR_UNSUPPORTED;
   if (c->batch < 1 || c->batch > LRKV_MAX_BATCH || c->num_kv_heads < 1) return LRKV_ERR_ARG;
   if (c->num_pages < 1 || c->max_pages_per_seq < 1) return LRKV_ERR_ARG;
-  if (!c->k_pages || !c->v_pages || !c->block_table || !c->seq_len || !c->append_counter)
-    return LRKV_ERR_ARG;
-  if (!aligned16(c->k_pages) || !aligned16(c->v_pages)) return LRKV_ERR_ARG;
+  if (!c->kv_pages || !c->block_table || !c->seq_len || !c->append_counter) return LRKV_ERR_ARG;
+  if (!aligned16(c->kv_pages)) return LRKV_ERR_ARG;
   return LRKV_OK;
 }
 
@@ -108,12 +103,11 @@ int lrkv_decode_attn(const lrkv_cache* cache, const void* q, int32_t num_q_heads
   DecodeLaunch L;
   L.B = cache->batch; L.H_kv = cache->num_kv_heads; L.H_q = num_q_heads; L.dtype = cache->dtype;
   L.seq_len = cache->seq_len; L.n_sink = cache->n_sink; L.W = cache->window;
-  L.kc = cache->k_codes; L.vc = cache->v_codes; L.bt_lat = cache->block_table;
+  L.codes = cache->codes; L.bt_lat = cache->block_table;
   L.maxp_lat = cache->max_pages_per_seq; L.rk = cache->rank_k; L.rv = cache->rank_v;
   L.num_pages_lat = cache->num_pages;
   const bool has_fr = cache->n_sink + cache->window > 0;
-  L.fk = has_fr ? cache->anchor_k : nullptr;
-  L.fv = has_fr ? cache->anchor_v : nullptr;
+  L.fr = has_fr ? cache->anchors : nullptr;
   L.bt_fr = nullptr;
   L.maxp_fr = (cache->n_sink + cache->window + kFrTile - 1) / kFrTile;
   L.num_pages_fr = 0;
@@ -174,9 +168,9 @@ int lrkv_dense_decode_attn(const lrkv_dense_cache* cache, const void* q, int32_t
   DecodeLaunch L;
   L.B = cache->batch; L.H_kv = cache->num_kv_heads; L.H_q = num_q_heads; L.dtype = cache->dtype;
   L.seq_len = cache->seq_len; L.n_sink = 0; L.W = INT_MAX;
-  L.kc = nullptr; L.vc = nullptr; L.bt_lat = nullptr; L.maxp_lat = 0; L.rk = 0; L.rv = 0;
+  L.codes = nullptr; L.bt_lat = nullptr; L.maxp_lat = 0; L.rk = 0; L.rv = 0;
   L.num_pages_lat = 0;
-  L.fk = cache->k_pages; L.fv = cache->v_pages; L.bt_fr = cache->block_table;
+  L.fr = cache->kv_pages; L.bt_fr = cache->block_table;
   L.maxp_fr = cache->max_pages_per_seq; L.num_pages_fr = cache->num_pages;
   L.q = q; L.P_k = nullptr; L.P_v = nullptr; L.basis_bs = 0; L.scale = scale;
   L.o = o; L.ws = workspace; L.ws_bytes = workspace_bytes;

@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "lrkv.h"
 
@@ -92,6 +93,21 @@ __device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
     if (global_ns() - t0 > timeout_ns) return false;
   }
 }
+// L2 policy for data read once: evict first, so small hot data stays in L2.
+__device__ inline uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// Bulk copy with an L2 cache-policy hint.
+__device__ inline void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                     uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
 // One bulk copy global -> shared completing on an mbarrier (no multicast).
 __device__ inline void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -131,6 +147,35 @@ template <typename T> __device__ inline T from_f(float x);
 template <> __device__ inline float from_f<float>(float x) { return x; }
 template <> __device__ inline __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// ------------------------------------------------------------ packed fp32
+// d += a * b on two fp32 lanes at once (sm_100 packed FMA).
+__device__ __forceinline__ void fma2(float2& d, const float2 a, const float2 b) {
+  unsigned long long dd, aa, bb;
+  memcpy(&dd, &d, 8); memcpy(&aa, &a, 8); memcpy(&bb, &b, 8);
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(dd) : "l"(aa), "l"(bb));
+  memcpy(&d, &dd, 8);
+}
+__device__ __forceinline__ float2 mul2(const float2 a, const float2 b) {
+  unsigned long long dd, aa, bb;
+  memcpy(&aa, &a, 8); memcpy(&bb, &b, 8);
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(dd) : "l"(aa), "l"(bb));
+  float2 d;
+  memcpy(&d, &dd, 8);
+  return d;
+}
+// bf16 pair word -> (even, odd) floats as one packed pair.
+__device__ __forceinline__ float2 bf2(uint32_t w) { return make_float2(bf_lo(w), bf_hi(w)); }
+
+// Programmatic dependent launch controls.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Named barrier over `threads` threads (ids 1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ inline float warp_max(float v) {

@@ -31,7 +31,7 @@ __device__ inline int appended(const int* n_new, int n, int b) {
 
 struct AppendArgs {
   int B, H_kv, rk, rv, n_sink, W, maxp, num_pages, n, anchor_tiles;
-  void *kc, *vc, *ak, *av;
+  void *codes, *anchors;
   const int* bt;
   int* seq_len;
   int* counter;
@@ -42,68 +42,87 @@ struct AppendArgs {
   long long basis_bs;
 };
 
-// Element offset of (slot, dim d) in the anchor tiles of unit (b, kvh).
+// Element offset of (slot, dim d) of the key (isv = 0) or value (isv = 1)
+// in the anchor tiles of unit (b, kvh).
 template <typename T>
-__device__ inline size_t anchor_off(const AppendArgs& a, int b, int kvh, int slot, int d) {
+__device__ inline size_t anchor_off(const AppendArgs& a, int b, int kvh, int slot, int d, int isv) {
   constexpr int CE = Elem<T>::CE;
-  size_t tile = ((size_t)b * a.H_kv + kvh) * a.anchor_tiles + slot / kFrTile;
-  return (tile * (kHeadDim / CE) + d / CE) * kFrTile * CE + (slot % kFrTile) * CE + d % CE;
+  const size_t tile = ((size_t)b * a.H_kv + kvh) * a.anchor_tiles + slot / kFrTile;
+  const int chunk = isv * (kHeadDim / CE) + d / CE;
+  return (tile * (2 * kHeadDim / CE) + chunk) * kFrTile * CE + (slot % kFrTile) * CE + d % CE;
 }
 
-// Element offset of (latent index j, code dim jj) in a code pool; -1 if the
-// page is out of range.
+// Element offset of (latent index j, code dim jj) of the key (isv = 0) or
+// value (isv = 1) codes in the code pool; -1 if the page is out of range.
 template <typename T>
-__device__ inline long long code_off(const AppendArgs& a, int b, int kvh, int j, int jj, int r) {
+__device__ inline long long code_off(const AppendArgs& a, int b, int kvh, int j, int jj, int isv) {
   constexpr int CE = Elem<T>::CE;
-  int pi = j / kLatPage;
+  const int pi = j / kLatPage;
   if (pi >= a.maxp) return -1;
-  int page = a.bt[(size_t)b * a.maxp + pi];
+  const int page = a.bt[(size_t)b * a.maxp + pi];
   if (page < 0 || page >= a.num_pages) return -1;
-  return ((((long long)page * a.H_kv + kvh) * (r / CE) + jj / CE) * kLatPage + j % kLatPage) * CE +
+  const int nch = (a.rk + a.rv) / CE;
+  const int chunk = isv * (a.rk / CE) + jj / CE;
+  return ((((long long)page * a.H_kv + kvh) * nch + chunk) * kLatPage + j % kLatPage) * CE +
          jj % CE;
 }
 
-// codes of one token held in shared memory (xk, xv fp32) -> pages.
+// Codes of one token held in shared memory (xk, xv fp32) -> pages.  The
+// 128-long dot products are split over 4 row segments so every thread has
+// independent loads in flight; red holds [4][r_k + r_v] partial sums.
+constexpr int kSeg = 4;
 template <typename T>
 __device__ void project_one(const AppendArgs& a, int b, int kvh, int j, const float* xk,
-                            const float* xv) {
+                            const float* xv, float* red) {
   const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
   const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
-  for (int o = threadIdx.x; o < a.rk + a.rv; o += blockDim.x) {
+  const int NJ = a.rk + a.rv;
+  constexpr int rows = kHeadDim / kSeg;
+  for (int task = threadIdx.x; task < kSeg * NJ; task += blockDim.x) {
+    const int seg = task / NJ, o = task - seg * NJ;
     const bool isk = o < a.rk;
     const int jj = isk ? o : o - a.rk;
     const int r = isk ? a.rk : a.rv;
-    const float* P = isk ? Pk : Pv;
-    const float* x = isk ? xk : xv;
+    const float* P = (isk ? Pk : Pv) + (size_t)seg * rows * r + jj;
+    const float* x = (isk ? xk : xv) + seg * rows;
     float s = 0.f;
 #pragma unroll 8
-    for (int i = 0; i < kHeadDim; ++i) s = fmaf(P[(size_t)i * r + jj], x[i], s);
-    long long off = code_off<T>(a, b, kvh, j, jj, r);
-    if (off >= 0) static_cast<T*>(isk ? a.kc : a.vc)[off] = from_f<T>(s);
+    for (int i = 0; i < rows; ++i) s = fmaf(P[(size_t)i * r], x[i], s);
+    red[seg * NJ + o] = s;
+  }
+  __syncthreads();
+  for (int o = threadIdx.x; o < NJ; o += blockDim.x) {
+    float s = 0.f;
+#pragma unroll
+    for (int seg = 0; seg < kSeg; ++seg) s += red[seg * NJ + o];
+    const bool isk = o < a.rk;
+    const int jj = isk ? o : o - a.rk;
+    const long long off = code_off<T>(a, b, kvh, j, jj, isk ? 0 : 1);
+    if (off >= 0) static_cast<T*>(a.codes)[off] = from_f<T>(s);
   }
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_latent) {
   __shared__ float xk[kHeadDim], xv[kHeadDim];
+  __shared__ float red[kSeg * 2 * kHeadDim];
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int L0 = a.seq_len[b], L1 = L0 + appended(a.n_new, a.n, b);
   const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
   const T* kin = static_cast<const T*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
   const T* vin = static_cast<const T*>(a.v) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
-  const T* ak = static_cast<const T*>(a.ak);
-  const T* av = static_cast<const T*>(a.av);
+  const T* anc = static_cast<const T*>(a.anchors);
 
   // 1. evictions from the ring (token index < L0), oldest first.
   const int ev_lo = a.n_sink + s0.lat, ev_hi = min(L0, a.n_sink + s1.lat);
   for (int t = ev_lo; t < ev_hi; ++t) {
     const int slot = a.n_sink + (t - a.n_sink) % a.W;
     for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x) {
-      xk[d] = to_f<T>(ak[anchor_off<T>(a, b, kvh, slot, d)]);
-      xv[d] = to_f<T>(av[anchor_off<T>(a, b, kvh, slot, d)]);
+      xk[d] = to_f<T>(anc[anchor_off<T>(a, b, kvh, slot, d, 0)]);
+      xv[d] = to_f<T>(anc[anchor_off<T>(a, b, kvh, slot, d, 1)]);
     }
     __syncthreads();
-    project_one<T>(a, b, kvh, t - a.n_sink, xk, xv);
+    project_one<T>(a, b, kvh, t - a.n_sink, xk, xv, red);
     __syncthreads();
   }
   // 2. input tokens that go straight to latent (small n only).
@@ -115,14 +134,13 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
         xv[d] = to_f<T>(vin[(size_t)(t - L0) * kHeadDim + d]);
       }
       __syncthreads();
-      project_one<T>(a, b, kvh, t - a.n_sink, xk, xv);
+      project_one<T>(a, b, kvh, t - a.n_sink, xk, xv, red);
       __syncthreads();
     }
   }
   // 3. sink and window writes (full-rank, verbatim).
   if (a.n_sink + a.W > 0) {
-    T* akw = static_cast<T*>(a.ak);
-    T* avw = static_cast<T*>(a.av);
+    T* ancw = static_cast<T*>(a.anchors);
     const int w_lo = max(L0, max(a.n_sink, L1 - a.W));
     // sink first (t < n_sink), then the window tokens [w_lo, L1)
     const int n_sink_new = max(0, min(a.n_sink, L1) - L0);
@@ -133,9 +151,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
       int t, slot;
       if (q < n_sink_new) { t = L0 + q; slot = t; }
       else { t = w_lo + (q - n_sink_new); slot = a.n_sink + (t - a.n_sink) % a.W; }
-      const size_t off = anchor_off<T>(a, b, kvh, slot, d);
-      akw[off] = kin[(size_t)(t - L0) * kHeadDim + d];
-      avw[off] = vin[(size_t)(t - L0) * kHeadDim + d];
+      ancw[anchor_off<T>(a, b, kvh, slot, d, 0)] = kin[(size_t)(t - L0) * kHeadDim + d];
+      ancw[anchor_off<T>(a, b, kvh, slot, d, 1)] = vin[(size_t)(t - L0) * kHeadDim + d];
     }
   }
   // 4. the last CTA of this sequence advances seq_len.
@@ -174,14 +191,14 @@ __global__ void __launch_bounds__(256) bulk_compress_kernel(AppendArgs a) {
     const int r = pass == 0 ? a.rk : a.rv;
     const float* P = (pass == 0 ? a.P_k : a.P_v) + (size_t)b * a.basis_bs +
                      (size_t)kvh * kHeadDim * r;
-    T* dst = static_cast<T*>(pass == 0 ? a.kc : a.vc);
+    T* dst = static_cast<T*>(a.codes);
     for (int o = threadIdx.x; o < rows * r; o += blockDim.x) {
       const int rr = o / r, jj = o - rr * r;
       float s = 0.f;
 #pragma unroll 8
       for (int i = 0; i < kHeadDim; ++i) s = fmaf(P[(size_t)i * r + jj], xs[rr][i], s);
       const int j = L0 + r0 + rr - a.n_sink;  // latent index
-      long long off = code_off<T>(a, b, kvh, j, jj, r);
+      long long off = code_off<T>(a, b, kvh, j, jj, pass);
       if (off >= 0) dst[off] = from_f<T>(s);
     }
     __syncthreads();
@@ -208,7 +225,7 @@ int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, co
   a.B = c.batch; a.H_kv = c.num_kv_heads; a.rk = c.rank_k; a.rv = c.rank_v;
   a.n_sink = c.n_sink; a.W = c.window; a.maxp = c.max_pages_per_seq; a.num_pages = c.num_pages;
   a.n = n; a.anchor_tiles = (c.n_sink + c.window + kFrTile - 1) / kFrTile;
-  a.kc = c.k_codes; a.vc = c.v_codes; a.ak = c.anchor_k; a.av = c.anchor_v;
+  a.codes = c.codes; a.anchors = c.anchors;
   a.bt = c.block_table; a.seq_len = c.seq_len; a.counter = c.append_counter; a.n_new = n_new;
   a.k = k; a.v = v; a.seq_stride = seq_stride; a.head_stride = head_stride;
   a.P_k = P_k; a.P_v = P_v; a.basis_bs = basis_bs;
@@ -218,7 +235,7 @@ int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, co
 // ------------------------------------------------------------ dense baseline
 struct DenseAppendArgs {
   int B, H_kv, maxp, num_pages, n;
-  void *kp, *vp;
+  void* kvp;
   const int* bt;
   int* seq_len;
   int* counter;
@@ -234,18 +251,17 @@ __global__ void __launch_bounds__(256) dense_append_kernel(DenseAppendArgs a) {
   const int L0 = a.seq_len[b], nb = appended(a.n_new, a.n, b);
   const T* kin = static_cast<const T*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
   const T* vin = static_cast<const T*>(a.v) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
-  T* kp = static_cast<T*>(a.kp);
-  T* vp = static_cast<T*>(a.vp);
+  T* kvp = static_cast<T*>(a.kvp);
   for (int x = threadIdx.x; x < nb * kHeadDim; x += blockDim.x) {
     const int q = x / kHeadDim, d = x - q * kHeadDim;
     const int t = L0 + q, pi = t / kFrTile;
     if (pi >= a.maxp) continue;
     const int page = a.bt[(size_t)b * a.maxp + pi];
     if (page < 0 || page >= a.num_pages) continue;
-    const size_t off = (((size_t)page * a.H_kv + kvh) * (kHeadDim / CE) + d / CE) * kFrTile * CE +
-                       (t % kFrTile) * CE + d % CE;
-    kp[off] = kin[(size_t)q * kHeadDim + d];
-    vp[off] = vin[(size_t)q * kHeadDim + d];
+    const size_t slab = ((size_t)page * a.H_kv + kvh) * (2 * kHeadDim / CE);
+    const size_t row = (size_t)(t % kFrTile) * CE + d % CE;
+    kvp[(slab + d / CE) * kFrTile * CE + row] = kin[(size_t)q * kHeadDim + d];
+    kvp[(slab + kHeadDim / CE + d / CE) * kFrTile * CE + row] = vin[(size_t)q * kHeadDim + d];
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -263,7 +279,7 @@ int dense_append_launch(const lrkv_dense_cache& c, const void* k, const void* v,
                         const int* n_new, long long seq_stride, long long head_stride, cudaStream_t st) {
   DenseAppendArgs a;
   a.B = c.batch; a.H_kv = c.num_kv_heads; a.maxp = c.max_pages_per_seq;
-  a.num_pages = c.num_pages; a.n = n; a.kp = c.k_pages; a.vp = c.v_pages;
+  a.num_pages = c.num_pages; a.n = n; a.kvp = c.kv_pages;
   a.bt = c.block_table; a.seq_len = c.seq_len; a.counter = c.append_counter; a.n_new = n_new;
   a.k = k; a.v = v; a.seq_stride = seq_stride; a.head_stride = head_stride;
   dim3 g(a.H_kv, a.B);

@@ -12,10 +12,10 @@ struct DecodeLaunch {
   int B, H_kv, H_q, dtype;
   const int* seq_len;
   int n_sink, W;
-  const void *kc, *vc;
+  const void* codes;  // latent slabs (nullptr: no latent space)
   const int* bt_lat;
   int maxp_lat, rk, rv, num_pages_lat;
-  const void *fk, *fv;
+  const void* fr;     // full-rank tiles (nullptr: no full-rank space)
   const int* bt_fr;
   int maxp_fr, num_pages_fr;
   const void* q;

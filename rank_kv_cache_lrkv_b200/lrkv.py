@@ -38,9 +38,8 @@ class CacheDesc(ctypes.Structure):
                 ("rank_v", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("n_sink", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
-                ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
-                ("block_table", ctypes.c_void_p), ("anchor_k", ctypes.c_void_p),
-                ("anchor_v", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
+                ("codes", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("anchors", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
                 ("append_counter", ctypes.c_void_p)]
 
 
@@ -48,7 +47,7 @@ class DenseDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
-                ("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p),
+                ("kv_pages", ctypes.c_void_p),
                 ("block_table", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
                 ("append_counter", ctypes.c_void_p)]
 
@@ -130,29 +129,25 @@ class LatentCache:
         max_lat = max(1, max_tokens - n_sink - window)
         self.max_pages = math.ceil(max_lat / PAGE_TOKENS)
         self.num_pages = B * self.max_pages
-        self.k_codes = torch.zeros((self.num_pages, H_kv, r_k // ce, PAGE_TOKENS, ce),
-                                   dtype=dtype, device=device)
-        self.v_codes = torch.zeros((self.num_pages, H_kv, r_v // ce, PAGE_TOKENS, ce),
-                                   dtype=dtype, device=device)
+        # one slab per (page, kv head): key-code chunks, then value-code chunks
+        self.codes = torch.zeros((self.num_pages, H_kv, (r_k + r_v) // ce, PAGE_TOKENS, ce),
+                                 dtype=dtype, device=device)
         ids = torch.arange(self.num_pages, dtype=torch.int32) if page_perm is None else \
             torch.as_tensor(page_perm, dtype=torch.int32)
         self.block_table = ids.reshape(B, self.max_pages).to(device)
         self.anchor_tiles = math.ceil((n_sink + window) / FULL_RANK_TILE)
         na = max(1, self.anchor_tiles)
-        self.anchor_k = torch.zeros((B, H_kv, na, HEAD_DIM // ce, FULL_RANK_TILE, ce),
-                                    dtype=dtype, device=device)
-        self.anchor_v = torch.zeros_like(self.anchor_k)
+        self.anchors = torch.zeros((B, H_kv, na, 2 * HEAD_DIM // ce, FULL_RANK_TILE, ce),
+                                   dtype=dtype, device=device)
         self.seq_len = torch.zeros(B, dtype=torch.int32, device=device)
         self.append_counter = torch.zeros(B, dtype=torch.int32, device=device)
         self.desc = CacheDesc(B, H_kv, HEAD_DIM, r_k, r_v, _dtype_code(dtype), n_sink, window,
-                              self.num_pages, self.max_pages, self.k_codes.data_ptr(),
-                              self.v_codes.data_ptr(), self.block_table.data_ptr(),
-                              self.anchor_k.data_ptr(), self.anchor_v.data_ptr(),
+                              self.num_pages, self.max_pages, self.codes.data_ptr(),
+                              self.block_table.data_ptr(), self.anchors.data_ptr(),
                               self.seq_len.data_ptr(), self.append_counter.data_ptr())
 
     def nbytes_codes(self) -> int:
-        return self.k_codes.numel() * self.k_codes.element_size() + \
-            self.v_codes.numel() * self.v_codes.element_size()
+        return self.codes.numel() * self.codes.element_size()
 
 
 def _kv_strides(k: torch.Tensor):
@@ -181,10 +176,11 @@ def decode_workspace_bytes(cache: LatentCache, num_q_heads: int) -> int:
 
 
 def decode_workspace(cache: LatentCache, num_q_heads: int, device="cuda") -> torch.Tensor:
+    """Zero-filled decode workspace (the library keeps its counters at zero)."""
     n = decode_workspace_bytes(cache, num_q_heads)
     if n == 0:
         raise LrkvError("lrkv_decode_workspace_bytes", -2)
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def decode_attn(cache: LatentCache, q: torch.Tensor, P_k: torch.Tensor, P_v: torch.Tensor,
@@ -225,16 +221,15 @@ class DenseCache:
         self.B, self.H_kv, self.dtype = B, H_kv, dtype
         self.max_pages = math.ceil(max_tokens / FULL_RANK_TILE)
         self.num_pages = B * self.max_pages
-        shape = (self.num_pages, H_kv, HEAD_DIM // ce, FULL_RANK_TILE, ce)
-        self.k_pages = torch.zeros(shape, dtype=dtype, device=device)
-        self.v_pages = torch.zeros(shape, dtype=dtype, device=device)
+        self.kv_pages = torch.zeros((self.num_pages, H_kv, 2 * HEAD_DIM // ce, FULL_RANK_TILE, ce),
+                                    dtype=dtype, device=device)
         ids = torch.arange(self.num_pages, dtype=torch.int32) if page_perm is None else \
             torch.as_tensor(page_perm, dtype=torch.int32)
         self.block_table = ids.reshape(B, self.max_pages).to(device)
         self.seq_len = torch.zeros(B, dtype=torch.int32, device=device)
         self.append_counter = torch.zeros(B, dtype=torch.int32, device=device)
         self.desc = DenseDesc(B, H_kv, HEAD_DIM, _dtype_code(dtype), self.num_pages,
-                              self.max_pages, self.k_pages.data_ptr(), self.v_pages.data_ptr(),
+                              self.max_pages, self.kv_pages.data_ptr(),
                               self.block_table.data_ptr(), self.seq_len.data_ptr(),
                               self.append_counter.data_ptr())
 
@@ -253,7 +248,7 @@ def dense_decode_workspace(cache: DenseCache, num_q_heads: int, device="cuda") -
     n = int(_lib.lrkv_dense_decode_workspace_bytes(ctypes.byref(cache.desc), num_q_heads))
     if n == 0:
         raise LrkvError("lrkv_dense_decode_workspace_bytes", -2)
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def dense_decode_attn(cache: DenseCache, q: torch.Tensor, scale: float, o: torch.Tensor,

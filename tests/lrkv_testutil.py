@@ -23,21 +23,29 @@ def torch_dtype(wl):
 
 
 def gather_codes(cache, b, kvh, n, kind="k"):
-    """Codes of latent tokens 0..n-1 of (b, kvh) as float64 [n, r]."""
-    pool = cache.k_codes if kind == "k" else cache.v_codes
+    """Codes of latent tokens 0..n-1 of (b, kvh) as float64 [n, r]; the slab
+    of a page holds the key-code chunks first, then the value-code chunks."""
+    ce = cache.codes.shape[-1]
+    nk = cache.r_k // ce
+    lo, hi = (0, nk) if kind == "k" else (nk, nk + cache.r_v // ce)
     r = cache.r_k if kind == "k" else cache.r_v
     bt = cache.block_table[b].long().cpu()
     j = torch.arange(n)
     pages = bt[j // 64]
     rows = j % 64
-    x = pool[pages.to(pool.device), kvh, :, rows.to(pool.device), :]  # [n, r/CE, CE]
+    x = cache.codes[pages.to(cache.codes.device), kvh, lo:hi][
+        torch.arange(n, device=cache.codes.device), :, rows.to(cache.codes.device), :]
     return x.reshape(n, r).double().cpu().numpy()
 
 
 def gather_anchor_slots(cache, b, kvh, slots, kind="k"):
-    pool = cache.anchor_k if kind == "k" else cache.anchor_v
+    ce = cache.anchors.shape[-1]
+    h = 128 // ce
+    lo, hi = (0, h) if kind == "k" else (h, 2 * h)
     s = torch.as_tensor(slots, dtype=torch.long)
-    x = pool[b, kvh, (s // 32).to(pool.device), :, (s % 32).to(pool.device), :]
+    dev = cache.anchors.device
+    x = cache.anchors[b, kvh, (s // 32).to(dev), lo:hi][torch.arange(len(slots), device=dev), :,
+                                                         (s % 32).to(dev), :]
     return x.reshape(len(slots), D).double().cpu().numpy()
 
 

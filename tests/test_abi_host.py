@@ -45,21 +45,20 @@ def test_struct_layout_matches_header(lrkv, tmp_path):
     src.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "lrkv.h"\n'
         'int main(void){printf("%zu %zu %zu %zu %zu\\n", sizeof(lrkv_cache),'
-        ' offsetof(lrkv_cache, k_codes), offsetof(lrkv_cache, append_counter),'
+        ' offsetof(lrkv_cache, codes), offsetof(lrkv_cache, append_counter),'
         ' sizeof(lrkv_dense_cache), offsetof(lrkv_dense_cache, append_counter));return 0;}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     got = list(map(int, subprocess.check_output([str(exe)]).split()))
     C, Dn = lrkv.CacheDesc, lrkv.DenseDesc
-    assert got == [ctypes.sizeof(C), C.k_codes.offset, C.append_counter.offset,
+    assert got == [ctypes.sizeof(C), C.codes.offset, C.append_counter.offset,
                    ctypes.sizeof(Dn), Dn.append_counter.offset]
 
 
 def _desc(lrkv, **kw):
     base = dict(batch=2, num_kv_heads=2, head_dim=128, rank_k=64, rank_v=32, dtype=0,
-                n_sink=0, window=0, num_pages=4, max_pages_per_seq=2, k_codes=16,
-                v_codes=16, block_table=16, anchor_k=16, anchor_v=16, seq_len=16,
-                append_counter=16)
+                n_sink=0, window=0, num_pages=4, max_pages_per_seq=2, codes=16,
+                block_table=16, anchors=16, seq_len=16, append_counter=16)
     base.update(kw)
     return lrkv.CacheDesc(**base)
 
@@ -70,7 +69,7 @@ FAKE = ctypes.c_void_p(4096)  # never dereferenced: every case fails validation
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 64, -2), ("rank_k", 12, -2), ("rank_v", 0, -2), ("rank_k", 136, -2),
     ("dtype", 7, -2), ("batch", 0, -1), ("n_sink", 2, -1), ("window", -1, -1),
-    ("k_codes", 0, -1), ("k_codes", 8, -1), ("num_pages", 0, -1), ("seq_len", 0, -1),
+    ("codes", 0, -1), ("codes", 8, -1), ("num_pages", 0, -1), ("seq_len", 0, -1),
     ("append_counter", 0, -1)])
 def test_compress_rejects_bad_cache(lrkv, field, value, status):
     d = _desc(lrkv, **{field: value})
@@ -90,7 +89,7 @@ def test_compress_rejects_bad_calls(lrkv):
     assert L.lrkv_compress(ctypes.byref(d), FAKE, FAKE, 129, None, 0, 0, FAKE, FAKE, 0, None) == -3
     # zero tokens is a no-op that launches nothing
     assert L.lrkv_compress(ctypes.byref(d), FAKE, FAKE, 0, None, 0, 0, FAKE, FAKE, 0, None) == 0
-    anch = _desc(lrkv, window=4, anchor_k=0)
+    anch = _desc(lrkv, window=4, anchors=0)
     assert L.lrkv_compress(ctypes.byref(anch), FAKE, FAKE, 4, None, 0, 0, FAKE, FAKE, 0, None) == -1
 
 
@@ -119,7 +118,7 @@ def test_oja_and_dense_reject_bad_calls(lrkv):
     assert L.lrkv_oja_update(FAKE, 1, 8, 1024, None, 0, 0, 0, 0.1, 0, 0, None) == 0
     assert L.lrkv_qr_orthonormalize(FAKE, 1, 0, 1024, None) == -1
     dd = lrkv.DenseDesc(batch=1, num_kv_heads=1, head_dim=100, dtype=0, num_pages=1,
-                        max_pages_per_seq=1, k_pages=16, v_pages=16, block_table=16,
+                        max_pages_per_seq=1, kv_pages=16, block_table=16,
                         seq_len=16, append_counter=16)
     assert L.lrkv_dense_append(ctypes.byref(dd), FAKE, FAKE, 1, None, 0, 0, None) == -2
     dd.head_dim = 128

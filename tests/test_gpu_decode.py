@@ -116,7 +116,9 @@ def test_llama_layer_anchors_small(lrkv):
     dict(T=250, r_k=128, r_v=8),
 ])
 def test_edge_cases(lrkv, case):
-    wl = wk.LLAMA31_LAYER_32K_ANCHORS.with_(B=2, n_decode=2, n_sink=0, window=0, **case)
+    kw = dict(B=2, n_decode=2, n_sink=0, window=0)
+    kw.update(case)
+    wl = wk.LLAMA31_LAYER_32K_ANCHORS.with_(**kw)
     _run_and_compare(lrkv, wl)
 
 
