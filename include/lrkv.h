@@ -140,6 +140,30 @@ int lrkv_decode_attn(const lrkv_cache *cache, const void *q, int32_t num_q_heads
                      int64_t basis_batch_stride, float scale, void *o,
                      void *workspace, size_t workspace_bytes, void *stream);
 
+/* Decode attention that allocates nothing and takes no workspace.  The
+ * pages have no counterpart to this entry point: it exists for callers that
+ * cannot allocate device memory or hand the library a buffer -- a plugin
+ * inside a host framework that owns every allocation, or code on a path
+ * where cudaMalloc's device synchronisation is not allowed.
+ *   Same arguments and results as lrkv_decode_attn, minus the workspace.
+ *   Scratch: a fixed array of LRKV_STATIC_WORKSPACE_BYTES compiled into the
+ *     library, resident on every GPU that loads it until the process exits.
+ *     Configurations needing more scratch than that (see
+ *     lrkv_decode_workspace_bytes) return LRKV_ERR_WORKSPACE and launch
+ *     nothing.
+ *   The first call on a device (with that device current) looks up the
+ *     array's device address once; make that first call before any stream
+ *     capture.
+ *   All calls share the one array: calls whose work overlaps on the GPU
+ *     (other streams, other host threads) race and give wrong results;
+ *     keep them ordered on one stream.  Each call clears the parts that must
+ *     start at zero.  The error word is not reported by this entry point. */
+#define LRKV_STATIC_WORKSPACE_BYTES (4u << 20)
+int lrkv_decode_attn_static(const lrkv_cache *cache, const void *q,
+                            int32_t num_q_heads, const float *P_k,
+                            const float *P_v, int64_t basis_batch_stride,
+                            float scale, void *o, void *stream);
+
 /* Oja subspace update of S independent bases, in place (OjaKV article:
  * online PCA with Oja's algorithm during prefill and periodically during
  * decode).  For each token x of stream s in order: y = P^T x,

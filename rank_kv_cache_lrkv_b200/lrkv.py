@@ -55,7 +55,7 @@ class DenseDesc(ctypes.Structure):
 EXPORTS = ["lrkv_compress", "lrkv_decode_workspace_bytes", "lrkv_decode_attn",
            "lrkv_oja_update", "lrkv_qr_orthonormalize", "lrkv_dense_append",
            "lrkv_dense_decode_workspace_bytes", "lrkv_dense_decode_attn",
-           "lrkv_status_string", "lrkv_version"]
+           "lrkv_status_string", "lrkv_version", "lrkv_decode_attn_static"]
 
 
 def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
@@ -74,6 +74,7 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "lrkv_dense_append": (ctypes.c_int, [P, P, P, I32, P, I64, I64, P]),
         "lrkv_dense_decode_workspace_bytes": (SZ, [P, I32]),
         "lrkv_dense_decode_attn": (ctypes.c_int, [P, P, I32, F32, P, P, SZ, P]),
+        "lrkv_decode_attn_static": (ctypes.c_int, [P, P, I32, P, P, I64, F32, P, P]),
         "lrkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "lrkv_version": (ctypes.c_int, []),
     }
@@ -191,6 +192,18 @@ def decode_attn(cache: LatentCache, q: torch.Tensor, P_k: torch.Tensor, P_v: tor
     _check("lrkv_decode_attn", _lib.lrkv_decode_attn(
         ctypes.byref(cache.desc), _ptr(q), q.shape[1], _ptr(P_k), _ptr(P_v), basis_batch_stride,
         float(scale), _ptr(o), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o
+
+
+def decode_attn_static(cache: LatentCache, q: torch.Tensor, P_k: torch.Tensor,
+                       P_v: torch.Tensor, scale: float, o: torch.Tensor,
+                       basis_batch_stride: int = 0, stream=None) -> torch.Tensor:
+    """lrkv_decode_attn_static: decode attention using the library's built-in
+    scratch instead of a workspace, for callers that cannot allocate one."""
+    assert q.is_contiguous() and o.is_contiguous() and q.dtype == cache.dtype
+    _check("lrkv_decode_attn_static", _lib.lrkv_decode_attn_static(
+        ctypes.byref(cache.desc), _ptr(q), q.shape[1], _ptr(P_k), _ptr(P_v), basis_batch_stride,
+        float(scale), _ptr(o), _stream(stream)))
     return o
 
 
