@@ -9,6 +9,19 @@ from rank_kv_cache_lrkv_b200 import workloads as wk
 
 D = 128
 
+# Tolerances (max over rows of ||o - o_ref||_inf / ||o_ref||_inf):
+#  * bf16 codes, fp32 accumulation, end to end vs the oracle's float64 codes:
+#    2e-2 (the stated bar for bf16 codes).
+#  * fp32 path end to end: 1e-4 (the stated bar for fp32 paths).
+#  * attention alone (oracle on the GPU's own stored codes and anchors):
+#    5e-3 for bf16 outputs (one bf16 rounding of o is 2^-9 of ||o||_inf, plus
+#    fp32 accumulation) and 2e-5 for fp32.
+#  * codes: bf16 storage rounds each code to 2^-9 relative; rows are checked
+#    at 1e-2 of the row's largest code.  fp32 codes at 1e-5.
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+TOL_ISO = {"bf16": 5e-3, "f32": 2e-5}
+TOL_CODE = {"bf16": 1e-2, "f32": 1e-5}
+
 
 def row_rel_err(o, ref) -> float:
     """max over rows (b, h) of ||o - ref||_inf / ||ref||_inf."""
@@ -133,3 +146,55 @@ def run_oracle(wl, inp, n_steps=None, units=None):
             outs.append(oc.attend(q, Pk, Pv, wl.scale)[0])
         res[(b, h)] = (oc, outs)
     return res
+
+
+def check_state(wl, inp, cache, oc, L):
+    """Codes and anchors on the GPU vs the oracle's cache (same schedule)."""
+    for b in range(wl.B):
+        for h in range(wl.H_kv):
+            n = oc.codes_k[b][h].shape[0]
+            for kind, ref in (("k", oc.codes_k[b][h]), ("v", oc.codes_v[b][h])):
+                if n == 0:
+                    continue
+                got = gather_codes(cache, b, h, n, kind)
+                den = np.maximum(np.max(np.abs(ref), axis=1), 1e-30)
+                err = np.max(np.max(np.abs(got - ref), axis=1) / den)
+                assert err < TOL_CODE[wl.dtype], (b, h, kind, err)
+            Ka, Va = oc.anchors(b, h)
+            if Ka.shape[0]:
+                slots = window_slots(L, wl.n_sink, wl.window)
+                assert np.array_equal(gather_anchor_slots(cache, b, h, slots, "k"), Ka)
+                assert np.array_equal(gather_anchor_slots(cache, b, h, slots, "v"), Va)
+
+
+def isolated(wl, inp, cache, L, q, o_gpu):
+    """Oracle attention over the GPU's stored codes and anchors."""
+    Ck, Cv, Ka, Va = [], [], [], []
+    _, lat, _ = orc.partition(L, wl.n_sink, wl.window)
+    slots = window_slots(L, wl.n_sink, wl.window)
+    for b in range(wl.B):
+        Ck.append([gather_codes(cache, b, h, len(lat), "k") for h in range(wl.H_kv)])
+        Cv.append([gather_codes(cache, b, h, len(lat), "v") for h in range(wl.H_kv)])
+        Ka.append([gather_anchor_slots(cache, b, h, slots, "k") if slots else np.zeros((0, 128))
+                   for h in range(wl.H_kv)])
+        Va.append([gather_anchor_slots(cache, b, h, slots, "v") if slots else np.zeros((0, 128))
+                   for h in range(wl.H_kv)])
+    ref = orc.decode_from_parts(q, inp.Pk.double().numpy()[None], inp.Pv.double().numpy()[None],
+                                Ck, Cv, Ka, Va, wl.G, wl.scale)
+    return row_rel_err(o_gpu, ref)
+
+
+def run_and_compare(lrkv, wl, steps=None, page_perm=None, chunks=None, iso=True):
+    inp = Inputs(wl)
+    cache, outs = run_gpu(wl, inp, steps, page_perm=page_perm, lrkv=lrkv,
+                          prefill_chunks=chunks)
+    oc, refs = run_oracle(wl, inp, steps)
+    errs = [row_rel_err(o, r) for o, r in zip(outs, refs)]
+    assert max(errs) < TOL[wl.dtype], errs
+    L = wl.T + (len(outs) if wl.append_before_attend else 0)
+    assert int(cache.seq_len.cpu().min()) == L == int(cache.seq_len.cpu().max())
+    check_state(wl, inp, cache, oc, L)
+    if iso:
+        e = isolated(wl, inp, cache, L, inp.q[len(outs) - 1].double().numpy(), outs[-1])
+        assert e < TOL_ISO[wl.dtype], e
+    return errs

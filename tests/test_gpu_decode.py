@@ -21,9 +21,8 @@ from tests import lrkv_testutil as tu
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"bf16": 2e-2, "f32": 1e-4}
-TOL_ISO = {"bf16": 5e-3, "f32": 2e-5}
-TOL_CODE = {"bf16": 1e-2, "f32": 1e-5}
+TOL, TOL_ISO, TOL_CODE = tu.TOL, tu.TOL_ISO, tu.TOL_CODE
+_run_and_compare = tu.run_and_compare
 
 
 @pytest.fixture(scope="module")
@@ -31,58 +30,6 @@ def lrkv():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     from rank_kv_cache_lrkv_b200 import lrkv as m
     return m
-
-
-def _check_state(wl, inp, cache, oc, L):
-    """Codes and anchors on the GPU vs the oracle's cache (same schedule)."""
-    for b in range(wl.B):
-        for h in range(wl.H_kv):
-            n = oc.codes_k[b][h].shape[0]
-            for kind, ref in (("k", oc.codes_k[b][h]), ("v", oc.codes_v[b][h])):
-                if n == 0:
-                    continue
-                got = tu.gather_codes(cache, b, h, n, kind)
-                den = np.maximum(np.max(np.abs(ref), axis=1), 1e-30)
-                err = np.max(np.max(np.abs(got - ref), axis=1) / den)
-                assert err < TOL_CODE[wl.dtype], (b, h, kind, err)
-            Ka, Va = oc.anchors(b, h)
-            if Ka.shape[0]:
-                slots = tu.window_slots(L, wl.n_sink, wl.window)
-                assert np.array_equal(tu.gather_anchor_slots(cache, b, h, slots, "k"), Ka)
-                assert np.array_equal(tu.gather_anchor_slots(cache, b, h, slots, "v"), Va)
-
-
-def _isolated(wl, inp, cache, L, q, o_gpu):
-    """Oracle attention over the GPU's stored codes and anchors."""
-    Ck, Cv, Ka, Va = [], [], [], []
-    _, lat, _ = orc.partition(L, wl.n_sink, wl.window)
-    slots = tu.window_slots(L, wl.n_sink, wl.window)
-    for b in range(wl.B):
-        Ck.append([tu.gather_codes(cache, b, h, len(lat), "k") for h in range(wl.H_kv)])
-        Cv.append([tu.gather_codes(cache, b, h, len(lat), "v") for h in range(wl.H_kv)])
-        Ka.append([tu.gather_anchor_slots(cache, b, h, slots, "k") if slots else np.zeros((0, 128))
-                   for h in range(wl.H_kv)])
-        Va.append([tu.gather_anchor_slots(cache, b, h, slots, "v") if slots else np.zeros((0, 128))
-                   for h in range(wl.H_kv)])
-    ref = orc.decode_from_parts(q, inp.Pk.double().numpy()[None], inp.Pv.double().numpy()[None],
-                                Ck, Cv, Ka, Va, wl.G, wl.scale)
-    return tu.row_rel_err(o_gpu, ref)
-
-
-def _run_and_compare(lrkv, wl, steps=None, page_perm=None, chunks=None, iso=True):
-    inp = tu.Inputs(wl)
-    cache, outs = tu.run_gpu(wl, inp, steps, page_perm=page_perm, lrkv=lrkv,
-                             prefill_chunks=chunks)
-    oc, refs = tu.run_oracle(wl, inp, steps)
-    errs = [tu.row_rel_err(o, r) for o, r in zip(outs, refs)]
-    assert max(errs) < TOL[wl.dtype], errs
-    L = wl.T + (len(outs) if wl.append_before_attend else 0)
-    assert int(cache.seq_len.cpu().min()) == L == int(cache.seq_len.cpu().max())
-    _check_state(wl, inp, cache, oc, L)
-    if iso:
-        e = _isolated(wl, inp, cache, L, inp.q[len(outs) - 1].double().numpy(), outs[-1])
-        assert e < TOL_ISO[wl.dtype], e
-    return errs
 
 
 def test_tiny_single_head_fp32(lrkv):
