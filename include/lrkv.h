@@ -115,25 +115,24 @@ int lrkv_compress(const lrkv_cache *cache, const void *k, const void *v,
                   const float *P_k, const float *P_v,
                   int64_t basis_batch_stride, void *stream);
 
-/* Bytes of workspace lrkv_decode_attn needs on the current device.  The
- * workspace must be zero-filled once when it is allocated: it holds per-
- * (sequence, KV head) tile counters that every completed call leaves at
- * zero, split-K partial records, and (first 4 bytes) an error word. */
+/* Bytes of workspace lrkv_decode_attn needs on the current device.  It
+ * holds the folded queries, the split-K partial records and (first 4 bytes)
+ * an error word; zero the error word when the workspace is allocated. */
 size_t lrkv_decode_workspace_bytes(const lrkv_cache *cache, int32_t num_q_heads);
 
 /* Decode attention of one query per q head over the latent cache plus the
  * full-rank anchors (Half the Memory, section 08: attend directly against
  * the codes; q folded as q~ = P_k^T q, o = P_v sum p c_v + sum p_a v_a).
- * One kernel launch.
+ * Three stream-ordered launches (q-fold, split-K, merge).
  *   q, o  : [batch][num_q_heads][128] in the cache dtype (q post-RoPE).
  *           q head h reads KV head h / (num_q_heads / num_kv_heads).
  *   scale : softmax scale applied to q . k (1/sqrt(128) for these models).
- *   workspace : zero-filled once (see above), at least
- *           lrkv_decode_workspace_bytes; calls sharing a workspace must be
- *           stream-ordered.  The error word is set (1 = a bounded wait timed
- *           out, 2 = a block-table entry out of range) and never cleared by
- *           the library; after a nonzero error word, zero the workspace
- *           again before reusing it.
+ *   P_v must be 16-byte aligned and basis_batch_stride a multiple of 4
+ *           (LRKV_ERR_ARG otherwise).
+ *   workspace : at least lrkv_decode_workspace_bytes, 16-byte aligned; calls sharing a
+ *           workspace must be stream-ordered.  The error word is set (1 = a
+ *           bounded wait timed out, 2 = a block-table entry out of range)
+ *           and never cleared by the library.
  * A sequence with no tokens gets o = 0. */
 int lrkv_decode_attn(const lrkv_cache *cache, const void *q, int32_t num_q_heads,
                      const float *P_k, const float *P_v,
@@ -200,7 +199,7 @@ typedef struct lrkv_dense_cache {
 int lrkv_dense_append(const lrkv_dense_cache *cache, const void *k,
                       const void *v, int32_t n_tokens, const int32_t *n_new,
                       int64_t seq_stride, int64_t head_stride, void *stream);
-/* Workspace of the dense decode; the same zero-once contract as above. */
+/* Workspace of the dense decode; the same contract as above. */
 size_t lrkv_dense_decode_workspace_bytes(const lrkv_dense_cache *cache,
                                          int32_t num_q_heads);
 int lrkv_dense_decode_attn(const lrkv_dense_cache *cache, const void *q,

@@ -99,7 +99,8 @@ int lrkv_decode_attn(const lrkv_cache* cache, const void* q, int32_t num_q_heads
   rc = check_heads(cache->num_kv_heads, num_q_heads);
   if (rc != LRKV_OK) return rc;
   if (!q || !o || !P_k || !P_v || !workspace || basis_batch_stride < 0) return LRKV_ERR_ARG;
-  if (!aligned16(workspace)) return LRKV_ERR_ARG;
+  // the value basis is read four floats at a time
+  if (!aligned16(workspace) || !aligned16(P_v) || basis_batch_stride % 4 != 0) return LRKV_ERR_ARG;
   DecodeLaunch L;
   L.B = cache->batch; L.H_kv = cache->num_kv_heads; L.H_q = num_q_heads; L.dtype = cache->dtype;
   L.seq_len = cache->seq_len; L.n_sink = cache->n_sink; L.W = cache->window;

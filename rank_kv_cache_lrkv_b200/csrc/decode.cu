@@ -1,26 +1,30 @@
 // Decode attention over the latent code cache plus full-rank anchors.
 //
-// One persistent launch per call, one CTA per SM.  The tiles of all
-// (sequence, KV head) units are laid end to end -- latent pages (64 tokens)
-// in one space, full-rank anchor tiles (32 tokens) in another -- and each CTA
-// takes an equal contiguous range of each space, so any mix of sequence
-// lengths is balanced across SMs.
-//  * Two producer warps (odd and even tiles, each owning half the stages)
-//    compute tile addresses a batch ahead (block-table reads in parallel)
-//    and stream one slab per tile into a shared-memory ring with bulk
-//    copies that complete on mbarriers.
-//  * Eight consumer warps take every eighth tile.  At the start of each unit
-//    in the CTA's range they fold that unit's queries together:
-//    q~ = P_k^T q for its G query heads (Half the Memory, section 08: attend
-//    directly against the codes), pre-scaled by scale * log2(e) so the
-//    softmax runs on exp2.  Per tile: scores with lane = token (q chunks
-//    broadcast from shared memory, packed fp32 FMA), an exp2 online softmax
-//    with one max per tile, then p * c_v with lanes split over value chunks.
-//  * At a unit boundary the warps' partial (m, l, acc) are combined in
-//    shared memory into one record per (unit, CTA); the CTA whose record
-//    completes the unit's tile count combines all records of the unit and
-//    writes o = (P_v acc_lat + acc_fr) / l, then resets the unit's counter.
-// The dense full-rank baseline runs the same kernel with no latent space.
+// Three launches per call, stream-ordered; the second and third use
+// programmatic dependent launch so they start while their predecessor ends.
+//  1. qfold : per (sequence, KV head) unit, q~ = P_k^T q for its G query
+//             heads (Half the Memory, section 08: attend directly against the
+//             codes) and the full-rank q, both pre-scaled by scale * log2(e)
+//             so the softmax runs on exp2.
+//  2. split : persistent, one CTA per SM.  The latent pages of all units are
+//             laid end to end and each CTA takes an equal contiguous range,
+//             so any mix of sequence lengths is balanced.  A producer warp
+//             streams one slab per page into a shared-memory ring with bulk
+//             copies completing on mbarriers (addresses computed a batch
+//             ahead).  Eight consumer warps take every eighth page: scores
+//             with lane = token (q chunks broadcast from shared memory,
+//             packed fp32 FMA), an exp2 online softmax with one max per page,
+//             then p * c_v with lanes split over value chunks.  Each warp
+//             writes its own partial (m, l, acc) record per unit it touched;
+//             warps never wait for one another.  An anchor warp processes
+//             this CTA's share of the full-rank anchor tiles straight from
+//             global memory while the pages stream, and writes one record per
+//             unit.  (The dense baseline streams its full-rank pages through
+//             the ring instead and has no anchor warp.)
+//  3. merge : per unit, combines every record (running max, rescaled sums),
+//             up-projects the latent accumulator, o = (P_v acc_lat + acc_fr)
+//             / l, and writes zeros for sequences with no tokens.
+#include <limits.h>
 #include <math.h>
 
 #include <algorithm>
@@ -30,15 +34,16 @@
 
 namespace lrkv {
 
-constexpr int kConsumers = 8;                    // consumer warps per CTA
-constexpr int kProducers = 2;                    // producer warps per CTA
-constexpr int kCThreads = 32 * kConsumers;       // consumer threads
-constexpr int kThreads = 32 * (kProducers + kConsumers);
-constexpr int kMaxStages = 16;
-constexpr int kBarConsumers = 1;                 // named barrier id
-constexpr int kIssue = 4;                        // producer lanes issuing at once
-constexpr int kMaxPre = 4;                       // chunks whose queries are fetched at start
-constexpr int kMaxRec = 160;                     // records (CTAs) per unit and space
+constexpr int kConsumers = 8;                  // consumer warps per CTA
+constexpr int kProducerWarp = 0;
+constexpr int kAnchorWarp = 1;
+constexpr int kFirstConsumer = 2;
+constexpr int kThreads = 32 * (kFirstConsumer + kConsumers);
+constexpr int kMaxStages = 24;
+constexpr int kIssue = 4;                      // producer lanes issuing at once
+constexpr int kMergeThreads = 256;
+constexpr int kMergeBuf = 64 * 1024;           // merge: bytes of records per chunk
+constexpr int kMergeMaxRec = 256;              // merge: records per chunk at most
 
 struct DecodeArgs {
   int B, H_kv, G, H_q;
@@ -50,7 +55,7 @@ struct DecodeArgs {
   int maxp_lat, rk, rv;
   // full-rank space (fr == nullptr: empty); one slab per tile
   const void* fr;
-  const int* bt_fr;  // nullptr: tiles of a unit are contiguous
+  const int* bt_fr;  // nullptr: anchors (tiles of a unit contiguous), else dense pages
   int maxp_fr;       // block-table row length, or tiles per unit
   int num_pages_lat, num_pages_fr;
   const float* P_v;
@@ -61,13 +66,12 @@ struct DecodeArgs {
   float qscale;        // scale * log2(e)
   // workspace
   int* err;            // sticky error word
-  int* unit_cnt;       // [B * H_kv] tile counters, zero between calls
   float* qlat;         // [B][H_q][rk] folded queries (scaled)
   float* qfr;          // [B][H_q][128] scaled queries
-  float* part_lat;
-  float* part_fr;
-  int C;   // CTAs of the split grid
-  int NS;  // ring stages
+  float* part_lat;     // [(U + C - 1) * kConsumers] latent records
+  float* part_fr;      // anchors: [U + C - 1]; dense: [(U + C - 1) * kConsumers]
+  int C;               // CTAs of the split grid
+  int NS;              // ring stages
   int stage_bytes;
 };
 
@@ -268,7 +272,62 @@ __device__ __forceinline__ void process_tile(const uint4* kch, int n_valid, int 
   __syncwarp();
 }
 
-// ------------------------------------------------------------ kernel pieces
+// ------------------------------------------------------------ q-fold kernel
+constexpr int kFoldThreads = 128;  // small, so q-fold CTAs fit beside split CTAs
+constexpr int kFoldSplit = 2;      // CTAs per unit, each folding a share of the columns
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kFoldThreads) qfold_kernel(DecodeArgs a) {
+  __shared__ float qs[G * kHeadDim];
+  __shared__ float red[G * kFoldThreads];
+  pdl_trigger();
+  const int unit = blockIdx.x / kFoldSplit, part = blockIdx.x % kFoldSplit;
+  const int b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
+  const size_t h0 = (size_t)b * a.H_q + (size_t)kvh * G;
+  const T* q = static_cast<const T*>(a.q) + h0 * kHeadDim;
+  for (int x = tid; x < G * kHeadDim; x += kFoldThreads) qs[x] = to_f<T>(q[x]);
+  __syncthreads();
+  if (part == 0) {
+    if (a.fr)
+      for (int x = tid; x < G * kHeadDim; x += kFoldThreads)
+        a.qfr[h0 * kHeadDim + x] = qs[x] * a.qscale;
+  }
+  if (!a.codes) return;
+  // This CTA folds columns [c0, c1); thread -> (column, row segment) with at
+  // most 32 rows, all loads in flight at once.
+  const int rk = a.rk, cper = (rk + kFoldSplit - 1) / kFoldSplit;
+  const int c0 = part * cper, c1 = min(rk, c0 + cper), nc = c1 - c0;
+  if (nc <= 0) return;
+  const int nseg = max(1, kFoldThreads / nc), rows = (kHeadDim + nseg - 1) / nseg;
+  const float* P = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * rk;
+  for (int col = tid; col < nseg * nc; col += kFoldThreads) {
+    const int j = c0 + col % nc, seg = col / nc;
+    float acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = 0.f;
+    const int i0 = seg * rows, i1 = min(kHeadDim, i0 + rows);
+    for (int ib = i0; ib < i1; ib += 32) {
+      float pij[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) pij[u] = ib + u < i1 ? __ldg(P + (size_t)(ib + u) * rk + j) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 32; ++u)
+        if (ib + u < i1)
+#pragma unroll
+          for (int g = 0; g < G; ++g) acc[g] = fmaf(pij[u], qs[g * kHeadDim + ib + u], acc[g]);
+    }
+    for (int g = 0; g < G; ++g) red[(seg * G + g) * nc + (j - c0)] = acc[g];
+  }
+  __syncthreads();
+  for (int x = tid; x < G * nc; x += kFoldThreads) {
+    const int g = x / nc, jj = x - g * nc;
+    float sum = 0.f;
+    for (int sg = 0; sg < nseg; ++sg) sum += red[(sg * G + g) * nc + jj];
+    a.qlat[h0 * rk + g * rk + c0 + jj] = sum * a.qscale;
+  }
+}
+
+
 // Bounded spin until the producer has issued tile k into this stage.
 __device__ inline bool tag_wait_bounded(volatile int* tag, int k,
                                         uint64_t timeout_ns = 2000000000ull) {
@@ -281,10 +340,14 @@ __device__ inline bool tag_wait_bounded(volatile int* tag, int k,
   }
 }
 
+// True when the anchor warp (not the ring) handles the full-rank space.
+__host__ __device__ inline bool anchor_mode(const void* fr, const int* bt_fr) {
+  return fr != nullptr && bt_fr == nullptr;
+}
+
 // Shared-memory plan of the split kernel (byte offsets from the base).
 struct SmemPlan {
-  int ring, full, empty, tag, start_lat, start_fr, pbuf, qv, cml, cacc, fin_lat, recs, flags,
-      total;
+  int ring, full, empty, tag, start_lat, start_fr, pbuf, qown, flags, total;
 };
 __host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, int G) {
   SmemPlan p;
@@ -301,192 +364,145 @@ __host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, in
   p.tag = take(kMaxStages * 4, 4);
   p.start_lat = take((B + 1) * 4, 4);
   p.start_fr = take((B + 1) * 4, 4);
-  p.pbuf = take(kConsumers * kLatPage * G * 8, 16);
-  p.qv = take((kMaxPre + 1) * G * kHeadDim * 4, 16);  // folded queries per chunk
-  p.cml = take(kConsumers * 2 * G * 4, 16);
-  p.cacc = take(G * kHeadDim * 4, 16);
-  p.fin_lat = take(G * kHeadDim * 4, 16);
-  p.recs = take(2 * kMaxRec * 4, 16);
+  // per consumer warp and the anchor warp: probabilities [G][64] as pairs and
+  // the unit's folded queries [G][128]
+  p.pbuf = take((kConsumers + 1) * kLatPage * G * 8, 16);
+  p.qown = take((kConsumers + 1) * G * kHeadDim * 4, 16);
   p.flags = take(16, 16);
   p.total = off;
   return p;
 }
 
-// Folded queries of every (sequence, KV head) unit, computed before the
-// split kernel streams anything (the memory system is still quiet):
-// q~ = P_k^T q for the latent space (Half the Memory, section 08: attend
-// directly against the codes) and q for the full-rank space, both times
-// scale * log2(e) so the softmax runs on exp2.  Also writes o = 0 for
-// sequences with no tokens.  One CTA of 256 threads per unit.
-template <typename T, int G>
-__global__ void __launch_bounds__(256) qfold_kernel(DecodeArgs a) {
-  __shared__ float qs[G * kHeadDim];
-  __shared__ float red[G * 256];
-  pdl_trigger();
-  const int unit = blockIdx.x, b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
-  const size_t h0 = (size_t)b * a.H_q + (size_t)kvh * G;
-  const T* q = static_cast<const T*>(a.q) + h0 * kHeadDim;
-  for (int x = tid; x < G * kHeadDim; x += 256) qs[x] = to_f<T>(q[x]);
-  __syncthreads();
-  if (a.seq_len[b] <= 0) {
-    T* o = static_cast<T*>(a.o) + h0 * kHeadDim;
-    for (int x = tid; x < G * kHeadDim; x += 256) o[x] = from_f<T>(0.f);
-  }
-  if (a.fr)
-    for (int x = tid; x < G * kHeadDim; x += 256) a.qfr[h0 * kHeadDim + x] = qs[x] * a.qscale;
-  if (!a.codes) return;
-  // thread -> (column j, row segment); all of a thread's loads in flight.
-  const int rk = a.rk, nseg = 256 / rk, rows = (kHeadDim + nseg - 1) / nseg;
-  const int j = tid % rk, seg = tid / rk;
-  const float* P = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * rk;
-  float acc[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) acc[g] = 0.f;
-  if (seg < nseg) {
-    const int i0 = seg * rows, i1 = min(kHeadDim, i0 + rows);
-    for (int ib = i0; ib < i1; ib += 32) {
-      float pij[32];
-#pragma unroll
-      for (int u = 0; u < 32; ++u) pij[u] = ib + u < i1 ? __ldg(P + (size_t)(ib + u) * rk + j) : 0.f;
-#pragma unroll
-      for (int u = 0; u < 32; ++u)
-        if (ib + u < i1)
-#pragma unroll
-          for (int g = 0; g < G; ++g) acc[g] = fmaf(pij[u], qs[g * kHeadDim + ib + u], acc[g]);
-    }
-    for (int g = 0; g < G; ++g) red[(seg * G + g) * rk + j] = acc[g];
-  }
-  __syncthreads();
-  for (int x = tid; x < G * rk; x += 256) {
-    const int g = x / rk, jj = x - g * rk;
-    float sum = 0.f;
-    for (int sg = 0; sg < nseg; ++sg) sum += red[(sg * G + g) * rk + jj];
-    a.qlat[h0 * rk + x] = sum * a.qscale;
-  }
-}
-
-// Copy the folded queries of unit (b, kvh) for space sp into dst.
+// The folded queries of unit (b, kvh) for space sp -> dst (one warp).
 template <int G>
-__device__ inline void fetch_queries(const DecodeArgs& a, int sp, int b, int kvh, float* dst,
-                                     int ctid) {
+__device__ inline void fetch_queries_warp(const DecodeArgs& a, int sp, int b, int kvh,
+                                          float* dst, int lane) {
   const int dim = sp == 0 ? a.rk : kHeadDim;
-  const float* src = (sp == 0 ? a.qlat : a.qfr) + ((size_t)b * a.H_q + (size_t)kvh * G) * dim;
-  for (int x = ctid; x < G * dim; x += kCThreads) dst[x] = __ldcg(src + x);
+  const float4* src = reinterpret_cast<const float4*>(
+      (sp == 0 ? a.qlat : a.qfr) + ((size_t)b * a.H_q + (size_t)kvh * G) * dim);
+  float4* d4 = reinterpret_cast<float4*>(dst);
+  for (int x = lane; x < G * dim / 4; x += 32) d4[x] = __ldcg(src + x);
+  __syncwarp();
 }
 
-// Online merge of one more (max m, weight-sum) pair into (M, S1, S2).
-__device__ __forceinline__ void merge_rec(float m, float l, float v, float& M, float& L, float& S) {
-  if (!(m > -INFINITY)) return;
-  if (m > M) {
-    const float r = exp2f(M - m);
-    L *= r;
-    S *= r;
-    M = m;
-  }
-  const float w = exp2f(m - M);
-  L = fmaf(w, l, L);
-  S = fmaf(w, v, S);
-}
-
-// Combine every record of `unit` and write its G output rows.  Run by all
-// consumer threads of the CTA that completed the unit.  The records' offsets
-// (or -1 where a CTA's range is empty) are listed first; then one load phase:
-// each thread loads, for the accumulator elements it owns, every record's
-// (m, l, value) eight at a time and merges them online (running max,
-// rescaled sums).  One barrier publishes the latent accumulator, then
-// o = (P_v acc_lat + acc_fr) / l.
+// A warp's partial (m, l, acc) -> record rec: m[G], l[G] then acc [G][rvd].
+// The lanes hold acc for value chunk jc of tokens tsub (TS lanes per chunk).
 template <typename T, int G>
-__device__ void finalize_unit(const DecodeArgs& a, int unit, const int* start_lat,
-                              const int* start_fr, float* fin_lat, int* recs, int ctid) {
-  const int b = unit / a.H_kv, kvh = unit - b * a.H_kv;
+__device__ inline void write_record(float* rec, int rvd, int TS, int ncv, const float (&m)[G],
+                                    const float (&l)[G], float2 (&acc)[G][Elem<T>::CE / 2],
+                                    int lane) {
+  constexpr int CE = Elem<T>::CE, NP = CE / 2;
   const int H = hdr_floats(G);
-  int nr[2];
-  const int* starts[2] = {start_lat, start_fr};
-  const int rvs[2] = {a.rv, kHeadDim};
-  const float* parts[2] = {a.part_lat, a.part_fr};
-  // record list: recs[sp * kMaxRec + r] = record index (unit + c) or -1
 #pragma unroll
-  for (int sp = 0; sp < 2; ++sp) {
-    const int total = starts[sp][a.B];
-    const int tiles = (starts[sp][b + 1] - starts[sp][b]) / a.H_kv;
-    nr[sp] = 0;
-    if (total == 0 || tiles == 0) continue;
-    const int us = starts[sp][b] + kvh * tiles;
-    const int c0 = cta_of(us, total, a.C);
-    nr[sp] = min(kMaxRec, cta_of(us + tiles - 1, total, a.C) - c0 + 1);
-    for (int r = ctid; r < nr[sp]; r += kCThreads) {
-      const int c = c0 + r;
-      recs[sp * kMaxRec + r] =
-          range_lo(c, total, a.C) == range_lo(c + 1, total, a.C) ? -1 : unit + c;
-    }
+  for (int h = 0; h < G; ++h) {
+    const float lt = warp_sum(l[h]);
+    if (lane == 0) { rec[h] = m[h]; rec[G + h] = lt; }
   }
-  named_bar(kBarConsumers, kCThreads);
-  auto combine = [&](int g, int vsp, int vx, float& M, float& L, float& S) {
-    M = -INFINITY; L = 0.f; S = 0.f;
-    for (int sp = 0; sp < 2; ++sp) {
-      const int stride = H + G * rvs[sp];
-      for (int r0 = 0; r0 < nr[sp]; r0 += 8) {
-        float mm[8], ll[8], vv[8];
+  for (int o = TS >> 1; o > 0; o >>= 1)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          mm[u] = -INFINITY; ll[u] = 0.f; vv[u] = 0.f;
-          const int ri = r0 + u < nr[sp] ? recs[sp * kMaxRec + r0 + u] : -1;
-          if (ri >= 0) {
-            const float* rec = parts[sp] + (size_t)ri * stride;
-            mm[u] = __ldcg(rec + g);
-            ll[u] = __ldcg(rec + G + g);
-            if (sp == vsp) vv[u] = __ldcg(rec + H + vx);
-          }
-        }
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) merge_rec(mm[u], ll[u], vv[u], M, L, S);
+      for (int e = 0; e < NP; ++e) {
+        acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
+        acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
       }
-    }
-  };
-  if (a.codes)
-    for (int x = ctid; x < G * a.rv; x += kCThreads) {
-      float M, L, S;
-      combine(x / a.rv, 0, x, M, L, S);
-      fin_lat[x] = S;
-    }
-  constexpr int kPer = (G * kHeadDim + kCThreads - 1) / kCThreads;
-  float accf[kPer], den[kPer];
+  const int jc = lane / TS, tsub = lane - jc * TS;
+  if (tsub == 0 && jc < ncv)
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int x = ctid + i * kCThreads;
-    accf[i] = 0.f; den[i] = 0.f;
-    if (x < G * kHeadDim) {
-      float M, L, S;
-      combine(x / kHeadDim, a.fr ? 1 : -1, x, M, L, S);
-      accf[i] = S;
-      den[i] = L;
-    }
-  }
-  named_bar(kBarConsumers, kCThreads);
-  T* o = static_cast<T*>(a.o) + ((size_t)b * a.H_q + (size_t)kvh * G) * kHeadDim;
-  const float* P = a.codes ? a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv : nullptr;
+    for (int h = 0; h < G; ++h) {
+      float4* dst = reinterpret_cast<float4*>(rec + H + h * rvd + jc * CE);
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int x = ctid + i * kCThreads;
-    if (x >= G * kHeadDim) break;
-    const int g = x / kHeadDim, d = x - g * kHeadDim;
-    float out = accf[i];
-    if (P) {
-      const float4* Pd = reinterpret_cast<const float4*>(P + (size_t)d * a.rv);
-      const float4* al = reinterpret_cast<const float4*>(fin_lat + g * a.rv);
-#pragma unroll 8
-      for (int j4 = 0; j4 < a.rv / 4; ++j4) {
-        const float4 pv = __ldg(Pd + j4), av = al[j4];
-        out = fmaf(pv.x, av.x, fmaf(pv.y, av.y, fmaf(pv.z, av.z, fmaf(pv.w, av.w, out))));
-      }
+      for (int e4 = 0; e4 < NP / 2; ++e4)
+        dst[e4] = make_float4(acc[h][2 * e4].x, acc[h][2 * e4].y, acc[h][2 * e4 + 1].x,
+                              acc[h][2 * e4 + 1].y);
     }
-    o[x] = from_f<T>(den[i] > 0.f ? out / den[i] : 0.f);
-  }
-  if (ctid == 0) a.unit_cnt[unit] = 0;  // ready for the next call
-  named_bar(kBarConsumers, kCThreads);
 }
 
-// ------------------------------------------------------------ the kernel
+// One full-rank anchor tile of 32 tokens read straight from global memory by
+// one warp (no ring stage): lane = token for the scores, lanes split over
+// value chunks for the accumulation.  Same math as process_tile.
+template <typename T, int G>
+__device__ void anchor_tile(const uint4* kch, int n_valid, const float* qv, float2* pbuf,
+                            float (&m)[G], float (&l)[G], float2 (&acc)[G][Elem<T>::CE / 2],
+                            int lane) {
+  constexpr int CE = Elem<T>::CE, NP = CE / 2, TT = kFrTile, NC = kHeadDim / CE;
+  const uint4* vch = kch + NC * TT;
+  // Phase A: the lane's key chunks, eight loads in flight at a time.
+  float2 s2[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) s2[h] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j0 = 0; j0 < NC; j0 += 8) {
+    uint4 kc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      kc[u] = lane < n_valid ? __ldcs(kch + (j0 + u) * TT + lane) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u;
+      float2 f[NP];
+      chunk_pairs<T>(kc[u], f);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float4* src = reinterpret_cast<const float4*>(qv + h * kHeadDim + j * CE);
+#pragma unroll
+        for (int e4 = 0; e4 < NP / 2; ++e4) {
+          const float4 x = src[e4];
+          fma2(s2[h], make_float2(x.x, x.y), f[2 * e4]);
+          fma2(s2[h], make_float2(x.z, x.w), f[2 * e4 + 1]);
+        }
+      }
+    }
+  }
+  float alpha[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float sc = lane < n_valid ? s2[h].x + s2[h].y : -INFINITY;
+    const float mn = fmaxf(m[h], warp_max(sc));
+    alpha[h] = exp2f(m[h] - mn);
+    m[h] = mn;
+    const float pr = exp2f(sc - mn);
+    l[h] = l[h] * alpha[h] + pr;
+    pbuf[h * TT + lane] = make_float2(pr, pr);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float2 a2 = make_float2(alpha[h], alpha[h]);
+#pragma unroll
+    for (int e = 0; e < NP; ++e) acc[h][e] = mul2(acc[h][e], a2);
+  }
+  // Phase B: lane -> (value chunk jc, token parity tsub); loads first.
+  constexpr int TS = 32 / NC;  // 2 (bf16) or 1 (fp32)
+  const int jc = lane / TS, tsub = lane - jc * TS;
+  constexpr int STEPS = TT / TS;
+#pragma unroll
+  for (int i0 = 0; i0 < STEPS; i0 += 8) {  // eight loads in flight at a time
+    uint4 vc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = (i0 + u) * TS + tsub;
+      vc[u] = t < n_valid ? __ldcs(vch + jc * TT + t) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = (i0 + u) * TS + tsub;
+      if (t < n_valid) {
+        float2 f[NP];
+        chunk_pairs<T>(vc[u], f);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float2 pp = pbuf[h * TT + t];
+#pragma unroll
+          for (int e = 0; e < NP; ++e) fma2(acc[h][e], pp, f[e]);
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------ split kernel
 template <typename T, int G>
 __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
   constexpr int CE = Elem<T>::CE;
@@ -504,15 +520,14 @@ __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
   volatile int* tag = reinterpret_cast<volatile int*>(smem + sp_.tag);
   int* start_lat = reinterpret_cast<int*>(smem + sp_.start_lat);
   int* start_fr = reinterpret_cast<int*>(smem + sp_.start_fr);
-  // flags: [0] failure (any warp, any time), [1] finalize this unit,
-  // [2] consumers' snapshot of [0] taken between their named barriers.
-  int* flags = reinterpret_cast<int*>(smem + sp_.flags);
+  volatile int* fail = reinterpret_cast<volatile int*>(smem + sp_.flags);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
+  pdl_trigger();  // the merge grid may be scheduled; it waits for this grid to finish
   if (warp == 0) build_prefix(a, start_lat, start_fr);
   if (threadIdx.x == 32) {
-    flags[0] = flags[1] = flags[2] = 0;
+    *fail = 0;
     for (int s = 0; s < a.NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -522,62 +537,53 @@ __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
   }
   __syncthreads();
 
-  const int tot0 = start_lat[a.B], tot1 = start_fr[a.B];
-  const int lo0 = range_lo(c, tot0, a.C), hi0 = range_lo(c + 1, tot0, a.C);
-  const int lo1 = range_lo(c, tot1, a.C), hi1 = range_lo(c + 1, tot1, a.C);
-  const int n0 = hi0 - lo0, N = n0 + (hi1 - lo1);
+  const bool anchors = anchor_mode(a.fr, a.bt_fr);
+  // The ring carries the latent pages, or the full-rank pages in dense mode.
+  const int rsp = a.codes ? 0 : 1;
+  const int* rstart = rsp == 0 ? start_lat : start_fr;
+  const int rtot = rstart[a.B];
+  const int lo = range_lo(c, rtot, a.C), hi = range_lo(c + 1, rtot, a.C), N = hi - lo;
 
-  if (warp < kProducers) {
-    // ---------------- producer warp p: tiles k = p, p + 2, p + 4, ...
-    // Lane l holds the slab address of tile base + kProducers * l; the next
-    // batch's block-table reads are in flight while this batch is issued,
-    // kIssue lanes at a time.
-    const int p = warp;
+  if (warp == kProducerWarp) {
+    // ---------------- producer: lane l holds the slab address of tile base + l;
+    // the next batch's block-table reads are in flight while this batch is
+    // issued, kIssue lanes at a time.
+    const uint64_t pol = l2_evict_first_policy();
     auto addr = [&](int kk, const void*& src, uint32_t& bytes, int& good) {
       src = nullptr; bytes = 0; good = 0;
       if (kk >= N) return;
-      const int sp = kk < n0 ? 0 : 1;
-      const int t = sp == 0 ? lo0 + kk : lo1 + (kk - n0);
       int b, kvh, i, tiles;
-      locate(sp == 0 ? start_lat : start_fr, a.B, a.H_kv, t, b, kvh, i, tiles);
-      size_t slab;
-      if (sp == 0) {
+      locate(rstart, a.B, a.H_kv, lo + kk, b, kvh, i, tiles);
+      if (rsp == 0) {
         const int page = a.bt_lat[(size_t)b * a.maxp_lat + i];
         good = page >= 0 && page < a.num_pages_lat;
-        slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
+        const size_t slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
         bytes = kLatPage * (a.rk + a.rv) * sizeof(T);
         src = static_cast<const T*>(a.codes) + slab * kLatPage * (a.rk + a.rv);
       } else {
-        if (a.bt_fr) {
-          const int page = a.bt_fr[(size_t)b * a.maxp_fr + i];
-          good = page >= 0 && page < a.num_pages_fr;
-          slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
-        } else {
-          good = 1;
-          slab = ((size_t)b * a.H_kv + kvh) * a.maxp_fr + i;
-        }
+        const int page = a.bt_fr[(size_t)b * a.maxp_fr + i];
+        good = page >= 0 && page < a.num_pages_fr;
+        const size_t slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
         bytes = 2 * kFrTile * kHeadDim * sizeof(T);
         src = static_cast<const T*>(a.fr) + slab * 2 * kFrTile * kHeadDim;
       }
     };
-    constexpr int kBatch = 32 * kProducers;
     const void *csrc, *nsrc;
     uint32_t cbytes, nbytes;
     int cgood, ngood;
-    const uint64_t pol = l2_evict_first_policy();
-    addr(p + kProducers * lane, csrc, cbytes, cgood);
-    int issued_last = -1;  // last tile this warp issued
+    addr(lane, csrc, cbytes, cgood);
+    int issued = 0;
     bool ok = true;
-    for (int base = 0; base < N && ok; base += kBatch) {
-      addr(base + kBatch + p + kProducers * lane, nsrc, nbytes, ngood);
-      const int cnt = min(32, (N - base - p + kProducers - 1) / kProducers);
+    for (int base = 0; base < N && ok; base += 32) {
+      addr(base + 32 + lane, nsrc, nbytes, ngood);
+      const int cnt = min(32, N - base);
       for (int j0 = 0; j0 < cnt; j0 += kIssue) {
-        int fail = 0;
+        int f = 0;
         if (lane >= j0 && lane < min(j0 + kIssue, cnt)) {
-          const int k = base + p + kProducers * lane, s = k % a.NS, n = k / a.NS;
+          const int k = base + lane, s = k % a.NS, n = k / a.NS;
           if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) {
             *a.err = kErrTimeout;
-            fail = 1;
+            f = 1;
           } else {
             uint8_t* dst = ring + (size_t)s * a.stage_bytes;
             if (cgood) {
@@ -590,186 +596,360 @@ __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
             tag[s] = k;
           }
         }
-        if (__any_sync(0xffffffffu, fail) || *(volatile int*)&flags[0]) {
+        if (__any_sync(0xffffffffu, f) || *fail) {
           ok = false;
-          flags[0] = 1;
+          *fail = 1;
           break;
         }
-        issued_last = base + p + kProducers * (min(j0 + kIssue, cnt) - 1);
+        issued = base + min(j0 + kIssue, cnt);
       }
       csrc = nsrc; cbytes = nbytes; cgood = ngood;
     }
-    // Drain: wait (bounded) for every copy this warp issued (its stages are
-    // those with s % kProducers == p, since NS is a multiple of kProducers).
-    if (lane == 0 && issued_last >= 0)
-      for (int s = p; s < a.NS; s += kProducers) {
-        if (s > issued_last) break;
-        const int last = s + ((issued_last - s) / a.NS) * a.NS;
+    // Drain: wait (bounded) for every copy this CTA issued before exiting.
+    if (lane == 0)
+      for (int s = 0; s < a.NS && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / a.NS) * a.NS;
         if (!mbar_wait_bounded(&full[s], (last / a.NS) & 1)) *a.err = kErrTimeout;
       }
-  } else {
-    // ---------------- consumers
-    const int w = warp - kProducers, ctid = threadIdx.x - 32 * kProducers;
-    float2* pbuf = reinterpret_cast<float2*>(smem + sp_.pbuf) + w * kLatPage * G;
-    float* qv = reinterpret_cast<float*>(smem + sp_.qv);
-    float* cml = reinterpret_cast<float*>(smem + sp_.cml);
-    float* cacc = reinterpret_cast<float*>(smem + sp_.cacc);
-    for (int x = ctid; x < G * kHeadDim; x += kCThreads) cacc[x] = 0.f;
-    named_bar(kBarConsumers, kCThreads);
-    // Fetch the folded queries of the first kMaxPre chunks now, while the
-    // first tiles are in flight (later these loads would queue behind the
-    // streaming copies).
-    pdl_wait();  // the q-fold kernel's results (and counters) are visible
-    {
-      int npre = 0;
-      for (int sp = 0; sp < 2 && npre < kMaxPre; ++sp) {
-        const int lo = sp == 0 ? lo0 : lo1, hi = sp == 0 ? hi0 : hi1;
-        for (int t = lo; t < hi && npre < kMaxPre; ++npre) {
-          int b, kvh, i0, tiles;
-          locate(sp == 0 ? start_lat : start_fr, a.B, a.H_kv, t, b, kvh, i0, tiles);
-          fetch_queries<G>(a, sp, b, kvh, qv + npre * G * kHeadDim, ctid);
-          t = min(hi, t - i0 + tiles);
-        }
+    return;
+  }
+
+  pdl_wait();  // the q-fold results are visible from here on
+  float2* pbuf = reinterpret_cast<float2*>(smem + sp_.pbuf) +
+                 (warp == kAnchorWarp ? kConsumers : warp - kFirstConsumer) * kLatPage * G;
+  float* qv = reinterpret_cast<float*>(smem + sp_.qown) +
+              (warp == kAnchorWarp ? kConsumers : warp - kFirstConsumer) * G * kHeadDim;
+
+  if (warp == kAnchorWarp) {
+    // ---------------- anchor warp: this CTA's share of the anchor tiles
+    if (!anchors) return;
+    const int tot = start_fr[a.B];
+    const int flo = range_lo(c, tot, a.C), fhi = range_lo(c + 1, tot, a.C);
+    const int rec_stride = hdr_floats(G) + G * kHeadDim;
+    int t = flo;
+    while (t < fhi) {
+      int b, kvh, i0, tiles;
+      locate(start_fr, a.B, a.H_kv, t, b, kvh, i0, tiles);
+      const int unit = b * a.H_kv + kvh, ustart = t - i0, ce = min(fhi, ustart + tiles);
+      const int ntok = space_tokens(a, 1, b);
+      fetch_queries_warp<G>(a, 1, b, kvh, qv, lane);
+      float m[G], l[G];
+      float2 acc[G][NP];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        m[h] = -INFINITY; l[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
       }
-      named_bar(kBarConsumers, kCThreads);
-    }
-    int chunk = 0;
-    for (int sp = 0; sp < 2; ++sp) {
-      const int lo = sp == 0 ? lo0 : lo1, hi = sp == 0 ? hi0 : hi1;
-      const int kbase = sp == 0 ? 0 : n0;
-      if (lo >= hi) continue;
-      const int* start = sp == 0 ? start_lat : start_fr;
-      const int nck = sp == 0 ? a.rk / CE : kHeadDim / CE;
-      const int ncv = sp == 0 ? a.rv / CE : kHeadDim / CE;
-      const int rvd = sp == 0 ? a.rv : kHeadDim;
-      int TS = 1;
-      while (TS * 2 * ncv <= 32) TS *= 2;
-      const int jc = lane / TS, tsub = lane - jc * TS;
-      const int qdim = sp == 0 ? a.rk : kHeadDim;
-      float* part = sp == 0 ? a.part_lat : a.part_fr;
-      const int rec_stride = hdr_floats(G) + G * rvd;
-      int t = lo;
-      while (t < hi) {
-        int b, kvh, i0, tiles;
-        locate(start, a.B, a.H_kv, t, b, kvh, i0, tiles);
-        const int unit = b * a.H_kv + kvh;
-        const int ustart = t - i0;
-        const int ce = min(hi, ustart + tiles);
-        const int ntok = space_tokens(a, sp, b);
-        float* qc = qv + min(chunk, kMaxPre) * G * kHeadDim;
-        if (chunk >= kMaxPre) {
-          fetch_queries<G>(a, sp, b, kvh, qc, ctid);
-          named_bar(kBarConsumers, kCThreads);
-        }
-        ++chunk;
-        float m[G], l[G];
-        float2 acc[G][NP];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          m[h] = -INFINITY; l[h] = 0.f;
-#pragma unroll
-          for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
-        }
-        const int k0 = kbase + (t - lo);
-        for (int tt = t + ((w - k0 % kConsumers) + kConsumers) % kConsumers; tt < ce;
-             tt += kConsumers) {
-          const int k = kbase + (tt - lo), s = k % a.NS, n = k / a.NS;
-          if (!tag_wait_bounded(tag + s, k) || !mbar_wait_bounded(&full[s], n & 1)) {
-            *a.err = kErrTimeout;
-            flags[0] = 1;
-            break;
-          }
-          const int it = tt - ustart;
-          const uint4* st = reinterpret_cast<const uint4*>(ring + (size_t)s * a.stage_bytes);
-          if (sp == 0)
-            process_tile<T, G, kLatPage>(st, min(kLatPage, ntok - it * kLatPage), nck, ncv, TS,
-                                         qc, qdim, pbuf, m, l, acc, lane);
-          else
-            process_tile<T, G, kFrTile>(st, min(kFrTile, ntok - it * kFrTile), nck, ncv, TS,
-                                        qc, qdim, pbuf, m, l, acc, lane);
-          if (lane == 0) mbar_arrive(&empty[s]);
-        }
-        // ---- combine the warps' partials into one record for (unit, CTA)
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float lt = warp_sum(l[h]);
-          if (lane == 0) { cml[w * 2 * G + h] = m[h]; cml[w * 2 * G + G + h] = lt; }
-        }
-        for (int o = TS >> 1; o > 0; o >>= 1)
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int e = 0; e < NP; ++e) {
-              acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
-              acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
-            }
-        named_bar(kBarConsumers, kCThreads);
-        if (tsub == 0 && jc < ncv) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float M = -INFINITY;
-            for (int ww = 0; ww < kConsumers; ++ww) M = fmaxf(M, cml[ww * 2 * G + h]);
-            const float sc = m[h] > -INFINITY ? exp2f(m[h] - M) : 0.f;
-            if (sc != 0.f)
-#pragma unroll
-              for (int e = 0; e < NP; ++e) {
-                atomicAdd(&cacc[h * rvd + jc * CE + 2 * e], acc[h][e].x * sc);
-                atomicAdd(&cacc[h * rvd + jc * CE + 2 * e + 1], acc[h][e].y * sc);
-              }
-          }
-        }
-        named_bar(kBarConsumers, kCThreads);
-        if (w == 0) {
-          float* rec = part + (size_t)(unit + c) * rec_stride;
-          if (lane < G) {
-            float M = -INFINITY;
-            for (int ww = 0; ww < kConsumers; ++ww) M = fmaxf(M, cml[ww * 2 * G + lane]);
-            float L = 0.f;
-            for (int ww = 0; ww < kConsumers; ++ww) {
-              const float mw = cml[ww * 2 * G + lane];
-              if (mw > -INFINITY) L += exp2f(mw - M) * cml[ww * 2 * G + G + lane];
-            }
-            rec[lane] = M;
-            rec[G + lane] = L;
-          }
-          const int H = hdr_floats(G);
-          for (int x = lane; x < G * rvd; x += 32) {
-            rec[H + x] = cacc[x];
-            cacc[x] = 0.f;
-          }
-          __syncwarp();
-          if (lane == 0) {
-            __threadfence();
-            const int need = (start_lat[b + 1] - start_lat[b]) / a.H_kv +
-                             (start_fr[b + 1] - start_fr[b]) / a.H_kv;
-            const int got = atomicAdd(&a.unit_cnt[unit], ce - t) + (ce - t);
-            flags[1] = (got == need);
-            flags[2] = *(volatile int*)&flags[0];
-            if (got == need) __threadfence();
-          }
-        }
-        named_bar(kBarConsumers, kCThreads);
-        if (flags[1])
-          finalize_unit<T, G>(a, unit, start_lat, start_fr,
-                              reinterpret_cast<float*>(smem + sp_.fin_lat),
-                              reinterpret_cast<int*>(smem + sp_.recs), ctid);
-        t = ce;
-        if (flags[2]) break;  // uniform: written before the last named barrier
+      for (int tt = t; tt < ce; ++tt) {
+        const size_t slab = ((size_t)b * a.H_kv + kvh) * a.maxp_fr + (tt - ustart);
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(a.fr) +
+                                                          slab * 2 * kFrTile * kHeadDim);
+        anchor_tile<T, G>(src, min(kFrTile, ntok - (tt - ustart) * kFrTile), qv, pbuf, m, l,
+                          acc, lane);
       }
-      if (flags[2]) break;
+      write_record<T, G>(a.part_fr + (size_t)(unit + c) * rec_stride, kHeadDim, 32 / (kHeadDim / CE),
+                         kHeadDim / CE, m, l, acc, lane);
+      t = ce;
     }
+    return;
+  }
+
+  // ---------------- consumers
+  const int w = warp - kFirstConsumer;
+  const int nck = rsp == 0 ? a.rk / CE : kHeadDim / CE;
+  const int ncv = rsp == 0 ? a.rv / CE : kHeadDim / CE;
+  const int rvd = rsp == 0 ? a.rv : kHeadDim;
+  const int qdim = rsp == 0 ? a.rk : kHeadDim;
+  int TS = 1;
+  while (TS * 2 * ncv <= 32) TS *= 2;
+  float* part = rsp == 0 ? a.part_lat : a.part_fr;
+  const int rec_stride = hdr_floats(G) + G * rvd;
+  int t = lo;
+  while (t < hi) {
+    int b, kvh, i0, tiles;
+    locate(rstart, a.B, a.H_kv, t, b, kvh, i0, tiles);
+    const int unit = b * a.H_kv + kvh, ustart = t - i0, ce = min(hi, ustart + tiles);
+    const int ntok = space_tokens(a, rsp, b);
+    fetch_queries_warp<G>(a, rsp, b, kvh, qv, lane);
+    float m[G], l[G];
+    float2 acc[G][NP];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      m[h] = -INFINITY; l[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
+    }
+    const int k0 = t - lo;
+    for (int tt = t + ((w - k0 % kConsumers) + kConsumers) % kConsumers; tt < ce;
+         tt += kConsumers) {
+      const int k = tt - lo, s = k % a.NS, n = k / a.NS;
+      if (!tag_wait_bounded(tag + s, k) || !mbar_wait_bounded(&full[s], n & 1)) {
+        *a.err = kErrTimeout;
+        *fail = 1;
+        break;
+      }
+      const int it = tt - ustart;
+      const uint4* st = reinterpret_cast<const uint4*>(ring + (size_t)s * a.stage_bytes);
+      if (rsp == 0)
+        process_tile<T, G, kLatPage>(st, min(kLatPage, ntok - it * kLatPage), nck, ncv, TS, qv,
+                                     qdim, pbuf, m, l, acc, lane);
+      else
+        process_tile<T, G, kFrTile>(st, min(kFrTile, ntok - it * kFrTile), nck, ncv, TS, qv,
+                                    qdim, pbuf, m, l, acc, lane);
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // This warp's record for (unit, CTA); m = -inf when it had no tile.
+    write_record<T, G>(part + ((size_t)(unit + c) * kConsumers + w) * rec_stride, rvd, TS, ncv,
+                       m, l, acc, lane);
+    t = ce;
+    if (*fail) break;
+  }
+}
+
+// ------------------------------------------------------------ merge kernel
+// Shared-memory plan of the merge kernel (byte offsets from the base).
+struct MergePlan {
+  int pv, recb, fin, mh, ah, lh, red, wts, vflag, starts, bars, total;
+};
+__host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B) {
+  MergePlan p;
+  int off = 0;
+  auto take = [&](int bytes, int align) {
+    off = (off + align - 1) / align * align;
+    const int at = off;
+    off += bytes;
+    return at;
+  };
+  p.pv = take(lat ? kHeadDim * rv * 4 : 0, 128);
+  p.recb = take(kMergeBuf, 128);
+  p.fin = take(G * kHeadDim * 4, 16);
+  p.mh = take(32, 16);
+  p.ah = take(32, 16);
+  p.lh = take(32, 16);
+  p.red = take((kMergeThreads / 32) * G * 4, 16);
+  p.wts = take(kMergeMaxRec * G * 4, 16);
+  p.vflag = take(kMergeMaxRec * 4, 16);
+  p.starts = take(2 * (B + 1) * 4, 8);
+  p.bars = take(16, 8);
+  p.total = off;
+  return p;
+}
+
+// Block-wide reduction of one value per head; the result lands in dst[G].
+template <int G, bool kMax>
+__device__ inline void block_reduce_heads(float (&v)[G], float* red, float* dst, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float r = kMax ? warp_max(v[g]) : warp_sum(v[g]);
+    if (lane == 0) red[warp * G + g] = r;
+  }
+  __syncthreads();
+  if (tid < G) {
+    float r = kMax ? -INFINITY : 0.f;
+    for (int w = 0; w < kMergeThreads / 32; ++w)
+      r = kMax ? fmaxf(r, red[w * G + tid]) : r + red[w * G + tid];
+    dst[tid] = r;
   }
   __syncthreads();
 }
 
+// Per unit, over every record (m, l, acc) of both spaces:
+//   M_g = max m,  w = exp2(m - M_g),  L_g = sum w l,
+//   lat = sum_latent w acc,  fr = sum_full-rank w acc,
+//   o = (P_v lat + fr) / L_g   (0 where L_g = 0: a sequence with no tokens).
+// A unit's records sit in consecutive slots of each space, so they arrive in
+// shared memory by bulk copies (chunks of kMergeBuf bytes, merged online with
+// a running max), as does the unit's P_v block, fetched before the wait for
+// the split grid since it does not depend on it.
+template <typename T, int G>
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const MergePlan mp = merge_plan(a.rv, a.codes != nullptr, G, a.B);
+  float* pv = reinterpret_cast<float*>(smem + mp.pv);        // [128][r_v]
+  float* recb = reinterpret_cast<float*>(smem + mp.recb);    // records of one chunk
+  float* fin_lat = reinterpret_cast<float*>(smem + mp.fin);  // [G][r_v]
+  float* Mh = reinterpret_cast<float*>(smem + mp.mh);        // running max per head
+  float* Ah = reinterpret_cast<float*>(smem + mp.ah);        // rescale of this chunk
+  float* Lh = reinterpret_cast<float*>(smem + mp.lh);
+  float* red = reinterpret_cast<float*>(smem + mp.red);
+  float* wts = reinterpret_cast<float*>(smem + mp.wts);      // [record][G]
+  int* vflag = reinterpret_cast<int*>(smem + mp.vflag);
+  int* start_lat = reinterpret_cast<int*>(smem + mp.starts);
+  int* start_fr = start_lat + (a.B + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + mp.bars);  // [0] records, [1] P_v
+
+  const int unit = blockIdx.x, b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
+  const float* P = a.codes ? a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv
+                           : nullptr;
+  const uint32_t pv_bytes = (uint32_t)(kHeadDim * a.rv * 4);
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_fence_init();
+  }
+  if (tid < G) Mh[tid] = -INFINITY;
+  __syncthreads();
+  if (tid == 0 && P) {
+    mbar_arrive_expect_tx(&bars[1], pv_bytes);
+    bulk_g2s(pv, P, pv_bytes, &bars[1]);
+  }
+  pdl_wait();  // every record of the split kernel is visible
+  if (tid < 32) build_prefix(a, start_lat, start_fr);
+  __syncthreads();
+  const bool anchors = anchor_mode(a.fr, a.bt_fr);
+  const int H = hdr_floats(G);
+  // records: latent (CTA, warp) pairs, then full-rank (CTA[, warp]) records
+  int c0[2] = {0, 0}, ncta[2] = {0, 0}, total[2];
+  const int* starts[2] = {start_lat, start_fr};
+#pragma unroll
+  for (int sp = 0; sp < 2; ++sp) {
+    total[sp] = starts[sp][a.B];
+    const int tiles = (starts[sp][b + 1] - starts[sp][b]) / a.H_kv;
+    if (total[sp] == 0 || tiles == 0) continue;
+    const int us = starts[sp][b] + kvh * tiles;
+    c0[sp] = cta_of(us, total[sp], a.C);
+    ncta[sp] = cta_of(us + tiles - 1, total[sp], a.C) - c0[sp] + 1;
+  }
+  const int per[2] = {kConsumers, anchors ? 1 : kConsumers};
+  const int rvs[2] = {a.rv, kHeadDim};
+  const float* parts[2] = {a.part_lat, a.part_fr};
+
+  constexpr int kPer = (G * kHeadDim + kMergeThreads - 1) / kMergeThreads;
+  const int E_lat = a.codes ? G * a.rv : 0, E_fr = G * kHeadDim;
+  float lacc[kPer], facc[kPer], ls[G];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) { lacc[i] = 0.f; facc[i] = 0.f; }
+#pragma unroll
+  for (int g = 0; g < G; ++g) ls[g] = 0.f;
+  int chunk = 0;
+  bool ok = true;
+  for (int sp = 0; sp < 2 && ok; ++sp) {
+    const int n = ncta[sp] * per[sp];
+    const int S = H + G * rvs[sp];  // floats per record
+    const int cap = min(kMergeMaxRec, kMergeBuf / (S * 4));
+    const float* base = parts[sp] + (size_t)(unit + c0[sp]) * per[sp] * S;
+    for (int q0 = 0; q0 < n; q0 += cap) {
+      const int nq = min(cap, n - q0);
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&bars[0], (uint32_t)(nq * S * 4));
+        bulk_g2s(recb, base + (size_t)q0 * S, (uint32_t)(nq * S * 4), &bars[0]);
+      }
+      // a record is valid when its CTA's tile range was not empty
+      float mx[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
+      const bool landed = mbar_wait_bounded(&bars[0], chunk & 1);
+      ++chunk;
+      if (!__syncthreads_and(landed)) {
+        ok = false;
+        break;
+      }
+      for (int x = tid; x < nq; x += kMergeThreads) {
+        const int cc = c0[sp] + (q0 + x) / per[sp];
+        const int v = range_lo(cc, total[sp], a.C) != range_lo(cc + 1, total[sp], a.C);
+        vflag[x] = v;
+        if (v)
+#pragma unroll
+          for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], recb[x * S + g]);
+      }
+      block_reduce_heads<G, true>(mx, red, Ah, tid);
+      if (tid < G) {
+        const float nm = fmaxf(Mh[tid], Ah[tid]);
+        Ah[tid] = nm > -INFINITY ? exp2f(Mh[tid] - nm) : 1.f;
+        Mh[tid] = nm;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) ls[g] *= Ah[g];
+      for (int x = tid; x < nq; x += kMergeThreads)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float m = recb[x * S + g];
+          float w = 0.f;
+          if (vflag[x] && m > -INFINITY) {
+            w = exp2f(m - Mh[g]);
+            ls[g] = fmaf(w, recb[x * S + G + g], ls[g]);
+          }
+          wts[x * G + g] = w;
+        }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int e = tid + i * kMergeThreads;
+        if (e < E_lat) lacc[i] *= Ah[e / a.rv];
+        if (e < E_fr) facc[i] *= Ah[e / kHeadDim];
+        const int E = sp == 0 ? E_lat : E_fr;
+        if (e < E) {
+          const int g = e / rvs[sp];
+          const float* col = recb + H + e;
+          float s0 = 0.f, s1 = 0.f;
+          int x = 0;
+          for (; x + 1 < nq; x += 2) {
+            s0 = fmaf(wts[x * G + g], col[x * S], s0);
+            s1 = fmaf(wts[(x + 1) * G + g], col[(x + 1) * S], s1);
+          }
+          if (x < nq) s0 = fmaf(wts[x * G + g], col[x * S], s0);
+          if (sp == 0) lacc[i] += s0 + s1;
+          else facc[i] += s0 + s1;
+        }
+      }
+      __syncthreads();  // the next chunk overwrites recb
+    }
+  }
+  if (!ok) {
+    if (tid == 0) {
+      *a.err = kErrTimeout;
+      // wait (bounded) for the copies still in flight before leaving
+      mbar_wait_bounded(&bars[0], (chunk - 1) & 1);
+      if (P) mbar_wait_bounded(&bars[1], 0);
+    }
+    return;
+  }
+  block_reduce_heads<G, false>(ls, red, Lh, tid);
+
+  // o = (P_v lat + fr) / L
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = tid + i * kMergeThreads;
+    if (e < E_lat) fin_lat[e] = lacc[i];
+  }
+  const bool pv_ok = !P || mbar_wait_bounded(&bars[1], 0);
+  if (!__syncthreads_and(pv_ok)) {
+    if (tid == 0) *a.err = kErrTimeout;
+    return;
+  }
+  T* o = static_cast<T*>(a.o) + ((size_t)b * a.H_q + (size_t)kvh * G) * kHeadDim;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int x = tid + i * kMergeThreads;
+    if (x >= G * kHeadDim) break;
+    const int g = x / kHeadDim, d = x - g * kHeadDim;
+    float out = facc[i];
+    if (P) {
+      // rotated start per row keeps the lanes of a warp on distinct banks
+      const float* row = pv + d * a.rv;
+      const float* lat = fin_lat + g * a.rv;
+      int j = d % a.rv;
+      for (int k = 0; k < a.rv; ++k) {
+        out = fmaf(row[j], lat[j], out);
+        j = j + 1 == a.rv ? 0 : j + 1;
+      }
+    }
+    const float L = Lh[g];
+    o[x] = from_f<T>(L > 0.f ? out / L : 0.f);
+  }
+}
+
 // ------------------------------------------------------------ host side
 struct Plan {
-  int C, NS, stage_bytes, smem;
-  size_t off_cnt, off_qlat, off_qfr, off_lat, off_fr, total;
+  int C, NS, stage_bytes, smem, merge_smem;
+  size_t off_qlat, off_qfr, off_lat, off_fr, total;
 };
 
 static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, bool has_fr,
-                       int esize, Plan& p) {
+                       bool anchors, int esize, Plan& p) {
   int dev = 0, sms = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LRKV_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -777,24 +957,27 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return LRKV_ERR_CUDA;
   const int G = H_q / H_kv;
-  const int lat_b = has_lat ? kLatPage * (rk + rv) * esize : 0;
-  const int fr_b = has_fr ? 2 * kFrTile * kHeadDim * esize : 0;  // key + value
-  p.stage_bytes = std::max(lat_b, fr_b);
+  // the ring holds latent pages, or dense full-rank pages (no latent space)
+  p.stage_bytes = has_lat ? kLatPage * (rk + rv) * esize : 2 * kFrTile * kHeadDim * esize;
+  // Leave room for a q-fold CTA beside each split CTA.
+  const int budget = optin - 8 * 1024;
   const int fixed = smem_plan(0, p.stage_bytes, B, G).total + 1024;
-  p.NS = std::min(kMaxStages, (optin - fixed) / p.stage_bytes);
-  p.NS -= p.NS % kProducers;
-  if (p.NS < kProducers) return LRKV_ERR_UNSUPPORTED;
+  p.NS = std::min(kMaxStages, (budget - fixed) / p.stage_bytes);
+  if (p.NS < 2) return LRKV_ERR_UNSUPPORTED;
   p.smem = smem_plan(p.NS, p.stage_bytes, B, G).total;
   p.C = sms;
+  p.merge_smem = merge_plan(rv, has_lat, G, B).total;
   const int U = B * H_kv;
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   size_t off = 256;
-  p.off_cnt = off;  off = al(off + (size_t)U * 4);
   p.off_qlat = off; off = al(off + (size_t)B * H_q * (has_lat ? rk : 0) * 4);
   p.off_qfr = off;  off = al(off + (size_t)B * H_q * (has_fr ? kHeadDim : 0) * 4);
   const size_t slots = (size_t)(U + p.C - 1);
-  p.off_lat = off;  off = al(off + (has_lat ? slots * (hdr_floats(G) + G * rv) * 4 : 0));
-  p.off_fr = off;   off = al(off + (has_fr ? slots * (hdr_floats(G) + G * kHeadDim) * 4 : 0));
+  p.off_lat = off;
+  off = al(off + (has_lat ? slots * kConsumers * (hdr_floats(G) + G * rv) * 4 : 0));
+  p.off_fr = off;
+  off = al(off + (has_fr ? slots * (anchors ? 1 : kConsumers) * (hdr_floats(G) + G * kHeadDim) * 4
+                         : 0));
   p.total = off;
   return LRKV_OK;
 }
@@ -802,32 +985,51 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
 size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has_lat,
                               bool has_fr, int dtype) {
   Plan p;
-  if (plan_decode(B, H_kv, H_q, rk, rv, has_lat, has_fr, dtype == LRKV_BF16 ? 2 : 4, p) !=
-      LRKV_OK)
+  // anchors: full-rank space present next to a latent one (no block table)
+  if (plan_decode(B, H_kv, H_q, rk, rv, has_lat, has_fr, has_lat && has_fr,
+                  dtype == LRKV_BF16 ? 2 : 4, p) != LRKV_OK)
     return 0;
   return p.total;
 }
 
-template <typename T, int G>
-static int launch_decode_t(const DecodeArgs& a, const Plan& p, cudaStream_t st) {
-  qfold_kernel<T, G><<<a.B * a.H_kv, 256, 0, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
-  if (cudaFuncSetAttribute(split_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           p.smem) != cudaSuccess)
-    return LRKV_ERR_CUDA;
-  // Programmatic dependent launch: the split kernel's producers start
-  // streaming while the q-fold finishes; its consumers wait for it.
+static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, void** args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.C);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = p.smem;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, split_kernel<T, G>, a) != cudaSuccess) return LRKV_ERR_CUDA;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+template <typename T, int G>
+static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st) {
+  // Keep SMs in the large-shared-memory configuration while the q-fold runs,
+  // so the split kernel's CTAs can start beside it without a reconfiguration.
+  cudaFuncSetAttribute(qfold_kernel<T, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       (int)cudaSharedmemCarveoutMaxShared);
+  qfold_kernel<T, G><<<a.B * a.H_kv * kFoldSplit, kFoldThreads, 0, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
+  if (cudaFuncSetAttribute(split_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           p.smem) != cudaSuccess)
+    return LRKV_ERR_CUDA;
+  cudaFuncSetAttribute(split_kernel<T, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       (int)cudaSharedmemCarveoutMaxShared);
+  void* args[] = {&a};
+  if (launch_pdl((const void*)split_kernel<T, G>, dim3(p.C), dim3(kThreads), p.smem, st, args) !=
+      cudaSuccess)
+    return LRKV_ERR_CUDA;
+  if (cudaFuncSetAttribute(merge_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           p.merge_smem) != cudaSuccess)
+    return LRKV_ERR_CUDA;
+  if (launch_pdl((const void*)merge_kernel<T, G>, dim3(a.B * a.H_kv), dim3(kMergeThreads),
+                 p.merge_smem, st, args) != cudaSuccess)
+    return LRKV_ERR_CUDA;
   return LRKV_OK;
 }
 
@@ -846,7 +1048,8 @@ int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
   const bool has_lat = L.codes != nullptr, has_fr = L.fr != nullptr;
   const int es = L.dtype == LRKV_BF16 ? 2 : 4;
   Plan p;
-  int rc = plan_decode(L.B, L.H_kv, L.H_q, L.rk, L.rv, has_lat, has_fr, es, p);
+  int rc = plan_decode(L.B, L.H_kv, L.H_q, L.rk, L.rv, has_lat, has_fr,
+                       anchor_mode(L.fr, L.bt_fr), es, p);
   if (rc != LRKV_OK) return rc;
   if (L.ws_bytes < p.total) return LRKV_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(L.ws);
@@ -860,7 +1063,6 @@ int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
   a.P_v = L.P_v; a.basis_bs = L.basis_bs; a.o = L.o;
   a.q = L.q; a.P_k = L.P_k; a.qscale = L.scale * kLog2e;
   a.err = reinterpret_cast<int*>(ws);
-  a.unit_cnt = reinterpret_cast<int*>(ws + p.off_cnt);
   a.qlat = reinterpret_cast<float*>(ws + p.off_qlat);
   a.qfr = reinterpret_cast<float*>(ws + p.off_qfr);
   a.part_lat = reinterpret_cast<float*>(ws + p.off_lat);

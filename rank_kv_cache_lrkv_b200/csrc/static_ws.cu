@@ -56,12 +56,9 @@ extern "C" int lrkv_decode_attn_static(const lrkv_cache* cache, const void* q,
   void* ws = nullptr;
   int rc = scratch_address(&ws);
   if (rc != LRKV_OK) return rc;
-  // The array keeps the previous call's contents.  The error word and the
-  // per-(sequence, KV head) tile counters (the first 256 bytes plus 4 bytes
-  // per unit) must start at zero, so clear them on the call's stream.
-  const size_t zero = (256 + (size_t)cache->batch * cache->num_kv_heads * 4 + 255) & ~size_t(255);
-  if (cudaMemsetAsync(ws, 0, zero < need ? zero : need, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  // The array keeps the previous call's contents; only the error word in its
+  // first bytes must start at zero, so clear it on the call's stream.
+  if (cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return LRKV_ERR_CUDA;
   return lrkv_decode_attn(cache, q, num_q_heads, P_k, P_v, basis_batch_stride, scale, o, ws,
                           (size_t)LRKV_STATIC_WORKSPACE_BYTES, stream);
