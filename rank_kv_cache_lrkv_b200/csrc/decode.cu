@@ -28,13 +28,14 @@
 #include <math.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
 
 namespace lrkv {
 
-constexpr int kConsumers = 8;                  // consumer warps per CTA
+constexpr int kConsumers = 6;                  // consumer warps per CTA
 constexpr int kProducerWarp = 0;
 constexpr int kAnchorWarp = 1;
 constexpr int kFirstConsumer = 2;
@@ -272,6 +273,183 @@ __device__ __forceinline__ void process_tile(const uint4* kch, int n_valid, int 
   __syncwarp();
 }
 
+// ------------------------------------------------------------ tensor-core tile math (bf16)
+// The same page computation on the tensor cores, one warp per page.
+//  scores:  S^T (m = token, n = head) = C_k (token x dim) . q~^T, q~ split
+//           as hi + lo bf16 so the product keeps about 16 mantissa bits;
+//  softmax: per head over the page's tokens (shuffles across the lanes of
+//           one column pair), p split as hi + lo bf16 like q~;
+//  values:  acc^T (m = value dim, n = head) += C_v^T (dim x token) . P^T.
+// The chunk-major page layout (16-byte rows = 8 elements of one token) is
+// what ldmatrix reads: plain for C_k rows, transposed for C_v^T.  P moves
+// from the score accumulator into the value step's B operand by movmatrix.
+// Heads G..7 of the n = 8 tile are padding (zero queries, never stored).
+// KS / VB: 16-wide steps of the score / value rows the code is built for
+// (a rank class: r_k <= 16 KS, r_v <= 16 VB); the actual counts may be lower.
+template <int KS>
+struct QFrag {
+  uint32_t hi[KS][2], lo[KS][2];  // B operands (k = dim, n = head)
+};
+
+template <int G, int KS>
+__device__ inline void load_qfrag(const float* qv, int qdim, int lane, QFrag<KS>& f) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int s = 0; s < KS; ++s)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int d = 16 * s + 8 * r + 2 * t;
+      float x0 = 0.f, x1 = 0.f;
+      if (g < G && d < qdim) {
+        x0 = qv[g * qdim + d];
+        x1 = qv[g * qdim + d + 1];
+      }
+      const uint32_t h = pack_bf16x2(x0, x1);
+      f.hi[s][r] = h;
+      f.lo[s][r] = pack_bf16x2(x0 - bf_lo(h), x1 - bf_hi(h));
+    }
+}
+
+// Zero the bf16 halves of a (token k, token k + 1) pair that lie at or past n.
+__device__ __forceinline__ uint32_t mask_tokens(uint32_t x, int k, int n) {
+  return (k < n ? x & 0xffffu : 0u) | (k + 1 < n ? x & 0xffff0000u : 0u);
+}
+
+// One page (TT tokens) of a ring stage; running state per lane: m, l for
+// heads 2t and 2t + 1 (l is this lane's partial), acc fragments per 16 value dims.
+template <int TT, int KS, int VB>
+__device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, int nck, int ncv,
+                                                 const QFrag<KS>& qf, float (&m)[2],
+                                                 float (&l)[2], float (&acc)[VB][4], int lane) {
+  constexpr int MB = TT / 16;
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t kbase = smem_u32(kch), vbase = smem_u32(kch + nck * TT);
+  const int nks = (nck + 1) >> 1, nvb = (ncv + 1) >> 1;
+  const bool partial = n_valid < TT;
+
+  // Phase A (an odd last chunk is read twice; its q~ half is zero)
+  float sc[MB][4];
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[mb][i] = 0.f;
+  // (rows of tokens past n_valid are read but masked below)
+  const int arow = lane & 15, ahalf = lane >> 4;
+#pragma unroll
+  for (int s = 0; s < KS; ++s) {
+    if (s < nks) {
+      const int c = min(2 * s + ahalf, nck - 1);
+      uint32_t a[MB][4];
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb)
+        ldsm_x4(kbase + (uint32_t)((c * TT + mb * 16 + arow) * 16), a[mb]);
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) mma_bf16_16816(sc[mb], a[mb], qf.hi[s][0], qf.hi[s][1]);
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) mma_bf16_16816(sc[mb], a[mb], qf.lo[s][0], qf.lo[s][1]);
+    }
+  }
+
+  // Online softmax, one running max per head updated once per page
+  float mt0 = -INFINITY, mt1 = -INFINITY;
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+    if (partial) {
+      if (mb * 16 + g >= n_valid) sc[mb][0] = sc[mb][1] = -INFINITY;
+      if (mb * 16 + g + 8 >= n_valid) sc[mb][2] = sc[mb][3] = -INFINITY;
+    }
+    mt0 = fmaxf(mt0, fmaxf(sc[mb][0], sc[mb][2]));
+    mt1 = fmaxf(mt1, fmaxf(sc[mb][1], sc[mb][3]));
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, o));
+    mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
+  }
+  const float mn0 = fmaxf(m[0], mt0), mn1 = fmaxf(m[1], mt1);
+  const float al0 = exp2f(m[0] - mn0), al1 = exp2f(m[1] - mn1);
+  m[0] = mn0;
+  m[1] = mn1;
+  // p as hi + lo bf16 B operands (k = token, n = head)
+  float ps0 = 0.f, ps1 = 0.f;
+  uint32_t ph[MB][2], pl[MB][2];
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+    const float p0 = exp2f(sc[mb][0] - mn0), p1 = exp2f(sc[mb][1] - mn1);
+    const float p2 = exp2f(sc[mb][2] - mn0), p3 = exp2f(sc[mb][3] - mn1);
+    ps0 += p0 + p2;
+    ps1 += p1 + p3;
+    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+    ph[mb][0] = movmatrix_trans(h01);
+    ph[mb][1] = movmatrix_trans(h23);
+    pl[mb][0] = movmatrix_trans(pack_bf16x2(p0 - bf_lo(h01), p1 - bf_hi(h01)));
+    pl[mb][1] = movmatrix_trans(pack_bf16x2(p2 - bf_lo(h23), p3 - bf_hi(h23)));
+  }
+  l[0] = fmaf(l[0], al0, ps0);
+  l[1] = fmaf(l[1], al1, ps1);
+
+  // Phase B
+#pragma unroll
+  for (int vb = 0; vb < VB; ++vb) {
+    acc[vb][0] *= al0;
+    acc[vb][1] *= al1;
+    acc[vb][2] *= al0;
+    acc[vb][3] *= al1;
+  }
+  const int vrow = ((lane >> 4) << 3) + (lane & 7), vhalf = (lane >> 3) & 1;
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+    if (mb * 16 < n_valid) {
+#pragma unroll
+      for (int vb = 0; vb < VB; ++vb) {
+        if (vb < nvb) {
+          const int c = min(2 * vb + vhalf, ncv - 1);
+          uint32_t a[4];
+          ldsm_x4_trans(vbase + (uint32_t)((c * TT + mb * 16 + vrow) * 16), a);
+          if (partial) {
+            const int k0 = mb * 16 + 2 * t;
+            a[0] = mask_tokens(a[0], k0, n_valid);
+            a[1] = mask_tokens(a[1], k0, n_valid);
+            a[2] = mask_tokens(a[2], k0 + 8, n_valid);
+            a[3] = mask_tokens(a[3], k0 + 8, n_valid);
+          }
+          mma_bf16_16816(acc[vb], a, ph[mb][0], ph[mb][1]);
+          mma_bf16_16816(acc[vb], a, pl[mb][0], pl[mb][1]);
+        }
+      }
+    }
+  }
+}
+
+// The warp's (m, l, acc) of the tensor-core path -> record (m[G], l[G], acc [G][rvd]).
+template <int G, int VB>
+__device__ inline void write_record_mma(float* rec, int rvd, const float (&m)[2],
+                                        const float (&l)[2], const float (&acc)[VB][4],
+                                        int lane) {
+  const int g = lane >> 2, t = lane & 3, H = hdr_floats(G);
+  float l0 = l[0], l1 = l[1];
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  const int h0 = 2 * t, h1 = 2 * t + 1;
+  if (g == 0) {
+    if (h0 < G) { rec[h0] = m[0]; rec[G + h0] = l0; }
+    if (h1 < G) { rec[h1] = m[1]; rec[G + h1] = l1; }
+  }
+#pragma unroll
+  for (int vb = 0; vb < VB; ++vb)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int d = vb * 16 + g + 8 * r;
+      if (d < rvd) {
+        if (h0 < G) rec[H + h0 * rvd + d] = acc[vb][2 * r];
+        if (h1 < G) rec[H + h1 * rvd + d] = acc[vb][2 * r + 1];
+      }
+    }
+}
+
 // ------------------------------------------------------------ q-fold kernel
 constexpr int kFoldThreads = 128;  // small, so q-fold CTAs fit beside split CTAs
 constexpr int kFoldSplit = 2;      // CTAs per unit, each folding a share of the columns
@@ -503,8 +681,12 @@ __device__ void anchor_tile(const uint4* kch, int n_valid, const float* qv, floa
 }
 
 // ------------------------------------------------------------ split kernel
-template <typename T, int G>
-__global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
+// kDense: the ring carries full-rank pages (dense baseline) instead of latent
+// pages; KS / VB: rank class of the tensor-core tiles (bf16 only).
+// 200 registers: two warps per SM sub-partition, with room left for a q-fold
+// CTA beside the split CTA.
+template <typename T, int G, bool kDense, int KS, int VB>
+__global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
   constexpr int CE = Elem<T>::CE;
   constexpr int NP = CE / 2;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -537,9 +719,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
   }
   __syncthreads();
 
-  const bool anchors = anchor_mode(a.fr, a.bt_fr);
   // The ring carries the latent pages, or the full-rank pages in dense mode.
-  const int rsp = a.codes ? 0 : 1;
+  constexpr int rsp = kDense ? 1 : 0;
   const int* rstart = rsp == 0 ? start_lat : start_fr;
   const int rtot = rstart[a.B];
   const int lo = range_lo(c, rtot, a.C), hi = range_lo(c + 1, rtot, a.C), N = hi - lo;
@@ -622,7 +803,10 @@ __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
 
   if (warp == kAnchorWarp) {
     // ---------------- anchor warp: this CTA's share of the anchor tiles
-    if (!anchors) return;
+    if constexpr (kDense) {
+      return;
+    } else {
+    if (!anchor_mode(a.fr, a.bt_fr)) return;
     const int tot = start_fr[a.B];
     const int flo = range_lo(c, tot, a.C), fhi = range_lo(c + 1, tot, a.C);
     const int rec_stride = hdr_floats(G) + G * kHeadDim;
@@ -653,9 +837,11 @@ __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
       t = ce;
     }
     return;
+    }
   }
 
-  // ---------------- consumers
+  // ---------------- consumers (bf16 pages on the tensor cores, fp32 on SIMT)
+  constexpr bool kTensorTiles = std::is_same<T, __nv_bfloat16>::value;
   const int w = warp - kFirstConsumer;
   const int nck = rsp == 0 ? a.rk / CE : kHeadDim / CE;
   const int ncv = rsp == 0 ? a.rv / CE : kHeadDim / CE;
@@ -672,36 +858,59 @@ __global__ void __launch_bounds__(kThreads, 1) split_kernel(DecodeArgs a) {
     const int unit = b * a.H_kv + kvh, ustart = t - i0, ce = min(hi, ustart + tiles);
     const int ntok = space_tokens(a, rsp, b);
     fetch_queries_warp<G>(a, rsp, b, kvh, qv, lane);
-    float m[G], l[G];
-    float2 acc[G][NP];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m[h] = -INFINITY; l[h] = 0.f;
-#pragma unroll
-      for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
-    }
     const int k0 = t - lo;
-    for (int tt = t + ((w - k0 % kConsumers) + kConsumers) % kConsumers; tt < ce;
-         tt += kConsumers) {
+    const int first = t + ((w - k0 % kConsumers) + kConsumers) % kConsumers;
+    // Wait (bounded) for tile tt of the ring; nullptr on timeout.
+    auto acquire = [&](int tt) -> const uint4* {
       const int k = tt - lo, s = k % a.NS, n = k / a.NS;
       if (!tag_wait_bounded(tag + s, k) || !mbar_wait_bounded(&full[s], n & 1)) {
         *a.err = kErrTimeout;
         *fail = 1;
-        break;
+        return nullptr;
       }
-      const int it = tt - ustart;
-      const uint4* st = reinterpret_cast<const uint4*>(ring + (size_t)s * a.stage_bytes);
-      if (rsp == 0)
-        process_tile<T, G, kLatPage>(st, min(kLatPage, ntok - it * kLatPage), nck, ncv, TS, qv,
-                                     qdim, pbuf, m, l, acc, lane);
-      else
-        process_tile<T, G, kFrTile>(st, min(kFrTile, ntok - it * kFrTile), nck, ncv, TS, qv,
-                                    qdim, pbuf, m, l, acc, lane);
-      if (lane == 0) mbar_arrive(&empty[s]);
+      return reinterpret_cast<const uint4*>(ring + (size_t)s * a.stage_bytes);
+    };
+    auto release = [&](int tt) {
+      if (lane == 0) mbar_arrive(&empty[(tt - lo) % a.NS]);
+    };
+    float* rec = part + ((size_t)(unit + c) * kConsumers + w) * rec_stride;
+    if constexpr (kTensorTiles) {
+      constexpr int TT = kDense ? kFrTile : kLatPage;
+      QFrag<KS> qf;
+      load_qfrag<G, KS>(qv, qdim, lane, qf);
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, acc[VB][4];
+#pragma unroll
+      for (int vb = 0; vb < VB; ++vb)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[vb][i] = 0.f;
+      for (int tt = first; tt < ce; tt += kConsumers) {
+        const uint4* st = acquire(tt);
+        if (!st) break;
+        process_tile_mma<TT, KS, VB>(st, min(TT, ntok - (tt - ustart) * TT), nck, ncv, qf, m, l,
+                                     acc, lane);
+        release(tt);
+      }
+      // This warp's record for (unit, CTA); m = -inf when it had no tile.
+      write_record_mma<G, VB>(rec, rvd, m, l, acc, lane);
+    } else {
+      float m[G], l[G];
+      float2 acc[G][NP];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        m[h] = -INFINITY; l[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
+      }
+      for (int tt = first; tt < ce; tt += kConsumers) {
+        const uint4* st = acquire(tt);
+        if (!st) break;
+        constexpr int TT = kDense ? kFrTile : kLatPage;
+        process_tile<T, G, TT>(st, min(TT, ntok - (tt - ustart) * TT), nck, ncv, TS, qv, qdim,
+                               pbuf, m, l, acc, lane);
+        release(tt);
+      }
+      write_record<T, G>(rec, rvd, TS, ncv, m, l, acc, lane);
     }
-    // This warp's record for (unit, CTA); m = -inf when it had no tile.
-    write_record<T, G>(part + ((size_t)(unit + c) * kConsumers + w) * rec_stride, rvd, TS, ncv,
-                       m, l, acc, lane);
     t = ce;
     if (*fail) break;
   }
@@ -795,7 +1004,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     mbar_arrive_expect_tx(&bars[1], pv_bytes);
     bulk_g2s(pv, P, pv_bytes, &bars[1]);
   }
-  pdl_wait();  // every record of the split kernel is visible
+  // seq_len was final before the q-fold started (an ordinary launch), so the
+  // record ranges can be worked out before the split grid completes.
   if (tid < 32) build_prefix(a, start_lat, start_fr);
   __syncthreads();
   const bool anchors = anchor_mode(a.fr, a.bt_fr);
@@ -823,36 +1033,54 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
   for (int i = 0; i < kPer; ++i) { lacc[i] = 0.f; facc[i] = 0.f; }
 #pragma unroll
   for (int g = 0; g < G; ++g) ls[g] = 0.f;
+  // When both spaces' records fit in the buffer together (the usual case),
+  // both copies are in flight at once and there is a single wait.
+  const int S0 = H + G * rvs[0], S1 = H + G * rvs[1];  // floats per record
+  const int n0 = ncta[0] * per[0], n1 = ncta[1] * per[1];
+  const bool fused = n0 + n1 <= kMergeMaxRec && (n0 * S0 + n1 * S1) * 4 <= kMergeBuf;
+  pdl_wait();  // every record of the split kernel is visible
+  if (fused && tid == 0 && n0 + n1 > 0) {
+    mbar_arrive_expect_tx(&bars[0], (uint32_t)((n0 * S0 + n1 * S1) * 4));
+    if (n0)
+      bulk_g2s(recb, parts[0] + (size_t)(unit + c0[0]) * per[0] * S0, (uint32_t)(n0 * S0 * 4),
+               &bars[0]);
+    if (n1)
+      bulk_g2s(recb + n0 * S0, parts[1] + (size_t)(unit + c0[1]) * per[1] * S1,
+               (uint32_t)(n1 * S1 * 4), &bars[0]);
+  }
   int chunk = 0;
   bool ok = true;
   for (int sp = 0; sp < 2 && ok; ++sp) {
-    const int n = ncta[sp] * per[sp];
-    const int S = H + G * rvs[sp];  // floats per record
-    const int cap = min(kMergeMaxRec, kMergeBuf / (S * 4));
+    const int n = sp ? n1 : n0;
+    const int S = sp ? S1 : S0;
+    const int cap = fused ? n : min(kMergeMaxRec, kMergeBuf / (S * 4));
     const float* base = parts[sp] + (size_t)(unit + c0[sp]) * per[sp] * S;
+    const float* rb = fused && sp ? recb + n0 * S0 : recb;
     for (int q0 = 0; q0 < n; q0 += cap) {
       const int nq = min(cap, n - q0);
-      if (tid == 0) {
+      if (!fused && tid == 0) {
         mbar_arrive_expect_tx(&bars[0], (uint32_t)(nq * S * 4));
         bulk_g2s(recb, base + (size_t)q0 * S, (uint32_t)(nq * S * 4), &bars[0]);
       }
-      // a record is valid when its CTA's tile range was not empty
       float mx[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
-      const bool landed = mbar_wait_bounded(&bars[0], chunk & 1);
-      ++chunk;
-      if (!__syncthreads_and(landed)) {
-        ok = false;
-        break;
+      if (!fused || chunk == 0) {
+        const bool landed = mbar_wait_bounded(&bars[0], chunk & 1);
+        ++chunk;
+        if (!__syncthreads_and(landed)) {
+          ok = false;
+          break;
+        }
       }
+      // a record is valid when its CTA's tile range was not empty
       for (int x = tid; x < nq; x += kMergeThreads) {
         const int cc = c0[sp] + (q0 + x) / per[sp];
         const int v = range_lo(cc, total[sp], a.C) != range_lo(cc + 1, total[sp], a.C);
         vflag[x] = v;
         if (v)
 #pragma unroll
-          for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], recb[x * S + g]);
+          for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], rb[x * S + g]);
       }
       block_reduce_heads<G, true>(mx, red, Ah, tid);
       if (tid < G) {
@@ -866,11 +1094,11 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
       for (int x = tid; x < nq; x += kMergeThreads)
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float m = recb[x * S + g];
+          const float m = rb[x * S + g];
           float w = 0.f;
           if (vflag[x] && m > -INFINITY) {
             w = exp2f(m - Mh[g]);
-            ls[g] = fmaf(w, recb[x * S + G + g], ls[g]);
+            ls[g] = fmaf(w, rb[x * S + G + g], ls[g]);
           }
           wts[x * G + g] = w;
         }
@@ -883,7 +1111,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
         const int E = sp == 0 ? E_lat : E_fr;
         if (e < E) {
           const int g = e / rvs[sp];
-          const float* col = recb + H + e;
+          const float* col = rb + H + e;
           float s0 = 0.f, s1 = 0.f;
           int x = 0;
           for (; x + 1 < nq; x += 2) {
@@ -895,7 +1123,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
           else facc[i] += s0 + s1;
         }
       }
-      __syncthreads();  // the next chunk overwrites recb
+      __syncthreads();  // the next chunk overwrites recb, vflag and wts
     }
   }
   if (!ok) {
@@ -1007,6 +1235,16 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
+// The split kernel built for this call: dense or latent ring; for bf16 latent
+// pages the smallest rank class that holds (r_k, r_v).
+template <typename T, int G>
+static const void* split_fn(const DecodeArgs& a) {
+  if (!a.codes) return (const void*)split_kernel<T, G, true, 8, 8>;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+    if (a.rk <= 64 && a.rv <= 32) return (const void*)split_kernel<T, G, false, 4, 2>;
+  return (const void*)split_kernel<T, G, false, 8, 8>;
+}
+
 template <typename T, int G>
 static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st) {
   // Keep SMs in the large-shared-memory configuration while the q-fold runs,
@@ -1015,14 +1253,14 @@ static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st) {
                        (int)cudaSharedmemCarveoutMaxShared);
   qfold_kernel<T, G><<<a.B * a.H_kv * kFoldSplit, kFoldThreads, 0, st>>>(a);
   if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
-  if (cudaFuncSetAttribute(split_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           p.smem) != cudaSuccess)
+  const void* split = split_fn<T, G>(a);
+  if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) !=
+      cudaSuccess)
     return LRKV_ERR_CUDA;
-  cudaFuncSetAttribute(split_kernel<T, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+  cudaFuncSetAttribute(split, cudaFuncAttributePreferredSharedMemoryCarveout,
                        (int)cudaSharedmemCarveoutMaxShared);
   void* args[] = {&a};
-  if (launch_pdl((const void*)split_kernel<T, G>, dim3(p.C), dim3(kThreads), p.smem, st, args) !=
-      cudaSuccess)
+  if (launch_pdl(split, dim3(p.C), dim3(kThreads), p.smem, st, args) != cudaSuccess)
     return LRKV_ERR_CUDA;
   if (cudaFuncSetAttribute(merge_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            p.merge_smem) != cudaSuccess)
