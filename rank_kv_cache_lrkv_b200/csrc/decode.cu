@@ -919,7 +919,7 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
 // ------------------------------------------------------------ merge kernel
 // Shared-memory plan of the merge kernel (byte offsets from the base).
 struct MergePlan {
-  int pv, recb, fin, mh, ah, lh, red, wts, vflag, starts, bars, total;
+  int pvt, recb, fin, mh, lh, ah, mm, ll, wts, starts, bars, total;
 };
 __host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B) {
   MergePlan p;
@@ -930,82 +930,80 @@ __host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B) 
     off += bytes;
     return at;
   };
-  p.pv = take(lat ? kHeadDim * rv * 4 : 0, 128);
+  p.pvt = take(lat ? rv * (kHeadDim + 1) * 4 : 0, 16);
   p.recb = take(kMergeBuf, 128);
   p.fin = take(G * kHeadDim * 4, 16);
   p.mh = take(32, 16);
-  p.ah = take(32, 16);
   p.lh = take(32, 16);
-  p.red = take((kMergeThreads / 32) * G * 4, 16);
+  p.ah = take(32, 16);
+  p.mm = take(kMergeMaxRec * G * 4, 16);
+  p.ll = take(kMergeMaxRec * G * 4, 16);
   p.wts = take(kMergeMaxRec * G * 4, 16);
-  p.vflag = take(kMergeMaxRec * 4, 16);
   p.starts = take(2 * (B + 1) * 4, 8);
-  p.bars = take(16, 8);
+  p.bars = take(8, 8);
   p.total = off;
   return p;
 }
 
-// Block-wide reduction of one value per head; the result lands in dst[G].
-template <int G, bool kMax>
-__device__ inline void block_reduce_heads(float (&v)[G], float* red, float* dst, int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
+// sum over x < n of w[x * G] * col[x * S], eight loads in flight
+template <int G>
+__device__ __forceinline__ float weighted_column(const float* col, int S, const float* w, int n) {
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+  int x = 0;
+#pragma unroll 2
+  for (; x + 4 <= n; x += 4)
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float r = kMax ? warp_max(v[g]) : warp_sum(v[g]);
-    if (lane == 0) red[warp * G + g] = r;
-  }
-  __syncthreads();
-  if (tid < G) {
-    float r = kMax ? -INFINITY : 0.f;
-    for (int w = 0; w < kMergeThreads / 32; ++w)
-      r = kMax ? fmaxf(r, red[w * G + tid]) : r + red[w * G + tid];
-    dst[tid] = r;
-  }
-  __syncthreads();
+    for (int u = 0; u < 4; ++u) s[u] = fmaf(w[(x + u) * G], col[(x + u) * S], s[u]);
+  for (; x < n; ++x) s[0] = fmaf(w[x * G], col[x * S], s[0]);
+  return (s[0] + s[1]) + (s[2] + s[3]);
 }
 
 // Per unit, over every record (m, l, acc) of both spaces:
 //   M_g = max m,  w = exp2(m - M_g),  L_g = sum w l,
 //   lat = sum_latent w acc,  fr = sum_full-rank w acc,
 //   o = (P_v lat + fr) / L_g   (0 where L_g = 0: a sequence with no tokens).
-// A unit's records sit in consecutive slots of each space, so they arrive in
-// shared memory by bulk copies (chunks of kMergeBuf bytes, merged online with
-// a running max), as does the unit's P_v block, fetched before the wait for
-// the split grid since it does not depend on it.
+// A unit's records sit in consecutive slots of each space and arrive in
+// shared memory by bulk copies: both spaces at once when they fit in
+// kMergeBuf bytes (the usual case), else space by space in chunks merged
+// online with a running max.  Everything that does not depend on the split
+// grid (the sequence prefix, the record ranges, the unit's P_v block,
+// transposed for conflict-free reads) is done before waiting for it.
 template <typename T, int G>
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const MergePlan mp = merge_plan(a.rv, a.codes != nullptr, G, a.B);
-  float* pv = reinterpret_cast<float*>(smem + mp.pv);        // [128][r_v]
+  float* pvt = reinterpret_cast<float*>(smem + mp.pvt);      // [r_v][128 + 1]
   float* recb = reinterpret_cast<float*>(smem + mp.recb);    // records of one chunk
   float* fin_lat = reinterpret_cast<float*>(smem + mp.fin);  // [G][r_v]
   float* Mh = reinterpret_cast<float*>(smem + mp.mh);        // running max per head
+  float* Lh = reinterpret_cast<float*>(smem + mp.lh);        // running denominator
   float* Ah = reinterpret_cast<float*>(smem + mp.ah);        // rescale of this chunk
-  float* Lh = reinterpret_cast<float*>(smem + mp.lh);
-  float* red = reinterpret_cast<float*>(smem + mp.red);
-  float* wts = reinterpret_cast<float*>(smem + mp.wts);      // [record][G]
-  int* vflag = reinterpret_cast<int*>(smem + mp.vflag);
+  float* mm = reinterpret_cast<float*>(smem + mp.mm);        // [record][G]
+  float* ll = reinterpret_cast<float*>(smem + mp.ll);
+  float* wts = reinterpret_cast<float*>(smem + mp.wts);
   int* start_lat = reinterpret_cast<int*>(smem + mp.starts);
   int* start_fr = start_lat + (a.B + 1);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + mp.bars);  // [0] records, [1] P_v
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + mp.bars);
 
   const int unit = blockIdx.x, b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
-  const float* P = a.codes ? a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv
-                           : nullptr;
-  const uint32_t pv_bytes = (uint32_t)(kHeadDim * a.rv * 4);
+  const int warp = tid >> 5, lane = tid & 31;
+  constexpr int kPT = kHeadDim + 1;  // padded row of the transposed basis
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    mbar_init(bar, 1);
     mbar_fence_init();
   }
-  if (tid < G) Mh[tid] = -INFINITY;
-  __syncthreads();
-  if (tid == 0 && P) {
-    mbar_arrive_expect_tx(&bars[1], pv_bytes);
-    bulk_g2s(pv, P, pv_bytes, &bars[1]);
+  if (tid < G) {
+    Mh[tid] = -INFINITY;
+    Lh[tid] = 0.f;
   }
-  // seq_len was final before the q-fold started (an ordinary launch), so the
-  // record ranges can be worked out before the split grid completes.
+  if (a.codes) {
+    const float* P = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
+    for (int x = tid; x < kHeadDim * a.rv; x += kMergeThreads) {
+      const int d = x / a.rv, j = x - d * a.rv;
+      pvt[j * kPT + d] = __ldg(P + x);
+    }
+  }
+  // seq_len was final before the q-fold started (an ordinary launch).
   if (tid < 32) build_prefix(a, start_lat, start_fr);
   __syncthreads();
   const bool anchors = anchor_mode(a.fr, a.bt_fr);
@@ -1023,119 +1021,118 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     ncta[sp] = cta_of(us + tiles - 1, total[sp], a.C) - c0[sp] + 1;
   }
   const int per[2] = {kConsumers, anchors ? 1 : kConsumers};
-  const int rvs[2] = {a.rv, kHeadDim};
-  const float* parts[2] = {a.part_lat, a.part_fr};
+  const int S0 = H + G * a.rv, S1 = H + G * kHeadDim;  // floats per record
+  const int n0 = ncta[0] * per[0], n1 = ncta[1] * per[1];
+  const float* src0 = a.part_lat + (size_t)(unit + c0[0]) * per[0] * S0;
+  const float* src1 = a.part_fr + (size_t)(unit + c0[1]) * per[1] * S1;
+  const bool fused = n0 + n1 <= kMergeMaxRec && (n0 * S0 + n1 * S1) * 4 <= kMergeBuf;
+
+  pdl_wait();  // every record of the split kernel is visible
 
   constexpr int kPer = (G * kHeadDim + kMergeThreads - 1) / kMergeThreads;
   const int E_lat = a.codes ? G * a.rv : 0, E_fr = G * kHeadDim;
-  float lacc[kPer], facc[kPer], ls[G];
+  float lacc[kPer], facc[kPer];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) { lacc[i] = 0.f; facc[i] = 0.f; }
-#pragma unroll
-  for (int g = 0; g < G; ++g) ls[g] = 0.f;
-  // When both spaces' records fit in the buffer together (the usual case),
-  // both copies are in flight at once and there is a single wait.
-  const int S0 = H + G * rvs[0], S1 = H + G * rvs[1];  // floats per record
-  const int n0 = ncta[0] * per[0], n1 = ncta[1] * per[1];
-  const bool fused = n0 + n1 <= kMergeMaxRec && (n0 * S0 + n1 * S1) * 4 <= kMergeBuf;
-  pdl_wait();  // every record of the split kernel is visible
-  if (fused && tid == 0 && n0 + n1 > 0) {
-    mbar_arrive_expect_tx(&bars[0], (uint32_t)((n0 * S0 + n1 * S1) * 4));
-    if (n0)
-      bulk_g2s(recb, parts[0] + (size_t)(unit + c0[0]) * per[0] * S0, (uint32_t)(n0 * S0 * 4),
-               &bars[0]);
-    if (n1)
-      bulk_g2s(recb + n0 * S0, parts[1] + (size_t)(unit + c0[1]) * per[1] * S1,
-               (uint32_t)(n1 * S1 * 4), &bars[0]);
+  for (int i = 0; i < kPer; ++i) {
+    lacc[i] = 0.f;
+    facc[i] = 0.f;
   }
-  int chunk = 0;
+  int chunk = 0, sp = 0, q0 = 0;
   bool ok = true;
-  for (int sp = 0; sp < 2 && ok; ++sp) {
-    const int n = sp ? n1 : n0;
-    const int S = sp ? S1 : S0;
-    const int cap = fused ? n : min(kMergeMaxRec, kMergeBuf / (S * 4));
-    const float* base = parts[sp] + (size_t)(unit + c0[sp]) * per[sp] * S;
-    const float* rb = fused && sp ? recb + n0 * S0 : recb;
-    for (int q0 = 0; q0 < n; q0 += cap) {
-      const int nq = min(cap, n - q0);
-      if (!fused && tid == 0) {
-        mbar_arrive_expect_tx(&bars[0], (uint32_t)(nq * S * 4));
-        bulk_g2s(recb, base + (size_t)q0 * S, (uint32_t)(nq * S * 4), &bars[0]);
+  while (true) {
+    // this chunk: latent records [l0, l0 + nl) and full-rank [f0, f0 + nf)
+    int nl = 0, nf = 0, l0 = 0, f0 = 0;
+    if (fused) {
+      if (chunk > 0 || n0 + n1 == 0) break;
+      nl = n0;
+      nf = n1;
+      if (tid == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)((n0 * S0 + n1 * S1) * 4));
+        if (n0) bulk_g2s(recb, src0, (uint32_t)(n0 * S0 * 4), bar);
+        if (n1) bulk_g2s(recb + n0 * S0, src1, (uint32_t)(n1 * S1 * 4), bar);
       }
-      float mx[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
-      if (!fused || chunk == 0) {
-        const bool landed = mbar_wait_bounded(&bars[0], chunk & 1);
-        ++chunk;
-        if (!__syncthreads_and(landed)) {
-          ok = false;
-          break;
-        }
+    } else {
+      const int n = sp ? n1 : n0;
+      if (q0 >= n) {
+        if (sp == 1) break;
+        sp = 1;
+        q0 = 0;
+        continue;
       }
-      // a record is valid when its CTA's tile range was not empty
-      for (int x = tid; x < nq; x += kMergeThreads) {
-        const int cc = c0[sp] + (q0 + x) / per[sp];
-        const int v = range_lo(cc, total[sp], a.C) != range_lo(cc + 1, total[sp], a.C);
-        vflag[x] = v;
-        if (v)
-#pragma unroll
-          for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], rb[x * S + g]);
+      const int S = sp ? S1 : S0;
+      const int nq = min(min(kMergeMaxRec, kMergeBuf / (S * 4)), n - q0);
+      if (sp) { nf = nq; f0 = q0; } else { nl = nq; l0 = q0; }
+      if (tid == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(nq * S * 4));
+        bulk_g2s(recb, (sp ? src1 : src0) + (size_t)q0 * S, (uint32_t)(nq * S * 4), bar);
       }
-      block_reduce_heads<G, true>(mx, red, Ah, tid);
-      if (tid < G) {
-        const float nm = fmaxf(Mh[tid], Ah[tid]);
-        Ah[tid] = nm > -INFINITY ? exp2f(Mh[tid] - nm) : 1.f;
-        Mh[tid] = nm;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int g = 0; g < G; ++g) ls[g] *= Ah[g];
-      for (int x = tid; x < nq; x += kMergeThreads)
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float m = rb[x * S + g];
-          float w = 0.f;
-          if (vflag[x] && m > -INFINITY) {
-            w = exp2f(m - Mh[g]);
-            ls[g] = fmaf(w, rb[x * S + G + g], ls[g]);
-          }
-          wts[x * G + g] = w;
-        }
-      __syncthreads();
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int e = tid + i * kMergeThreads;
-        if (e < E_lat) lacc[i] *= Ah[e / a.rv];
-        if (e < E_fr) facc[i] *= Ah[e / kHeadDim];
-        const int E = sp == 0 ? E_lat : E_fr;
-        if (e < E) {
-          const int g = e / rvs[sp];
-          const float* col = rb + H + e;
-          float s0 = 0.f, s1 = 0.f;
-          int x = 0;
-          for (; x + 1 < nq; x += 2) {
-            s0 = fmaf(wts[x * G + g], col[x * S], s0);
-            s1 = fmaf(wts[(x + 1) * G + g], col[(x + 1) * S], s1);
-          }
-          if (x < nq) s0 = fmaf(wts[x * G + g], col[x * S], s0);
-          if (sp == 0) lacc[i] += s0 + s1;
-          else facc[i] += s0 + s1;
-        }
-      }
-      __syncthreads();  // the next chunk overwrites recb, vflag and wts
+      q0 += nq;
     }
+    const bool landed = mbar_wait_bounded(bar, chunk & 1);
+    ++chunk;
+    if (!__syncthreads_and(landed)) {
+      ok = false;
+      break;
+    }
+    const int nq = nl + nf;
+    const float* rf = recb + nl * S0;  // full-rank records of this chunk
+    // (1) (m, l) per record and head; a record whose CTA had an empty range
+    // was never written and counts as empty
+    for (int i = tid; i < nq * G; i += kMergeThreads) {
+      const int x = i / G, g = i - x * G;
+      const int s = x < nl ? 0 : 1, q = s ? f0 + x - nl : l0 + x;
+      const int cc = c0[s] + q / per[s];
+      const bool v = range_lo(cc, total[s], a.C) != range_lo(cc + 1, total[s], a.C);
+      const float* r = s ? rf + (x - nl) * S1 : recb + x * S0;
+      mm[i] = v ? r[g] : -INFINITY;
+      ll[i] = v ? r[G + g] : 0.f;
+    }
+    __syncthreads();
+    // (2) warp g: head g's running max, weights and denominator
+    if (warp < G) {
+      const int g = warp;
+      float cm = -INFINITY;
+      for (int x = lane; x < nq; x += 32) cm = fmaxf(cm, mm[x * G + g]);
+      cm = warp_max(cm);
+      const float Mo = Mh[g], Mn = fmaxf(Mo, cm);
+      float ls = 0.f;
+      for (int x = lane; x < nq; x += 32) {
+        const float m = mm[x * G + g];
+        const float w = m > -INFINITY ? exp2f(m - Mn) : 0.f;
+        wts[x * G + g] = w;
+        ls = fmaf(w, ll[x * G + g], ls);
+      }
+      ls = warp_sum(ls);
+      if (lane == 0) {
+        const float al = Mn > -INFINITY ? exp2f(Mo - Mn) : 1.f;
+        Ah[g] = al;
+        Mh[g] = Mn;
+        Lh[g] = fmaf(Lh[g], al, ls);
+      }
+    }
+    __syncthreads();
+    // (3) weighted sums of the accumulators
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = tid + i * kMergeThreads;
+      if (e < E_lat) {
+        const int g = e / a.rv;
+        lacc[i] = fmaf(lacc[i], Ah[g], weighted_column<G>(recb + H + e, S0, wts + g, nl));
+      }
+      if (e < E_fr) {
+        const int g = e / kHeadDim;
+        facc[i] = fmaf(facc[i], Ah[g], weighted_column<G>(rf + H + e, S1, wts + nl * G + g, nf));
+      }
+    }
+    __syncthreads();  // the next chunk overwrites recb, mm, ll and wts
   }
   if (!ok) {
     if (tid == 0) {
       *a.err = kErrTimeout;
-      // wait (bounded) for the copies still in flight before leaving
-      mbar_wait_bounded(&bars[0], (chunk - 1) & 1);
-      if (P) mbar_wait_bounded(&bars[1], 0);
+      mbar_wait_bounded(bar, (chunk - 1) & 1);  // the copy still in flight
     }
     return;
   }
-  block_reduce_heads<G, false>(ls, red, Lh, tid);
 
   // o = (P_v lat + fr) / L
 #pragma unroll
@@ -1143,11 +1140,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     const int e = tid + i * kMergeThreads;
     if (e < E_lat) fin_lat[e] = lacc[i];
   }
-  const bool pv_ok = !P || mbar_wait_bounded(&bars[1], 0);
-  if (!__syncthreads_and(pv_ok)) {
-    if (tid == 0) *a.err = kErrTimeout;
-    return;
-  }
+  __syncthreads();
   T* o = static_cast<T*>(a.o) + ((size_t)b * a.H_q + (size_t)kvh * G) * kHeadDim;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
@@ -1155,15 +1148,15 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(DecodeArgs a) {
     if (x >= G * kHeadDim) break;
     const int g = x / kHeadDim, d = x - g * kHeadDim;
     float out = facc[i];
-    if (P) {
-      // rotated start per row keeps the lanes of a warp on distinct banks
-      const float* row = pv + d * a.rv;
+    if (a.codes) {
       const float* lat = fin_lat + g * a.rv;
-      int j = d % a.rv;
-      for (int k = 0; k < a.rv; ++k) {
-        out = fmaf(row[j], lat[j], out);
-        j = j + 1 == a.rv ? 0 : j + 1;
-      }
+      const float* col = pvt + d;
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+      for (int j = 0; j < a.rv; j += 4)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) s[u] = fmaf(col[(j + u) * kPT], lat[j + u], s[u]);
+      out += (s[0] + s[1]) + (s[2] + s[3]);
     }
     const float L = Lh[g];
     o[x] = from_f<T>(L > 0.f ? out / L : 0.f);
