@@ -316,11 +316,14 @@ __device__ __forceinline__ uint32_t mask_tokens(uint32_t x, int k, int n) {
 }
 
 // One page (TT tokens) of a ring stage; running state per lane: m, l for
-// heads 2t and 2t + 1 (l is this lane's partial), acc fragments per 16 value dims.
+// heads 2t and 2t + 1 (l is this lane's partial), acc fragments per 16 value
+// dims, kept apart for the hi and lo halves of p (shorter MMA chains; the
+// record sums them).
 template <int TT, int KS, int VB>
 __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, int nck, int ncv,
                                                  const QFrag<KS>& qf, float (&m)[2],
-                                                 float (&l)[2], float (&acc)[VB][4], int lane) {
+                                                 float (&l)[2], float (&acc)[2][VB][4],
+                                                 int lane) {
   constexpr int MB = TT / 16;
   const int g = lane >> 2, t = lane & 3;
   const uint32_t kbase = smem_u32(kch), vbase = smem_u32(kch + nck * TT);
@@ -328,11 +331,11 @@ __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, 
   const bool partial = n_valid < TT;
 
   // Phase A (an odd last chunk is read twice; its q~ half is zero)
-  float sc[MB][4];
+  float sc[MB][4], sl[MB][4];
 #pragma unroll
   for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sc[mb][i] = 0.f;
+    for (int i = 0; i < 4; ++i) sc[mb][i] = sl[mb][i] = 0.f;
   // (rows of tokens past n_valid are read but masked below)
   const int arow = lane & 15, ahalf = lane >> 4;
 #pragma unroll
@@ -346,9 +349,13 @@ __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, 
 #pragma unroll
       for (int mb = 0; mb < MB; ++mb) mma_bf16_16816(sc[mb], a[mb], qf.hi[s][0], qf.hi[s][1]);
 #pragma unroll
-      for (int mb = 0; mb < MB; ++mb) mma_bf16_16816(sc[mb], a[mb], qf.lo[s][0], qf.lo[s][1]);
+      for (int mb = 0; mb < MB; ++mb) mma_bf16_16816(sl[mb], a[mb], qf.lo[s][0], qf.lo[s][1]);
     }
   }
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[mb][i] += sl[mb][i];
 
   // Online softmax, one running max per head updated once per page
   float mt0 = -INFINITY, mt1 = -INFINITY;
@@ -367,7 +374,7 @@ __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, 
     mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
   }
   const float mn0 = fmaxf(m[0], mt0), mn1 = fmaxf(m[1], mt1);
-  const float al0 = exp2f(m[0] - mn0), al1 = exp2f(m[1] - mn1);
+  const float al0 = ex2_approx(m[0] - mn0), al1 = ex2_approx(m[1] - mn1);
   m[0] = mn0;
   m[1] = mn1;
   // p as hi + lo bf16 B operands (k = token, n = head)
@@ -375,8 +382,8 @@ __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, 
   uint32_t ph[MB][2], pl[MB][2];
 #pragma unroll
   for (int mb = 0; mb < MB; ++mb) {
-    const float p0 = exp2f(sc[mb][0] - mn0), p1 = exp2f(sc[mb][1] - mn1);
-    const float p2 = exp2f(sc[mb][2] - mn0), p3 = exp2f(sc[mb][3] - mn1);
+    const float p0 = ex2_approx(sc[mb][0] - mn0), p1 = ex2_approx(sc[mb][1] - mn1);
+    const float p2 = ex2_approx(sc[mb][2] - mn0), p3 = ex2_approx(sc[mb][3] - mn1);
     ps0 += p0 + p2;
     ps1 += p1 + p3;
     const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
@@ -390,12 +397,14 @@ __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, 
 
   // Phase B
 #pragma unroll
-  for (int vb = 0; vb < VB; ++vb) {
-    acc[vb][0] *= al0;
-    acc[vb][1] *= al1;
-    acc[vb][2] *= al0;
-    acc[vb][3] *= al1;
-  }
+  for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+    for (int vb = 0; vb < VB; ++vb) {
+      acc[hl][vb][0] *= al0;
+      acc[hl][vb][1] *= al1;
+      acc[hl][vb][2] *= al0;
+      acc[hl][vb][3] *= al1;
+    }
   const int vrow = ((lane >> 4) << 3) + (lane & 7), vhalf = (lane >> 3) & 1;
 #pragma unroll
   for (int mb = 0; mb < MB; ++mb) {
@@ -413,8 +422,8 @@ __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, 
             a[2] = mask_tokens(a[2], k0 + 8, n_valid);
             a[3] = mask_tokens(a[3], k0 + 8, n_valid);
           }
-          mma_bf16_16816(acc[vb], a, ph[mb][0], ph[mb][1]);
-          mma_bf16_16816(acc[vb], a, pl[mb][0], pl[mb][1]);
+          mma_bf16_16816(acc[0][vb], a, ph[mb][0], ph[mb][1]);
+          mma_bf16_16816(acc[1][vb], a, pl[mb][0], pl[mb][1]);
         }
       }
     }
@@ -424,7 +433,7 @@ __device__ __forceinline__ void process_tile_mma(const uint4* kch, int n_valid, 
 // The warp's (m, l, acc) of the tensor-core path -> record (m[G], l[G], acc [G][rvd]).
 template <int G, int VB>
 __device__ inline void write_record_mma(float* rec, int rvd, const float (&m)[2],
-                                        const float (&l)[2], const float (&acc)[VB][4],
+                                        const float (&l)[2], const float (&acc)[2][VB][4],
                                         int lane) {
   const int g = lane >> 2, t = lane & 3, H = hdr_floats(G);
   float l0 = l[0], l1 = l[1];
@@ -444,8 +453,8 @@ __device__ inline void write_record_mma(float* rec, int rvd, const float (&m)[2]
     for (int r = 0; r < 2; ++r) {
       const int d = vb * 16 + g + 8 * r;
       if (d < rvd) {
-        if (h0 < G) rec[H + h0 * rvd + d] = acc[vb][2 * r];
-        if (h1 < G) rec[H + h1 * rvd + d] = acc[vb][2 * r + 1];
+        if (h0 < G) rec[H + h0 * rvd + d] = acc[0][vb][2 * r] + acc[1][vb][2 * r];
+        if (h1 < G) rec[H + h1 * rvd + d] = acc[0][vb][2 * r + 1] + acc[1][vb][2 * r + 1];
       }
     }
 }
@@ -878,11 +887,13 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
       constexpr int TT = kDense ? kFrTile : kLatPage;
       QFrag<KS> qf;
       load_qfrag<G, KS>(qv, qdim, lane, qf);
-      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, acc[VB][4];
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, acc[2][VB][4];
 #pragma unroll
-      for (int vb = 0; vb < VB; ++vb)
+      for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[vb][i] = 0.f;
+        for (int vb = 0; vb < VB; ++vb)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[hl][vb][i] = 0.f;
       for (int tt = first; tt < ce; tt += kConsumers) {
         const uint4* st = acquire(tt);
         if (!st) break;
