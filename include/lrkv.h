@@ -74,8 +74,9 @@ enum { LRKV_BF16 = 0, LRKV_F32 = 1 };
  *
  * seq_len[b] counts the tokens appended to sequence b so far; the library
  * advances it.  append_counter[b] is scratch the append kernels use to
- * advance seq_len: zero it once when the cache is created; every completed
- * lrkv_compress leaves it zero again. */
+ * advance seq_len when num_kv_heads > 8 (up to 8 the CTAs of a sequence
+ * form a thread-block cluster and need no counter): zero it once when the
+ * cache is created; every completed lrkv_compress leaves it zero again. */
 typedef struct lrkv_cache {
   int32_t batch;             /* B, 1..LRKV_MAX_BATCH                       */
   int32_t num_kv_heads;      /* H_kv                                       */
@@ -105,6 +106,9 @@ typedef struct lrkv_cache {
  *   P_k    : fp32 basis [Bp][H_kv][128][rank_k] (row-major 128 x r per head);
  *            sequence b uses P_k + b*basis_batch_stride (0 = shared by all).
  *   P_v    : the same for values with rank_v.
+ *   Alignment: k, v, P_k and P_v 16-byte aligned; seq_stride and
+ *            head_stride multiples of 8 elements (bf16) or 4 (fp32);
+ *            basis_batch_stride a multiple of 4 (LRKV_ERR_ARG otherwise).
  * The sink, window slots and codes of each sequence are written; seq_len is
  * advanced by n_tokens.  Returns LRKV_ERR_CAPACITY only when the host can see
  * the overflow (n_tokens larger than the page capacity); the kernels skip

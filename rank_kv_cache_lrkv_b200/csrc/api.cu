@@ -77,6 +77,11 @@ int lrkv_compress(const lrkv_cache* cache, const void* k, const void* v, int32_t
   if (n_tokens < 0) return LRKV_ERR_ARG;
   if (n_tokens == 0) return LRKV_OK;
   if (!k || !v || !P_k || !P_v || basis_batch_stride < 0) return LRKV_ERR_ARG;
+  // token rows are read in 16-byte chunks and the bases four floats at a time
+  const int ce = chunk_elems(cache->dtype);
+  if (!aligned16(k) || !aligned16(v) || seq_stride % ce != 0 || head_stride % ce != 0 ||
+      !aligned16(P_k) || !aligned16(P_v) || basis_batch_stride % 4 != 0)
+    return LRKV_ERR_ARG;
   const long long cap = (long long)cache->max_pages_per_seq * kLatPage + cache->n_sink + cache->window;
   if (n_tokens > cap) return LRKV_ERR_CAPACITY;
   return compress_launch(*cache, k, v, n_tokens, n_new, seq_stride, head_stride, P_k, P_v,

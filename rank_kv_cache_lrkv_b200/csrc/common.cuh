@@ -189,6 +189,34 @@ __device__ inline float warp_sum(float v) {
   return v;
 }
 
+// ---- 16-byte asynchronous copies global -> shared (zero-filled when
+// src_bytes == 0), committed and awaited in groups
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---- thread-block clusters
+__device__ __forceinline__ void cluster_arrive() {  // release: prior accesses ordered first
+  asm volatile("barrier.cluster.arrive;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {  // acquire
+  asm volatile("barrier.cluster.wait;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
 // ---- warp-level bf16 tensor-core tiles (m16n8k16, fp32 accumulate).
 // Fragment ownership, with g = lane / 4 and t = lane % 4:
 //   A (16x16, row-major): a0 (g, 2t..2t+1) a1 (g+8, 2t..) a2 (g, 2t+8..) a3 (g+8, 2t+8..)

@@ -14,6 +14,8 @@
 // input tokens, sink and window writes, and the seq_len advance).  seq_len
 // is advanced by the last CTA of each sequence to finish (a per-sequence
 // completion counter, reset to zero by that CTA).
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -67,103 +69,159 @@ __device__ inline long long code_off(const AppendArgs& a, int b, int kvh, int j,
          jj % CE;
 }
 
-// Codes of one token held in shared memory (xk, xv fp32) -> pages.  The
-// 128-long dot products are split over 4 row segments so every thread has
-// independent loads in flight; red holds [4][r_k + r_v] partial sums.
-constexpr int kSeg = 4;
+// Page of latent index j of sequence b (-1 when past the block table or
+// out of the pool), and the element offset of code dim jj of that token.
+__device__ inline int latent_page(const AppendArgs& a, int b, int j) {
+  const int pi = j / kLatPage;
+  if (pi >= a.maxp) return -1;
+  const int page = a.bt[(size_t)b * a.maxp + pi];
+  return page >= 0 && page < a.num_pages ? page : -1;
+}
 template <typename T>
-__device__ void project_one(const AppendArgs& a, int b, int kvh, int j, const float* xk,
-                            const float* xv, float* red) {
-  const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
-  const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
-  const int NJ = a.rk + a.rv;
-  constexpr int rows = kHeadDim / kSeg;
-  for (int task = threadIdx.x; task < kSeg * NJ; task += blockDim.x) {
-    const int seg = task / NJ, o = task - seg * NJ;
-    const bool isk = o < a.rk;
-    const int jj = isk ? o : o - a.rk;
-    const int r = isk ? a.rk : a.rv;
-    const float* P = (isk ? Pk : Pv) + (size_t)seg * rows * r + jj;
-    const float* x = (isk ? xk : xv) + seg * rows;
-    float s = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < rows; ++i) s = fmaf(P[(size_t)i * r], x[i], s);
-    red[seg * NJ + o] = s;
-  }
-  __syncthreads();
-  for (int o = threadIdx.x; o < NJ; o += blockDim.x) {
-    float s = 0.f;
-#pragma unroll
-    for (int seg = 0; seg < kSeg; ++seg) s += red[seg * NJ + o];
-    const bool isk = o < a.rk;
-    const int jj = isk ? o : o - a.rk;
-    const long long off = code_off<T>(a, b, kvh, j, jj, isk ? 0 : 1);
-    if (off >= 0) static_cast<T*>(a.codes)[off] = from_f<T>(s);
-  }
+__device__ inline long long code_off_in(const AppendArgs& a, int page, int kvh, int j, int jj,
+                                        int isv) {
+  constexpr int CE = Elem<T>::CE;
+  const int nch = (a.rk + a.rv) / CE;
+  const int chunk = isv * (a.rk / CE) + jj / CE;
+  return ((((long long)page * a.H_kv + kvh) * nch + chunk) * kLatPage + j % kLatPage) * CE +
+         jj % CE;
 }
 
-template <typename T>
+constexpr int kRowBatch = 16;  // token rows projected per pass
+// Dynamic shared memory of append_kernel: the unit's basis [128][r_k + r_v]
+// fp32, rows [kRowBatch][k, v][128] fp32, partial sums [256], and a page per row.
+inline size_t append_smem_bytes(int rk, int rv) {
+  return ((size_t)kHeadDim * (rk + rv) + (size_t)kRowBatch * 2 * kHeadDim + 256 + kRowBatch) * 4;
+}
+
+// One CTA per (KV head, sequence).  Latency matters here (a decode step
+// appends one token), so the loads that do not depend on each other are in
+// flight together: seq_len with the unit's basis, then the rows to project
+// with their block-table entries.  kCluster: the CTAs of one sequence form a
+// cluster; each arrives on the cluster barrier once it has read seq_len, and
+// rank 0 waits on it before advancing seq_len, so no CTA can read the new
+// value.  Without clusters (H_kv > 8) the last CTA to finish, found with a
+// per-sequence counter, advances seq_len.
+template <typename T, bool kCluster>
 __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_latent) {
-  __shared__ float xk[kHeadDim], xv[kHeadDim];
-  __shared__ float red[kSeg * 2 * kHeadDim];
-  const int kvh = blockIdx.x, b = blockIdx.y;
-  const int L0 = a.seq_len[b], L1 = L0 + appended(a.n_new, a.n, b);
+  constexpr int CE = Elem<T>::CE, NC = kHeadDim / CE;
+  extern __shared__ __align__(16) float sm[];
+  const int NJ = a.rk + a.rv;
+  float* Ps = sm;                                                      // [128][NJ]
+  float* xs = Ps + kHeadDim * NJ;                                      // [row][k, v][128]
+  float* red = xs + kRowBatch * 2 * kHeadDim;                          // [seg][NJ]
+  int* pg = reinterpret_cast<int*>(red + 256);                         // [row]
+  const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+
+  // 1. seq_len, and the basis into shared memory ([i][o]: P_k columns then P_v)
+  const int L0 = __ldcg(a.seq_len + b);
+  if constexpr (kCluster) cluster_arrive();
+  {
+    const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
+    const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
+    const int n4 = NJ / 4;
+#pragma unroll 4
+    for (int x = tid; x < kHeadDim * n4; x += blockDim.x) {
+      const int i = x / n4, o = 4 * (x - i * n4);
+      const float4 v = o < a.rk ? __ldg(reinterpret_cast<const float4*>(Pk + i * a.rk + o))
+                                : __ldg(reinterpret_cast<const float4*>(Pv + i * a.rv + o - a.rk));
+      reinterpret_cast<float4*>(Ps)[x] = v;
+    }
+  }
+  const int L1 = L0 + appended(a.n_new, a.n, b);
   const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
   const T* kin = static_cast<const T*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
   const T* vin = static_cast<const T*>(a.v) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
   const T* anc = static_cast<const T*>(a.anchors);
 
-  // 1. evictions from the ring (token index < L0), oldest first.
+  // 2. rows that become latent: evictions from the ring (token < L0, oldest
+  // first), then input tokens that go straight to latent (small n only)
   const int ev_lo = a.n_sink + s0.lat, ev_hi = min(L0, a.n_sink + s1.lat);
-  for (int t = ev_lo; t < ev_hi; ++t) {
-    const int slot = a.n_sink + (t - a.n_sink) % a.W;
-    for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x) {
-      xk[d] = to_f<T>(anc[anchor_off<T>(a, b, kvh, slot, d, 0)]);
-      xv[d] = to_f<T>(anc[anchor_off<T>(a, b, kvh, slot, d, 1)]);
+  const int in_lo = max(L0, a.n_sink + s0.lat), in_hi = a.n_sink + s1.lat;
+  const int n_ev = max(0, ev_hi - ev_lo), n_in = do_input_latent ? max(0, in_hi - in_lo) : 0;
+  const int nrows = n_ev + n_in;
+  auto token_of = [&](int r) { return r < n_ev ? ev_lo + r : in_lo + (r - n_ev); };
+  for (int r0 = 0; r0 < nrows; r0 += kRowBatch) {
+    const int nr = min(kRowBatch, nrows - r0);
+    for (int x = tid; x < nr * 2 * NC; x += blockDim.x) {
+      const int rr = x / (2 * NC), rem = x - rr * 2 * NC, isv = rem / NC, ch = rem - isv * NC;
+      const int r = r0 + rr, t = token_of(r);
+      const T* src;
+      if (r < n_ev) {
+        const int slot = a.n_sink + (t - a.n_sink) % a.W;
+        src = anc + anchor_off<T>(a, b, kvh, slot, ch * CE, isv);
+      } else {
+        src = (isv ? vin : kin) + (size_t)(t - L0) * kHeadDim + ch * CE;
+      }
+      unpack_chunk<T>(__ldcg(reinterpret_cast<const uint4*>(src)),
+                      xs + (rr * 2 + isv) * kHeadDim + ch * CE);
     }
+    if (tid < nr) pg[tid] = latent_page(a, b, token_of(r0 + tid) - a.n_sink);
     __syncthreads();
-    project_one<T>(a, b, kvh, t - a.n_sink, xk, xv, red);
-    __syncthreads();
-  }
-  // 2. input tokens that go straight to latent (small n only).
-  if (do_input_latent) {
-    const int in_lo = max(L0, a.n_sink + s0.lat), in_hi = a.n_sink + s1.lat;
-    for (int t = in_lo; t < in_hi; ++t) {
-      for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x) {
-        xk[d] = to_f<T>(kin[(size_t)(t - L0) * kHeadDim + d]);
-        xv[d] = to_f<T>(vin[(size_t)(t - L0) * kHeadDim + d]);
+    // c = P^T x, one row at a time: thread (seg, o) sums the dims of segment
+    // seg for code column o (nseg a power of two with nseg * NJ <= 256)
+    T* codes = static_cast<T*>(a.codes);
+    int nseg = 1;
+    while (nseg * 2 * NJ <= (int)blockDim.x && nseg < 8) nseg *= 2;
+    const int span = kHeadDim / nseg;
+    for (int rr = 0; rr < nr; ++rr) {
+      if (tid < nseg * NJ) {
+        const int seg = tid / NJ, o = tid - seg * NJ, isv = o < a.rk ? 0 : 1;
+        const float* x = xs + (rr * 2 + isv) * kHeadDim + seg * span;
+        const float* P = Ps + seg * span * NJ + o;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int i = 0; i < span; i += 4)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) s4[u] = fmaf(P[(i + u) * NJ], x[i + u], s4[u]);
+        red[seg * NJ + o] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       __syncthreads();
-      project_one<T>(a, b, kvh, t - a.n_sink, xk, xv, red);
-      __syncthreads();
+      if (tid < NJ && pg[rr] >= 0) {
+        float c = 0.f;
+        for (int seg = 0; seg < nseg; ++seg) c += red[seg * NJ + tid];
+        const int isv = tid < a.rk ? 0 : 1, jj = isv ? tid - a.rk : tid;
+        const int j = token_of(r0 + rr) - a.n_sink;
+        codes[code_off_in<T>(a, pg[rr], kvh, j, jj, isv)] = from_f<T>(c);
+      }
+      __syncthreads();  // red is reused by the next row
     }
+    // (rows and pages are reused by the next batch; ring slots were read
+    // before the window writes below)
   }
-  // 3. sink and window writes (full-rank, verbatim).
+
+  // 3. sink and window writes (full-rank, verbatim), 16-byte chunks
   if (a.n_sink + a.W > 0) {
     T* ancw = static_cast<T*>(a.anchors);
     const int w_lo = max(L0, max(a.n_sink, L1 - a.W));
-    // sink first (t < n_sink), then the window tokens [w_lo, L1)
     const int n_sink_new = max(0, min(a.n_sink, L1) - L0);
     const int n_win_new = max(0, L1 - w_lo);
-    const int total = (n_sink_new + n_win_new) * kHeadDim;
-    for (int x = threadIdx.x; x < total; x += blockDim.x) {
-      const int q = x / kHeadDim, d = x - q * kHeadDim;
+    const int total = (n_sink_new + n_win_new) * 2 * NC;
+    for (int x = tid; x < total; x += blockDim.x) {
+      const int q = x / (2 * NC), rem = x - q * 2 * NC, isv = rem / NC, ch = rem - isv * NC;
       int t, slot;
       if (q < n_sink_new) { t = L0 + q; slot = t; }
       else { t = w_lo + (q - n_sink_new); slot = a.n_sink + (t - a.n_sink) % a.W; }
-      ancw[anchor_off<T>(a, b, kvh, slot, d, 0)] = kin[(size_t)(t - L0) * kHeadDim + d];
-      ancw[anchor_off<T>(a, b, kvh, slot, d, 1)] = vin[(size_t)(t - L0) * kHeadDim + d];
+      const uint4 u = __ldcg(reinterpret_cast<const uint4*>((isv ? vin : kin) +
+                                                            (size_t)(t - L0) * kHeadDim + ch * CE));
+      *reinterpret_cast<uint4*>(ancw + anchor_off<T>(a, b, kvh, slot, ch * CE, isv)) = u;
     }
   }
-  // 4. the last CTA of this sequence advances seq_len.
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const int old = atomicAdd(&a.counter[b], 1);
-    if (old == a.H_kv - 1) {
-      a.seq_len[b] = L1;
-      a.counter[b] = 0;
+
+  // 4. advance seq_len
+  if constexpr (kCluster) {
+    cluster_wait();
+    if (cluster_rank() == 0 && tid == 0) a.seq_len[b] = L1;
+  } else {
+    __syncthreads();
+    if (tid == 0) {
       __threadfence();
+      const int old = atomicAdd(&a.counter[b], 1);
+      if (old == a.H_kv - 1) {
+        a.seq_len[b] = L1;
+        a.counter[b] = 0;
+        __threadfence();
+      }
     }
   }
 }
@@ -205,16 +263,176 @@ __global__ void __launch_bounds__(256) bulk_compress_kernel(AppendArgs a) {
   }
 }
 
+// ---- bf16 prefill compress on the tensor cores
+// c = x P for 64-token tiles of one (sequence, KV head): per warp 16 tokens
+// (m16) x the code columns (n8 blocks) x 128 dims (eight k16 steps), with P
+// split as hi + lo bf16 so the products keep about 16 mantissa bits and
+// accumulate in fp32.  Token rows are staged by cp.async into padded
+// shared-memory rows (two stages), P^T sits in padded rows too, so ldmatrix
+// reads both operands without bank conflicts.
+constexpr int kBulkTile = 64;          // tokens per tile (a warp takes 16)
+constexpr int kBulkTilesPerCta = 8;
+constexpr int kPadRow = kHeadDim + 8;  // bf16 elements per staged row
+
+__host__ __device__ inline int round16(int x) { return (x + 15) / 16 * 16; }
+inline size_t bulk_mma_smem_bytes(int rk, int rv) {
+  return ((size_t)2 * (round16(rk) + round16(rv)) + (size_t)2 * 2 * kBulkTile) * kPadRow * 2;
+}
+
+__global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
+  using bf16 = __nv_bfloat16;
+  extern __shared__ __align__(16) bf16 smb[];
+  const int RK = round16(a.rk), RV = round16(a.rv), NR = RK + RV;
+  bf16* PT = smb;                        // [hi, lo][NR][kPadRow]: rows K codes then V codes
+  bf16* X = smb + 2 * NR * kPadRow;      // [stage][k, v][64][kPadRow]
+  const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int L0 = __ldcg(a.seq_len + b), L1 = L0 + appended(a.n_new, a.n, b);
+  const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
+  // input rows that go straight to latent, relative to L0
+  const int in_lo = max(L0, a.n_sink + s0.lat) - L0, in_hi = a.n_sink + s1.lat - L0;
+  const int rbeg = in_lo + blockIdx.x * kBulkTile * kBulkTilesPerCta;
+  const int rend = min(in_hi, rbeg + kBulkTile * kBulkTilesPerCta);
+  if (rbeg >= rend) return;
+  const int ntiles = (rend - rbeg + kBulkTile - 1) / kBulkTile;
+  const bf16* kin = static_cast<const bf16*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
+  const bf16* vin = static_cast<const bf16*>(a.v) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
+
+  auto stage = [&](int i, int st) {
+    const int t0 = rbeg + i * kBulkTile;
+    for (int x = tid; x < 2 * kBulkTile * 16; x += blockDim.x) {
+      const int isv = x / (kBulkTile * 16), rem = x - isv * kBulkTile * 16;
+      const int row = rem >> 4, ch = rem & 15;
+      const int r = t0 + row;
+      const bool ok = r < rend;  // rows past the range are zero-filled
+      const bf16* src = (isv ? vin : kin) + (size_t)(ok ? r : rbeg) * kHeadDim + ch * 8;
+      cp_async16(X + ((st * 2 + isv) * kBulkTile + row) * kPadRow + ch * 8, src, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  stage(0, 0);
+  // P^T as hi + lo bf16 (rows past r_k / r_v are zero)
+  {
+    const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
+    const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
+    for (int x = tid; x < kHeadDim * NR; x += blockDim.x) {
+      const int i = x / NR, o = x - i * NR;
+      float p = 0.f;
+      if (o < RK) {
+        if (o < a.rk) p = __ldg(Pk + (size_t)i * a.rk + o);
+      } else if (o - RK < a.rv) {
+        p = __ldg(Pv + (size_t)i * a.rv + (o - RK));
+      }
+      const bf16 h = __float2bfloat16_rn(p);
+      PT[o * kPadRow + i] = h;
+      PT[(NR + o) * kPadRow + i] = __float2bfloat16_rn(p - __bfloat162float(h));
+    }
+  }
+  bf16* codes = static_cast<bf16*>(a.codes);
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i & 1;
+    if (i + 1 < ntiles) {
+      stage(i + 1, st ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int tok0 = rbeg + i * kBulkTile + 16 * warp;  // first input row of this warp
+    for (int isv = 0; isv < 2; ++isv) {
+      const int r = isv ? a.rv : a.rk, nb = r / 8, RB = isv ? RK : 0;
+      const bf16* xt = X + ((st * 2 + isv) * kBulkTile + 16 * warp) * kPadRow;
+      uint32_t af[8][4];
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        ldsm_x4(smem_u32(xt + (lane & 15) * kPadRow + 16 * s + (lane >> 4) * 8), af[s]);
+      // pages of the two token rows this lane stores (g and g + 8)
+      int jrow[2], prow[2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int rin = tok0 + g + 8 * h2;
+        jrow[h2] = L0 + rin - a.n_sink;
+        prow[h2] = rin < rend ? latent_page(a, b, jrow[h2]) : -1;
+      }
+      for (int ng = 0; ng < nb; ng += 8) {
+        float acc[8][4];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q][e] = 0.f;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            if (ng + 2 * p < nb) {
+              const int o = RB + 8 * (ng + 2 * p) + (lane & 7) + ((lane >> 4) << 3);
+              const int koff = 16 * s + ((lane >> 3) & 1) * 8;
+              uint32_t bh[4], bl[4];
+              ldsm_x4(smem_u32(PT + o * kPadRow + koff), bh);
+              ldsm_x4(smem_u32(PT + (NR + o) * kPadRow + koff), bl);
+              mma_bf16_16816(acc[2 * p], af[s], bh[0], bh[1]);
+              mma_bf16_16816(acc[2 * p + 1], af[s], bh[2], bh[3]);
+              mma_bf16_16816(acc[2 * p], af[s], bl[0], bl[1]);
+              mma_bf16_16816(acc[2 * p + 1], af[s], bl[2], bl[3]);
+            }
+          }
+        }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (prow[h2] < 0) continue;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (ng + q < nb) {
+              const long long off = code_off_in<bf16>(a, prow[h2], kvh, jrow[h2], 8 * (ng + q) + 2 * t, isv);
+              *reinterpret_cast<uint32_t*>(codes + off) =
+                  pack_bf16x2(acc[q][2 * h2], acc[q][2 * h2 + 1]);
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();  // stage st is refilled by the next iteration's prefetch
+  }
+}
+
 template <typename T>
 static int compress_t(const AppendArgs& a, cudaStream_t st) {
   const bool small = a.n <= kSmallN;
   if (!small) {
-    dim3 g((a.n + kBulkRows - 1) / kBulkRows, a.H_kv, a.B);
-    bulk_compress_kernel<T><<<g, 256, 0, st>>>(a);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      const size_t smem = bulk_mma_smem_bytes(a.rk, a.rv);
+      if (cudaFuncSetAttribute(bulk_compress_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem) != cudaSuccess)
+        return LRKV_ERR_CUDA;
+      const int per = kBulkTile * kBulkTilesPerCta;
+      bulk_compress_mma<<<dim3((a.n + per - 1) / per, a.H_kv, a.B), 128, smem, st>>>(a);
+    } else {
+      dim3 g((a.n + kBulkRows - 1) / kBulkRows, a.H_kv, a.B);
+      bulk_compress_kernel<T><<<g, 256, 0, st>>>(a);
+    }
     if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
   }
-  append_kernel<T><<<dim3(a.H_kv, a.B), 256, 0, st>>>(a, small ? 1 : 0);
-  if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
+  const size_t smem = append_smem_bytes(a.rk, a.rv);
+  const bool cluster = a.H_kv <= 8;
+  const void* fn = cluster ? (const void*)append_kernel<T, true> : (const void*)append_kernel<T, false>;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LRKV_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.H_kv, a.B);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.H_kv;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster ? 1 : 0;
+  int small_in = small ? 1 : 0;
+  void* args[] = {(void*)&a, (void*)&small_in};
+  if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return LRKV_ERR_CUDA;
   return LRKV_OK;
 }
 
