@@ -14,6 +14,7 @@
 // input tokens, sink and window writes, and the seq_len advance).  seq_len
 // is advanced by the last CTA of each sequence to finish (a per-sequence
 // completion counter, reset to zero by that CTA).
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -33,6 +34,7 @@ __device__ inline int appended(const int* n_new, int n, int b) {
 
 struct AppendArgs {
   int B, H_kv, rk, rv, n_sink, W, maxp, num_pages, n, anchor_tiles;
+  int bulk_tpc;  // bulk_compress_mma: 64-token tiles per CTA
   void *codes, *anchors;
   const int* bt;
   int* seq_len;
@@ -271,7 +273,6 @@ __global__ void __launch_bounds__(256) bulk_compress_kernel(AppendArgs a) {
 // shared-memory rows (two stages), P^T sits in padded rows too, so ldmatrix
 // reads both operands without bank conflicts.
 constexpr int kBulkTile = 64;          // tokens per tile (a warp takes 16)
-constexpr int kBulkTilesPerCta = 8;
 constexpr int kPadRow = kHeadDim + 8;  // bf16 elements per staged row
 
 __host__ __device__ inline int round16(int x) { return (x + 15) / 16 * 16; }
@@ -291,8 +292,8 @@ __global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
   const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
   // input rows that go straight to latent, relative to L0
   const int in_lo = max(L0, a.n_sink + s0.lat) - L0, in_hi = a.n_sink + s1.lat - L0;
-  const int rbeg = in_lo + blockIdx.x * kBulkTile * kBulkTilesPerCta;
-  const int rend = min(in_hi, rbeg + kBulkTile * kBulkTilesPerCta);
+  const int rbeg = in_lo + blockIdx.x * kBulkTile * a.bulk_tpc;
+  const int rend = min(in_hi, rbeg + kBulkTile * a.bulk_tpc);
   if (rbeg >= rend) return;
   const int ntiles = (rend - rbeg + kBulkTile - 1) / kBulkTile;
   const bf16* kin = static_cast<const bf16*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
@@ -311,21 +312,28 @@ __global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
     cp_async_commit();
   };
   stage(0, 0);
-  // P^T as hi + lo bf16 (rows past r_k / r_v are zero)
+  // P^T as hi + lo bf16 (rows past r_k / r_v are zero); four columns per
+  // load, eight loads in flight per thread
   {
     const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
     const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
-    for (int x = tid; x < kHeadDim * NR; x += blockDim.x) {
-      const int i = x / NR, o = x - i * NR;
-      float p = 0.f;
+    const int n4 = NR / 4;
+#pragma unroll 8
+    for (int x = tid; x < kHeadDim * n4; x += blockDim.x) {
+      const int i = x / n4, o = 4 * (x - i * n4);
+      float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
       if (o < RK) {
-        if (o < a.rk) p = __ldg(Pk + (size_t)i * a.rk + o);
+        if (o < a.rk) p = __ldg(reinterpret_cast<const float4*>(Pk + (size_t)i * a.rk + o));
       } else if (o - RK < a.rv) {
-        p = __ldg(Pv + (size_t)i * a.rv + (o - RK));
+        p = __ldg(reinterpret_cast<const float4*>(Pv + (size_t)i * a.rv + (o - RK)));
       }
-      const bf16 h = __float2bfloat16_rn(p);
-      PT[o * kPadRow + i] = h;
-      PT[(NR + o) * kPadRow + i] = __float2bfloat16_rn(p - __bfloat162float(h));
+      const float pv[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bf16 h = __float2bfloat16_rn(pv[u]);
+        PT[(o + u) * kPadRow + i] = h;
+        PT[(NR + o + u) * kPadRow + i] = __float2bfloat16_rn(pv[u] - __bfloat162float(h));
+      }
     }
   }
   bf16* codes = static_cast<bf16*>(a.codes);
@@ -404,8 +412,12 @@ static int compress_t(const AppendArgs& a, cudaStream_t st) {
       if (cudaFuncSetAttribute(bulk_compress_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem) != cudaSuccess)
         return LRKV_ERR_CUDA;
-      const int per = kBulkTile * kBulkTilesPerCta;
-      bulk_compress_mma<<<dim3((a.n + per - 1) / per, a.H_kv, a.B), 128, smem, st>>>(a);
+      // about two CTAs per SM over the whole call; each converts its basis once
+      AppendArgs b2 = a;
+      const long long tiles = (long long)((a.n + kBulkTile - 1) / kBulkTile) * a.H_kv * a.B;
+      b2.bulk_tpc = (int)std::min<long long>(64, std::max<long long>(1, (tiles + 295) / 296));
+      const int per = kBulkTile * b2.bulk_tpc;
+      bulk_compress_mma<<<dim3((a.n + per - 1) / per, a.H_kv, a.B), 128, smem, st>>>(b2);
     } else {
       dim3 g((a.n + kBulkRows - 1) / kBulkRows, a.H_kv, a.B);
       bulk_compress_kernel<T><<<g, 256, 0, st>>>(a);
