@@ -230,6 +230,7 @@ def run_ours(args, rank, world):
     import torch
     import torch.distributed as dist
     from rank_kv_cache_lrkv_b200 import lrkv
+    from rank_kv_cache_lrkv_b200 import replicas
     from rank_kv_cache_lrkv_b200 import workloads as wk
 
     base = workload(args.workload)
@@ -237,7 +238,8 @@ def run_ours(args, rank, world):
         base = base.with_(T=args.context)
     W, K = args.warmup, args.steps
     E = 0 if args.no_e2e else min(K, 64)
-    wl = base.with_(n_decode=W + K + E + 2)
+    # this rank's own B sequences (weak scaling; no data-path collective)
+    wl = replicas.shard(base.with_(n_decode=W + K + E + 2), rank, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = wk.layer_inputs(wl)
     qs = wk.layer_queries(wl).to(dev)
@@ -258,7 +260,7 @@ def run_ours(args, rank, world):
     lrkv.compress(cache, Kd[:, :, :wl.T], Vd[:, :, :wl.T], Pk, Pv)
     e1.record()
     torch.cuda.synchronize()
-    prefill_ms = e0.elapsed_time(e1)
+    prefill_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
     # prefill bytes: K and V rows read, codes and anchors written
     n_lat = wl.T - wl.n_sink - wl.window
     prefill_bytes = (wl.B * wl.H_kv * wl.T * 2 * 128 * Kd.element_size()
@@ -304,11 +306,8 @@ def run_ours(args, rank, world):
         g.replay()
         e1.record()
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     assert lrkv.workspace_error(ws) == 0
 
@@ -324,7 +323,7 @@ def run_ours(args, rank, world):
     g2.replay()
     e1.record()
     torch.cuda.synchronize()
-    attn_ms = e0.elapsed_time(e1) / R
+    attn_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / R
     L_now = wl.T + W + K
     abytes = step_bytes(wl, L_now)
     pk = peaks()
@@ -332,7 +331,7 @@ def run_ours(args, rank, world):
     achieved = abytes / (attn_ms * 1e-3) / 1e9
     out = {
         "metric": "latent-KV decode tokens/s and achieved HBM GB/s (fraction of ~8 TB/s) at 1 GPU",
-        "value": round(wl.B * K * world / (ms * 1e-3), 2),
+        "value": round(replicas.aggregate_tokens_per_s(wl.B, K, world, ms), 2),
         "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms / K, 5),
@@ -369,7 +368,7 @@ def run_ours(args, rank, world):
         g3.replay()
         e1.record()
         torch.cuda.synchronize()
-        dms = e0.elapsed_time(e1)
+        dms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
         g4 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g4, capture_error_mode="relaxed"):
             for _ in range(R):
@@ -380,7 +379,7 @@ def run_ours(args, rank, world):
         g4.replay()
         e1.record()
         torch.cuda.synchronize()
-        dattn = e0.elapsed_time(e1) / R
+        dattn = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / R
         db = dense_step_bytes(wl, L_now)
         out["dense_baseline"] = {
             "tokens_per_s": round(wl.B * K / (dms * 1e-3), 2), "ms_per_step": round(dms / K, 5),
@@ -410,13 +409,10 @@ def run_ours(args, rank, world):
             oh[s].copy_(o, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
         es = kd.element_size()
-        out["e2e"] = {"value": round(wl.B * E * world / (ems * 1e-3), 2), "unit": "tokens/s",
+        out["e2e"] = {"value": round(replicas.aggregate_tokens_per_s(wl.B, E, world, ems), 2),
+                      "unit": "tokens/s",
                       "h2d_bytes_per_step": 2 * kd.numel() * es + qd.numel() * es,
                       "d2h_bytes_per_step": o.numel() * es, "steps": E}
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -81,6 +81,7 @@ class Workload:
     oja_decode_every: int = 0
     prefill_oja: bool = False
     append_before_attend: bool = True   # decode token joins the cache first
+    seq0: int = 0            # global index of sequence 0 (a replica's shard)
 
     @property
     def G(self) -> int:
@@ -187,7 +188,7 @@ def stream(wl: Workload, kind: str, layer: int, b: int, kvh: int,
     n = total if n is None else n
     if Q is None:
         Q = head_q(wl, kind, layer, kvh)
-    z = _rng(wl, TAG_ZK if kind == "k" else TAG_ZV, layer, b, kvh).standard_normal(
+    z = _rng(wl, TAG_ZK if kind == "k" else TAG_ZV, layer, wl.seq0 + b, kvh).standard_normal(
         (total, HEAD_DIM))[:n]
     x = (z * spectrum(kind)[None, :]) @ Q
     if kind == "k" and wl.rope_theta is not None:
@@ -224,7 +225,7 @@ def queries(wl: Workload, layer: int, step: int) -> np.ndarray:
     q = np.empty((wl.B, wl.H_q, HEAD_DIM))
     pos = wl.T + step if wl.append_before_attend else wl.T
     for b in range(wl.B):
-        g = _rng(wl, TAG_QUERY, layer, b, step)
+        g = _rng(wl, TAG_QUERY, layer, wl.seq0 + b, step)
         qb = g.standard_normal((wl.H_q, HEAD_DIM)) / np.sqrt(HEAD_DIM)
         if wl.rope_theta is not None:
             qb = rope_rotate(qb, np.full(wl.H_q, pos), wl.rope_theta)
