@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-oja", action="store_true",
+                   help="skip the Oja-update timing of the 28-layer stack")
     p.add_argument("--profile", type=int, default=0,
                    help="profiling run: prefill, then this many eager decode steps "
                         "(append + decode attention), no timing and no JSON line")
@@ -100,6 +102,47 @@ def measured_traffic(wl, L):
             if hashlib.sha256(fh.read()).hexdigest() != h:
                 return None
     return int(round(rec["bytes"] * step_bytes(wl, L) / step_bytes(wl, rec["context"])))
+
+
+def time_oja(lrkv, dev, world):
+    """Prefill Oja update of the 28-layer Qwen3 stack: every (layer, sequence,
+    KV head) key and value stream (2 * 28 * 2 * 8 = 896 streams) over the
+    32,768-token prompt, r = 48, eta = 1e-3, QR every 256 tokens, in one call.
+    The update is sequential per stream, so this is latency-bound: wall time
+    and stream steps per second.  Rows are drawn on the device (Gaussian
+    with the key spectrum exp(-i/16) under a random rotation, in bf16); the
+    cost does not depend on the values."""
+    import torch
+    from rank_kv_cache_lrkv_b200 import replicas
+    from rank_kv_cache_lrkv_b200 import workloads as wk
+    wl = wk.QWEN3_STACK_OJA
+    S, n, r = 2 * wl.layers * wl.B * wl.H_kv, wl.T, wl.r_k
+    g = torch.Generator(device=dev)
+    g.manual_seed(4242)
+    Q, _ = torch.linalg.qr(torch.randn(HEAD_DIM, HEAD_DIM, device=dev, generator=g))
+    spec = torch.exp(-torch.arange(HEAD_DIM, device=dev, dtype=torch.float32) / 16.0)
+    x = torch.empty(S, n, HEAD_DIM, device=dev, dtype=torch.bfloat16)
+    for s0 in range(0, S, 32):
+        z = torch.randn(min(32, S - s0), n, HEAD_DIM, device=dev, generator=g)
+        x[s0:s0 + 32] = ((z * spec) @ Q).to(torch.bfloat16)
+        del z
+    P0, _ = torch.linalg.qr(torch.randn(S, HEAD_DIM, r, device=dev, generator=g))
+    P = P0.contiguous()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lrkv.oja_update(P[:4].clone(), x[:4, :512], wl.oja_eta, wl.oja_qr_every, 0)  # warm-up
+    torch.cuda.synchronize()
+    e0.record()
+    lrkv.oja_update(P, x, wl.oja_eta, wl.oja_qr_every, 0)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ok = bool(torch.isfinite(P).all().item())
+    del x, P, P0
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "streams": S, "tokens_per_stream": n, "rank": r,
+            "eta": wl.oja_eta, "qr_every": wl.oja_qr_every, "ms": round(ms, 3),
+            "stream_steps_per_s": round(S * n / (ms * 1e-3), 1),
+            "us_per_token_step": round(ms * 1e3 / n, 4), "finite": ok}
 
 
 def dense_step_bytes(wl, L):
@@ -352,6 +395,9 @@ def run_ours(args, rank, world):
                              "frac": round(prefill_bytes / (prefill_ms * 1e-3) / 1e9 / hbm, 4)},
         "clocks": clk.summary(),
     }
+
+    if not args.no_oja:
+        out["oja_update"] = time_oja(lrkv, dev, world)
 
     if not args.no_dense:
         dc = lrkv.DenseCache(wl.B, wl.H_kv, cap, dtype=Kd.dtype, device=dev)
