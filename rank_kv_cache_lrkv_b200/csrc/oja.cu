@@ -2,7 +2,8 @@
 // (OjaKV article: Oja's algorithm for online PCA adapts the projection basis
 // during prompt prefill and periodically during decode).
 //
-// One CTA of 128 threads per stream keeps its basis P [128][r] in shared
+// For r <= 64 the basis lives in registers (oja2_kernel below).  Otherwise
+// one CTA of 128 threads per stream keeps its basis P [128][r] in shared
 // memory (row stride r + 1, so row-wise and column-wise walks are both free
 // of bank conflicts).  For each token, in order:
 //   y_j = sum_i P[i][j] x_i          (thread j)
@@ -10,6 +11,8 @@
 //   P[i][j] += eta z_i y_j           (thread i updates its own row)
 // and after every qr_every-th token P <- Q of QR(P) with diag(R) > 0, by
 // Gram-Schmidt with a second orthogonalisation pass per column.
+#include <cstdint>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -106,11 +109,252 @@ __global__ void __launch_bounds__(kOjaThreads) qr_kernel(float* P, int r, long l
   for (int e = threadIdx.x; e < kHeadDim * r; e += blockDim.x) Pg[e] = Ps[(e / r) * ld + e % r];
 }
 
+// ---- register-resident Oja update for r <= 64
+// 64 threads per stream; thread t holds rows t and t + 64 of P as float
+// pairs (RM >= r columns, the padding columns are zero and stay zero).  Per
+// token:
+//   y = P^T x : per-thread products of its two rows, reduce-scattered across
+//               each warp in blocks of 16 columns (16 shuffles per block), the
+//               two warps combined through shared memory;
+//   z_i = x_i - P_i . y,  P_i += eta z_i y   (registers; y read back as
+//               broadcast 16-byte loads).
+// Token rows arrive by cp.async in chunks of kOjaChunk tokens, double
+// buffered.  The QR every qr_every tokens writes P to a padded shared tile,
+// runs classical Gram-Schmidt with a second pass per column, and reads it back.
+constexpr int kOja2Threads = 64;
+constexpr int kOjaChunk = 8;
+
+__device__ __forceinline__ void bar64() { named_bar(1, kOja2Threads); }
+
+// One reduce-scatter stage over lane bit O: the lanes with the bit set keep
+// the upper half of their N values, the others the lower half, each adding
+// the partner's copy of the half it keeps.
+template <int N, int O>
+__device__ __forceinline__ void rs_stage(float (&w)[16], int lane) {
+  const bool up = (lane & O) != 0;
+#pragma unroll
+  for (int k = 0; k < N / 2; ++k) {
+    const float send = up ? w[k] : w[k + N / 2];
+    const float keep = up ? w[k + N / 2] : w[k];
+    w[k] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+  }
+}
+
+// Sum of w[0..15] over the 32 lanes, scattered: the lane ends with the sum of
+// column (lane & 15) (lanes l and l ^ 16 hold the same column).
+__device__ __forceinline__ float reduce16(float (&w)[16], int lane) {
+  rs_stage<16, 8>(w, lane);
+  rs_stage<8, 4>(w, lane);
+  rs_stage<4, 2>(w, lane);
+  rs_stage<2, 1>(w, lane);
+  return w[0] + __shfl_xor_sync(0xffffffffu, w[0], 16);
+}
+
+// Q of QR(P), diag(R) > 0, on the padded shared tile [128][ld], 64 threads
+// (rows t and t + 64 each).
+__device__ void qr_shared64(float* PQ, int r, int ld, float* col, float* h, float* red) {
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  for (int j = 0; j < r; ++j) {
+    col[t] = PQ[t * ld + j];
+    col[t + 64] = PQ[(t + 64) * ld + j];
+    bar64();
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int k = t; k < j; k += kOja2Threads) {
+        float s0 = 0.f, s1 = 0.f;
+        for (int i = 0; i < kHeadDim; i += 2) {
+          s0 = fmaf(PQ[i * ld + k], col[i], s0);
+          s1 = fmaf(PQ[(i + 1) * ld + k], col[i + 1], s1);
+        }
+        h[k] = s0 + s1;
+      }
+      bar64();
+      float c0 = col[t], c1 = col[t + 64];
+      for (int k = 0; k < j; ++k) {
+        c0 = fmaf(-h[k], PQ[t * ld + k], c0);
+        c1 = fmaf(-h[k], PQ[(t + 64) * ld + k], c1);
+      }
+      bar64();
+      col[t] = c0;
+      col[t + 64] = c1;
+      bar64();
+    }
+    const float c0 = col[t], c1 = col[t + 64];
+    const float ss = warp_sum(c0 * c0 + c1 * c1);
+    if (lane == 0) red[w] = ss;
+    bar64();
+    const float nrm = sqrtf(red[0] + red[1]);
+    PQ[t * ld + j] = c0 / nrm;
+    PQ[(t + 64) * ld + j] = c1 / nrm;
+    bar64();
+  }
+}
+
+inline size_t oja2_smem_bytes(int r, int esize) {
+  const int RM = (r + 15) / 16 * 16;
+  return (size_t)kHeadDim * (r + 1) * 4            // PQ
+         + (size_t)2 * kOjaChunk * kHeadDim * esize  // x ring
+         + (size_t)2 * 2 * RM * 4                    // red [parity][warp][RM]
+         + (size_t)2 * RM * 4                        // ys [parity][RM]
+         + (size_t)kHeadDim * 4 + (size_t)RM * 4 + 16;  // col, h, norm
+}
+
+template <typename T, int RM>
+__global__ void __launch_bounds__(kOja2Threads, 6) oja2_kernel(float* P, int r, long long bstride,
+                                                            const T* __restrict__ x,
+                                                            long long xstride, int n, float eta,
+                                                            int qr_every, long long seen) {
+  constexpr int NB = RM / 16;                // column blocks
+  constexpr int NP = RM / 2;                 // float pairs per row
+  constexpr int CE = 16 / sizeof(T);         // elements per 16-byte copy
+  extern __shared__ __align__(16) float sm[];
+  const int ld = r + 1;
+  float* PQ = sm;                                                       // [128][ld]
+  T* xr = reinterpret_cast<T*>(PQ + ((kHeadDim * ld + 3) & ~3));         // [2][chunk][128]
+  float* red = reinterpret_cast<float*>(xr + 2 * kOjaChunk * kHeadDim);  // [2][2][RM]
+  float* ys = red + 2 * 2 * RM;                                         // [2][RM]
+  float* col = ys + 2 * RM;                                             // [128]
+  float* h = col + kHeadDim;                                            // [RM]
+  float* nred = h + RM;                                                 // [2]
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  float* Pg = P + (size_t)blockIdx.x * bstride;
+  const T* xg = x + (size_t)blockIdx.x * xstride;
+
+  auto stage = [&](int c, int buf) {  // chunk c of token rows into ring buffer buf
+    const int t0 = c * kOjaChunk;
+    for (int q = t; q < kOjaChunk * kHeadDim / CE; q += kOja2Threads) {
+      const int row = q / (kHeadDim / CE), e = (q - row * (kHeadDim / CE)) * CE;
+      const bool ok = t0 + row < n;
+      cp_async16(xr + (buf * kOjaChunk + row) * kHeadDim + e,
+                 xg + (size_t)(ok ? t0 + row : 0) * kHeadDim + e, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  if (n > 0) stage(0, 0);
+
+  float2 P0[NP], P1[NP];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int j = 2 * p;
+    P0[p] = make_float2(j < r ? Pg[t * r + j] : 0.f, j + 1 < r ? Pg[t * r + j + 1] : 0.f);
+    P1[p] = make_float2(j < r ? Pg[(t + 64) * r + j] : 0.f,
+                        j + 1 < r ? Pg[(t + 64) * r + j + 1] : 0.f);
+  }
+  for (int q = t; q < 2 * RM; q += kOja2Threads) ys[q] = 0.f;  // padding columns stay 0
+
+  for (int tok = 0; tok < n; ++tok) {
+    const int c = tok / kOjaChunk, slot = tok - c * kOjaChunk, buf = c & 1, par = tok & 1;
+    if (slot == 0) {
+      if ((c + 1) * kOjaChunk < n) {
+        stage(c + 1, buf ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      bar64();  // chunk c is in place for every thread
+    }
+    const T* xrow = xr + (buf * kOjaChunk + slot) * kHeadDim;
+    const float x0 = to_f<T>(xrow[t]), x1 = to_f<T>(xrow[t + 64]);
+    const float2 x02 = make_float2(x0, x0), x12 = make_float2(x1, x1);
+    // y = P^T x: this thread's two rows, then across the warp and the two warps
+#pragma unroll
+    for (int bk = 0; bk < NB; ++bk) {
+      float wv[16];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float2 v = mul2(P1[bk * 8 + u], x12);
+        fma2(v, P0[bk * 8 + u], x02);
+        wv[2 * u] = v.x;
+        wv[2 * u + 1] = v.y;
+      }
+      const float s = reduce16(wv, lane);
+      if (lane < 16) red[(par * 2 + w) * RM + bk * 16 + lane] = s;
+    }
+    bar64();
+    if (t < r) ys[par * RM + t] = red[(par * 2) * RM + t] + red[(par * 2 + 1) * RM + t];
+    bar64();
+    // z = x - P y, then P += eta z y^T
+    const float4* y4 = reinterpret_cast<const float4*>(ys + par * RM);
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < RM / 4; ++q) {
+      const float4 yv = y4[q];
+      const float2 ylo = make_float2(yv.x, yv.y), yhi = make_float2(yv.z, yv.w);
+      fma2(a0, P0[2 * q], ylo);
+      fma2(a0, P0[2 * q + 1], yhi);
+      fma2(a1, P1[2 * q], ylo);
+      fma2(a1, P1[2 * q + 1], yhi);
+    }
+    const float ez0 = eta * (x0 - (a0.x + a0.y)), ez1 = eta * (x1 - (a1.x + a1.y));
+    const float2 e02 = make_float2(ez0, ez0), e12 = make_float2(ez1, ez1);
+#pragma unroll
+    for (int q = 0; q < RM / 4; ++q) {
+      const float4 yv = y4[q];
+      const float2 ylo = make_float2(yv.x, yv.y), yhi = make_float2(yv.z, yv.w);
+      fma2(P0[2 * q], e02, ylo);
+      fma2(P0[2 * q + 1], e02, yhi);
+      fma2(P1[2 * q], e12, ylo);
+      fma2(P1[2 * q + 1], e12, yhi);
+    }
+    if (qr_every > 0 && (seen + tok + 1) % qr_every == 0) {
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const int j = 2 * p;
+        if (j < r) { PQ[t * ld + j] = P0[p].x; PQ[(t + 64) * ld + j] = P1[p].x; }
+        if (j + 1 < r) { PQ[t * ld + j + 1] = P0[p].y; PQ[(t + 64) * ld + j + 1] = P1[p].y; }
+      }
+      bar64();
+      qr_shared64(PQ, r, ld, col, h, nred);
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const int j = 2 * p;
+        P0[p] = make_float2(j < r ? PQ[t * ld + j] : 0.f, j + 1 < r ? PQ[t * ld + j + 1] : 0.f);
+        P1[p] = make_float2(j < r ? PQ[(t + 64) * ld + j] : 0.f,
+                            j + 1 < r ? PQ[(t + 64) * ld + j + 1] : 0.f);
+      }
+      bar64();
+    }
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int j = 2 * p;
+    if (j < r) { Pg[t * r + j] = P0[p].x; Pg[(t + 64) * r + j] = P1[p].x; }
+    if (j + 1 < r) { Pg[t * r + j + 1] = P0[p].y; Pg[(t + 64) * r + j + 1] = P1[p].y; }
+  }
+}
+
+template <typename T>
+static int oja2_launch_t(float* P, int S, int r, long long bs, const T* x, long long xs, int n,
+                         float eta, int qr_every, long long seen, cudaStream_t st) {
+  const size_t sm = oja2_smem_bytes(r, (int)sizeof(T));
+  auto go = [&](auto kern) -> int {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+        cudaSuccess)
+      return LRKV_ERR_CUDA;
+    kern<<<S, kOja2Threads, sm, st>>>(P, r, bs, x, xs, n, eta, qr_every, seen);
+    return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+  };
+  if (r <= 16) return go(oja2_kernel<T, 16>);
+  if (r <= 32) return go(oja2_kernel<T, 32>);
+  if (r <= 48) return go(oja2_kernel<T, 48>);
+  return go(oja2_kernel<T, 64>);
+}
+
 static size_t oja_smem(int r) { return (size_t)(kHeadDim * (r + 1) + 5 * kHeadDim) * 4; }
 
 int oja_launch(float* P, int S, int r, long long basis_stride, const void* x, int x_dtype,
                long long x_stride, int n, float eta, int qr_every, long long tokens_seen,
                cudaStream_t st) {
+  // register-resident kernel for r <= 64 when rows can be copied in 16-byte pieces
+  const int es = x_dtype == LRKV_BF16 ? 2 : 4;
+  const bool aligned = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (x_stride * es) % 16 == 0;
+  if (r <= 64 && aligned && n > 0) {
+    if (x_dtype == LRKV_BF16)
+      return oja2_launch_t(P, S, r, basis_stride, static_cast<const __nv_bfloat16*>(x), x_stride,
+                           n, eta, qr_every, tokens_seen, st);
+    return oja2_launch_t(P, S, r, basis_stride, static_cast<const float*>(x), x_stride, n, eta,
+                         qr_every, tokens_seen, st);
+  }
   const size_t sm = oja_smem(r);
   if (x_dtype == LRKV_BF16) {
     auto k = oja_kernel<__nv_bfloat16>;
