@@ -34,7 +34,6 @@ __device__ inline int appended(const int* n_new, int n, int b) {
 
 struct AppendArgs {
   int B, H_kv, rk, rv, n_sink, W, maxp, num_pages, n, anchor_tiles;
-  int bulk_tpc;  // bulk_compress_mma: 64-token tiles per CTA
   void *codes, *anchors;
   const int* bt;
   int* seq_len;
@@ -266,61 +265,126 @@ __global__ void __launch_bounds__(256) bulk_compress_kernel(AppendArgs a) {
 }
 
 // ---- bf16 prefill compress on the tensor cores
-// c = x P for 64-token tiles of one (sequence, KV head): per warp 16 tokens
-// (m16) x the code columns (n8 blocks) x 128 dims (eight k16 steps), with P
-// split as hi + lo bf16 so the products keep about 16 mantissa bits and
-// accumulate in fp32.  Token rows are staged by cp.async into padded
-// shared-memory rows (two stages), P^T sits in padded rows too, so ldmatrix
-// reads both operands without bank conflicts.
-constexpr int kBulkTile = 64;          // tokens per tile (a warp takes 16)
+// c = x P for the tokens that go straight to latent pages.  Persistent: one
+// CTA per SM; the tiles of TT tokens of every (sequence, KV head) unit are
+// laid end to end and each CTA takes an equal contiguous range, so ragged
+// prompts balance.  Per tile each warp projects 16 tokens (m16) x the code
+// columns (n8 blocks) x 128 dims (eight k16 steps), with P split as hi + lo
+// bf16 so the products keep about 16 mantissa bits and accumulate in fp32.
+// Token rows are staged by cp.async into padded shared-memory rows (two
+// stages); P^T hi/lo sits in padded rows too, rebuilt when the range enters
+// a new unit, so ldmatrix reads both operands without bank conflicts.
 constexpr int kPadRow = kHeadDim + 8;  // bf16 elements per staged row
 
 __host__ __device__ inline int round16(int x) { return (x + 15) / 16 * 16; }
-inline size_t bulk_mma_smem_bytes(int rk, int rv) {
-  return ((size_t)2 * (round16(rk) + round16(rv)) + (size_t)2 * 2 * kBulkTile) * kPadRow * 2;
+// Shared memory of bulk_compress_mma for tiles of TT tokens and B sequences.
+inline size_t bulk_mma_smem_bytes(int rk, int rv, int TT, int B) {
+  return ((size_t)2 * (round16(rk) + round16(rv)) + (size_t)2 * 2 * TT) * kPadRow * 2 +
+         (size_t)4 * (B + 1) * 4;
 }
 
-__global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
+// First tile of CTA c when `total` tiles are split evenly over C CTAs.
+__device__ inline int bulk_range_lo(int c, int total, int C) {
+  const int q = total / C, r = total - q * C;
+  return c * q + (c * r) / C;
+}
+
+// Input rows of sequence b that go straight to latent: [in_lo, in_hi), relative to L0.
+__device__ inline void bulk_rows(const AppendArgs& a, int b, int& L0, int& in_lo, int& in_hi) {
+  L0 = __ldcg(a.seq_len + b);
+  const int L1 = L0 + appended(a.n_new, a.n, b);
+  const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
+  in_lo = max(L0, a.n_sink + s0.lat) - L0;
+  in_hi = max(in_lo, a.n_sink + s1.lat - L0);
+}
+
+template <int TT>
+__global__ void __launch_bounds__(TT * 2) bulk_compress_mma(AppendArgs a) {
   using bf16 = __nv_bfloat16;
+  constexpr int kThreadsB = TT * 2;  // TT / 16 warps
   extern __shared__ __align__(16) bf16 smb[];
   const int RK = round16(a.rk), RV = round16(a.rv), NR = RK + RV;
   bf16* PT = smb;                        // [hi, lo][NR][kPadRow]: rows K codes then V codes
-  bf16* X = smb + 2 * NR * kPadRow;      // [stage][k, v][64][kPadRow]
-  const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  bf16* X = smb + 2 * NR * kPadRow;      // [stage][k, v][TT][kPadRow]
+  int* start = reinterpret_cast<int*>(X + 2 * 2 * TT * kPadRow);  // [B + 1] tile prefix
+  int* sL0 = start + (a.B + 1);                                    // [B] seq_len before
+  int* srlo = sL0 + (a.B + 1);                                     // [B] row range
+  int* srhi = srlo + (a.B + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int L0 = __ldcg(a.seq_len + b), L1 = L0 + appended(a.n_new, a.n, b);
-  const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
-  // input rows that go straight to latent, relative to L0
-  const int in_lo = max(L0, a.n_sink + s0.lat) - L0, in_hi = a.n_sink + s1.lat - L0;
-  const int rbeg = in_lo + blockIdx.x * kBulkTile * a.bulk_tpc;
-  const int rend = min(in_hi, rbeg + kBulkTile * a.bulk_tpc);
-  if (rbeg >= rend) return;
-  const int ntiles = (rend - rbeg + kBulkTile - 1) / kBulkTile;
-  const bf16* kin = static_cast<const bf16*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
-  const bf16* vin = static_cast<const bf16*>(a.v) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
 
-  auto stage = [&](int i, int st) {
-    const int t0 = rbeg + i * kBulkTile;
-    for (int x = tid; x < 2 * kBulkTile * 16; x += blockDim.x) {
-      const int isv = x / (kBulkTile * 16), rem = x - isv * kBulkTile * 16;
+  // tile prefix over sequences (tiles per unit = ceil(rows / TT)), one warp
+  if (warp == 0) {
+    const int per = (a.B + 31) / 32;
+    const int b0 = min(a.B, lane * per), b1 = min(a.B, b0 + per);
+    int own = 0;
+    for (int b = b0; b < b1; ++b) {
+      int L0, rl, rh;
+      bulk_rows(a, b, L0, rl, rh);
+      sL0[b] = L0;
+      srlo[b] = rl;
+      srhi[b] = rh;
+      own += (rh - rl + TT - 1) / TT * a.H_kv;
+    }
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int e = incl - own;
+    for (int b = b0; b < b1; ++b) {
+      start[b] = e;
+      e += (srhi[b] - srlo[b] + TT - 1) / TT * a.H_kv;
+    }
+    if (lane == 31) start[a.B] = incl;
+  }
+  __syncthreads();
+  const int total = start[a.B];
+  const int lo = bulk_range_lo(blockIdx.x, total, gridDim.x);
+  const int hi = bulk_range_lo(blockIdx.x + 1, total, gridDim.x);
+  if (lo >= hi) return;
+
+  // tile index -> (sequence, KV head, tile within the unit)
+  auto locate = [&](int k, int& b, int& kvh, int& i, int& tiles) {
+    int l = 0, h = a.B;
+    while (h - l > 1) {
+      const int mid = (l + h) >> 1;
+      if (start[mid] <= k) l = mid; else h = mid;
+    }
+    b = l;
+    tiles = (start[b + 1] - start[b]) / a.H_kv;
+    const int r = k - start[b];
+    kvh = r / tiles;
+    i = r - kvh * tiles;
+  };
+  auto stage = [&](int k, int st) {
+    int b, kvh, i, tiles;
+    locate(k, b, kvh, i, tiles);
+    const int rlo = srlo[b], rhi = srhi[b];
+    const bf16* kin = static_cast<const bf16*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
+    const bf16* vin = static_cast<const bf16*>(a.v) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
+    const int t0 = rlo + i * TT;
+    for (int x = tid; x < 2 * TT * 16; x += kThreadsB) {
+      const int isv = x / (TT * 16), rem = x - isv * TT * 16;
       const int row = rem >> 4, ch = rem & 15;
       const int r = t0 + row;
-      const bool ok = r < rend;  // rows past the range are zero-filled
-      const bf16* src = (isv ? vin : kin) + (size_t)(ok ? r : rbeg) * kHeadDim + ch * 8;
-      cp_async16(X + ((st * 2 + isv) * kBulkTile + row) * kPadRow + ch * 8, src, ok ? 16u : 0u);
+      const bool ok = r < rhi;  // rows past the range are zero-filled
+      const bf16* src = (isv ? vin : kin) + (size_t)(ok ? r : rlo) * kHeadDim + ch * 8;
+      cp_async16(X + ((st * 2 + isv) * TT + row) * kPadRow + ch * 8, src, ok ? 16u : 0u);
     }
     cp_async_commit();
   };
-  stage(0, 0);
-  // P^T as hi + lo bf16 (rows past r_k / r_v are zero); four columns per
-  // load, eight loads in flight per thread
-  {
+  // P^T as hi + lo bf16 for unit (b, kvh); rows past r_k / r_v are zero.
+  // Consecutive threads take consecutive dims i, so the transposed stores hit
+  // consecutive addresses (no bank conflicts).
+  auto load_basis = [&](int b, int kvh) {
     const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
     const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
     const int n4 = NR / 4;
 #pragma unroll 8
-    for (int x = tid; x < kHeadDim * n4; x += blockDim.x) {
-      const int i = x / n4, o = 4 * (x - i * n4);
+    for (int x = tid; x < kHeadDim * n4; x += kThreadsB) {
+      const int i = x & (kHeadDim - 1), o = 4 * (x / kHeadDim);
       float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
       if (o < RK) {
         if (o < a.rk) p = __ldg(reinterpret_cast<const float4*>(Pk + (size_t)i * a.rk + o));
@@ -335,21 +399,32 @@ __global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
         PT[(NR + o + u) * kPadRow + i] = __float2bfloat16_rn(pv[u] - __bfloat162float(h));
       }
     }
-  }
+  };
+
   bf16* codes = static_cast<bf16*>(a.codes);
-  for (int i = 0; i < ntiles; ++i) {
-    const int st = i & 1;
-    if (i + 1 < ntiles) {
-      stage(i + 1, st ^ 1);
+  int cur_unit = -1;
+  stage(lo, 0);
+  for (int k = lo; k < hi; ++k) {
+    const int st = (k - lo) & 1;
+    int b, kvh, i, tiles;
+    locate(k, b, kvh, i, tiles);
+    const int L0 = sL0[b], rlo = srlo[b], rhi = srhi[b];
+    const int unit = b * a.H_kv + kvh;
+    if (unit != cur_unit) {  // every warp is past the previous tile (barrier at its end)
+      load_basis(b, kvh);
+      cur_unit = unit;
+    }
+    if (k + 1 < hi) {
+      stage(k + 1, st ^ 1);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
-    __syncthreads();
-    const int tok0 = rbeg + i * kBulkTile + 16 * warp;  // first input row of this warp
+    __syncthreads();  // tile k and the basis are in place
+    const int tok0 = rlo + i * TT + 16 * warp;  // first input row of this warp
     for (int isv = 0; isv < 2; ++isv) {
       const int r = isv ? a.rv : a.rk, nb = r / 8, RB = isv ? RK : 0;
-      const bf16* xt = X + ((st * 2 + isv) * kBulkTile + 16 * warp) * kPadRow;
+      const bf16* xt = X + ((st * 2 + isv) * TT + 16 * warp) * kPadRow;
       uint32_t af[8][4];
 #pragma unroll
       for (int s = 0; s < 8; ++s)
@@ -360,7 +435,7 @@ __global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
       for (int h2 = 0; h2 < 2; ++h2) {
         const int rin = tok0 + g + 8 * h2;
         jrow[h2] = L0 + rin - a.n_sink;
-        prow[h2] = rin < rend ? latent_page(a, b, jrow[h2]) : -1;
+        prow[h2] = rin < rhi ? latent_page(a, b, jrow[h2]) : -1;
       }
       for (int ng = 0; ng < nb; ng += 8) {
         float acc[8][4];
@@ -391,7 +466,8 @@ __global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             if (ng + q < nb) {
-              const long long off = code_off_in<bf16>(a, prow[h2], kvh, jrow[h2], 8 * (ng + q) + 2 * t, isv);
+              const long long off =
+                  code_off_in<bf16>(a, prow[h2], kvh, jrow[h2], 8 * (ng + q) + 2 * t, isv);
               *reinterpret_cast<uint32_t*>(codes + off) =
                   pack_bf16x2(acc[q][2 * h2], acc[q][2 * h2 + 1]);
             }
@@ -399,7 +475,7 @@ __global__ void __launch_bounds__(128) bulk_compress_mma(AppendArgs a) {
         }
       }
     }
-    __syncthreads();  // stage st is refilled by the next iteration's prefetch
+    __syncthreads();  // stage st is refilled, and the basis may be rebuilt, next iteration
   }
 }
 
@@ -408,16 +484,24 @@ static int compress_t(const AppendArgs& a, cudaStream_t st) {
   const bool small = a.n <= kSmallN;
   if (!small) {
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-      const size_t smem = bulk_mma_smem_bytes(a.rk, a.rv);
-      if (cudaFuncSetAttribute(bulk_compress_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem) != cudaSuccess)
+      // persistent: one CTA per SM; 128-token tiles (8 warps) when they fit
+      int dev = 0, sms = 0, optin = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+              cudaSuccess)
         return LRKV_ERR_CUDA;
-      // about two CTAs per SM over the whole call; each converts its basis once
-      AppendArgs b2 = a;
-      const long long tiles = (long long)((a.n + kBulkTile - 1) / kBulkTile) * a.H_kv * a.B;
-      b2.bulk_tpc = (int)std::min<long long>(64, std::max<long long>(1, (tiles + 295) / 296));
-      const int per = kBulkTile * b2.bulk_tpc;
-      bulk_compress_mma<<<dim3((a.n + per - 1) / per, a.H_kv, a.B), 128, smem, st>>>(b2);
+      const bool big = bulk_mma_smem_bytes(a.rk, a.rv, 128, a.B) <= (size_t)optin;
+      const size_t smem = bulk_mma_smem_bytes(a.rk, a.rv, big ? 128 : 64, a.B);
+      if (smem > (size_t)optin) return LRKV_ERR_UNSUPPORTED;
+      const void* fn = big ? (const void*)bulk_compress_mma<128> : (const void*)bulk_compress_mma<64>;
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+        return LRKV_ERR_CUDA;
+      if (big)
+        bulk_compress_mma<128><<<sms, 256, smem, st>>>(a);
+      else
+        bulk_compress_mma<64><<<sms, 128, smem, st>>>(a);
     } else {
       dim3 g((a.n + kBulkRows - 1) / kBulkRows, a.H_kv, a.B);
       bulk_compress_kernel<T><<<g, 256, 0, st>>>(a);
