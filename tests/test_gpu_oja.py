@@ -37,7 +37,8 @@ def _setup(S, r, n, dtype, seed=0):
 
 
 @pytest.mark.parametrize("r,dtype,qr_every,seen", [(48, "bf16", 256, 100), (32, "f32", 64, 0),
-                                                   (8, "bf16", 0, 0), (128, "f32", 100, 7)])
+                                                   (8, "bf16", 0, 0), (128, "f32", 100, 7),
+                                                   (64, "bf16", 128, 0), (56, "f32", 200, 3)])
 def test_oja_matches_oracle(lrkv, r, dtype, qr_every, seen):
     S, n, eta = 5, 700, 1e-3
     P0, X = _setup(S, r, n, dtype)
