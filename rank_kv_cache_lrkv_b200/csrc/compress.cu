@@ -114,19 +114,35 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
   int* pg = reinterpret_cast<int*>(red + 256);                         // [row]
   const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
 
-  // 1. seq_len, and the basis into shared memory ([i][o]: P_k columns then P_v)
+  // Launched with programmatic dependent launch: wait for the previous grid
+  // before reading anything (only the launch latency is hidden).
+  pdl_wait();
+  // 1. seq_len, and the basis into shared memory ([i][o]: P_k columns then P_v),
+  // eight 16-byte loads in flight per thread
   const int L0 = __ldcg(a.seq_len + b);
   if constexpr (kCluster) cluster_arrive();
   {
     const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
     const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
-    const int n4 = NJ / 4;
-#pragma unroll 4
-    for (int x = tid; x < kHeadDim * n4; x += blockDim.x) {
-      const int i = x / n4, o = 4 * (x - i * n4);
-      const float4 v = o < a.rk ? __ldg(reinterpret_cast<const float4*>(Pk + i * a.rk + o))
-                                : __ldg(reinterpret_cast<const float4*>(Pv + i * a.rv + o - a.rk));
-      reinterpret_cast<float4*>(Ps)[x] = v;
+    const int n4 = NJ / 4, total4 = kHeadDim * n4;
+    constexpr int kB = 8;
+    for (int x0 = tid; x0 < total4; x0 += kB * (int)blockDim.x) {
+      float4 v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int x = x0 + u * (int)blockDim.x;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (x < total4) {
+          const int i = x / n4, o = 4 * (x - i * n4);
+          v[u] = o < a.rk ? __ldg(reinterpret_cast<const float4*>(Pk + i * a.rk + o))
+                          : __ldg(reinterpret_cast<const float4*>(Pv + i * a.rv + o - a.rk));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int x = x0 + u * (int)blockDim.x;
+        if (x < total4) reinterpret_cast<float4*>(Ps)[x] = v[u];
+      }
     }
   }
   const int L1 = L0 + appended(a.n_new, a.n, b);
@@ -519,13 +535,15 @@ static int compress_t(const AppendArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = a.H_kv;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = a.H_kv;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = cluster ? 1 : 0;
+  cfg.numAttrs = cluster ? 2 : 1;
   int small_in = small ? 1 : 0;
   void* args[] = {(void*)&a, (void*)&small_in};
   if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return LRKV_ERR_CUDA;

@@ -291,6 +291,8 @@ struct QFrag {
   uint32_t hi[KS][2], lo[KS][2];  // B operands (k = dim, n = head)
 };
 
+// q~ rows of the unit's G heads (qv: row of head 0, rows qdim apart, in the
+// workspace) -> B fragments.
 template <int G, int KS>
 __device__ inline void load_qfrag(const float* qv, int qdim, int lane, QFrag<KS>& f) {
   const int g = lane >> 2, t = lane & 3;
@@ -301,8 +303,9 @@ __device__ inline void load_qfrag(const float* qv, int qdim, int lane, QFrag<KS>
       const int d = 16 * s + 8 * r + 2 * t;
       float x0 = 0.f, x1 = 0.f;
       if (g < G && d < qdim) {
-        x0 = qv[g * qdim + d];
-        x1 = qv[g * qdim + d + 1];
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(qv + g * qdim + d));
+        x0 = x.x;
+        x1 = x.y;
       }
       const uint32_t h = pack_bf16x2(x0, x1);
       f.hi[s][r] = h;
@@ -536,7 +539,10 @@ __host__ __device__ inline bool anchor_mode(const void* fr, const int* bt_fr) {
 struct SmemPlan {
   int ring, full, empty, tag, start_lat, start_fr, pbuf, qown, flags, total;
 };
-__host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, int G) {
+// tc: the consumers run on the tensor cores and keep their query fragments in
+// registers, so only the anchor warp needs probability and query slices.
+__host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, int G, bool tc) {
+  const int slots = tc ? 1 : kConsumers + 1;
   SmemPlan p;
   int off = 0;
   auto take = [&](int bytes, int align) {
@@ -553,8 +559,8 @@ __host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, in
   p.start_fr = take((B + 1) * 4, 4);
   // per consumer warp and the anchor warp: probabilities [G][64] as pairs and
   // the unit's folded queries [G][128]
-  p.pbuf = take((kConsumers + 1) * kLatPage * G * 8, 16);
-  p.qown = take((kConsumers + 1) * G * kHeadDim * 4, 16);
+  p.pbuf = take(slots * kLatPage * G * 8, 16);
+  p.qown = take(slots * G * kHeadDim * 4, 16);
   p.flags = take(16, 16);
   p.total = off;
   return p;
@@ -699,7 +705,8 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
   constexpr int CE = Elem<T>::CE;
   constexpr int NP = CE / 2;
   extern __shared__ __align__(1024) uint8_t smem[];
-  const SmemPlan sp_ = smem_plan(a.NS, a.stage_bytes, a.B, G);
+  constexpr bool kTC = std::is_same<T, __nv_bfloat16>::value;
+  const SmemPlan sp_ = smem_plan(a.NS, a.stage_bytes, a.B, G, kTC);
   uint8_t* ring = smem + sp_.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp_.full);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + sp_.empty);
@@ -805,10 +812,9 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
   }
 
   pdl_wait();  // the q-fold results are visible from here on
-  float2* pbuf = reinterpret_cast<float2*>(smem + sp_.pbuf) +
-                 (warp == kAnchorWarp ? kConsumers : warp - kFirstConsumer) * kLatPage * G;
-  float* qv = reinterpret_cast<float*>(smem + sp_.qown) +
-              (warp == kAnchorWarp ? kConsumers : warp - kFirstConsumer) * G * kHeadDim;
+  const int slot = kTC ? 0 : (warp == kAnchorWarp ? kConsumers : warp - kFirstConsumer);
+  float2* pbuf = reinterpret_cast<float2*>(smem + sp_.pbuf) + slot * kLatPage * G;
+  float* qv = reinterpret_cast<float*>(smem + sp_.qown) + slot * G * kHeadDim;
 
   if (warp == kAnchorWarp) {
     // ---------------- anchor warp: this CTA's share of the anchor tiles
@@ -866,7 +872,7 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
     locate(rstart, a.B, a.H_kv, t, b, kvh, i0, tiles);
     const int unit = b * a.H_kv + kvh, ustart = t - i0, ce = min(hi, ustart + tiles);
     const int ntok = space_tokens(a, rsp, b);
-    fetch_queries_warp<G>(a, rsp, b, kvh, qv, lane);
+    if constexpr (!kTC) fetch_queries_warp<G>(a, rsp, b, kvh, qv, lane);
     const int k0 = t - lo;
     const int first = t + ((w - k0 % kConsumers) + kConsumers) % kConsumers;
     // Wait (bounded) for tile tt of the ring; nullptr on timeout.
@@ -886,7 +892,8 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
     if constexpr (kTensorTiles) {
       constexpr int TT = kDense ? kFrTile : kLatPage;
       QFrag<KS> qf;
-      load_qfrag<G, KS>(qv, qdim, lane, qf);
+      load_qfrag<G, KS>((rsp == 0 ? a.qlat : a.qfr) + ((size_t)b * a.H_q + (size_t)kvh * G) * qdim,
+                        qdim, lane, qf);
       float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, acc[2][VB][4];
 #pragma unroll
       for (int hl = 0; hl < 2; ++hl)
@@ -995,6 +1002,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
   int* start_lat = reinterpret_cast<int*>(smem + mp.starts);
   int* start_fr = start_lat + (a.B + 1);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + mp.bars);
+  pdl_trigger();  // whatever follows may be scheduled now; it waits for this grid itself
 
   const int unit = blockIdx.x, b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -1193,10 +1201,11 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   p.stage_bytes = has_lat ? kLatPage * (rk + rv) * esize : 2 * kFrTile * kHeadDim * esize;
   // Leave room for a q-fold CTA beside each split CTA.
   const int budget = optin - 8 * 1024;
-  const int fixed = smem_plan(0, p.stage_bytes, B, G).total + 1024;
+  const bool tc = esize == 2;  // bf16: tensor-core consumers
+  const int fixed = smem_plan(0, p.stage_bytes, B, G, tc).total + 1024;
   p.NS = std::min(kMaxStages, (budget - fixed) / p.stage_bytes);
   if (p.NS < 2) return LRKV_ERR_UNSUPPORTED;
-  p.smem = smem_plan(p.NS, p.stage_bytes, B, G).total;
+  p.smem = smem_plan(p.NS, p.stage_bytes, B, G, tc).total;
   p.C = sms;
   p.merge_smem = merge_plan(rv, has_lat, G, B).total;
   const int U = B * H_kv;
