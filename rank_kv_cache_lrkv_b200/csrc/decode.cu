@@ -35,7 +35,7 @@
 
 namespace lrkv {
 
-constexpr int kConsumers = 6;                  // consumer warps per CTA
+constexpr int kConsumers = 8;                  // consumer warps per CTA
 constexpr int kProducerWarp = 0;
 constexpr int kAnchorWarp = 1;
 constexpr int kFirstConsumer = 2;
@@ -43,6 +43,7 @@ constexpr int kThreads = 32 * (kFirstConsumer + kConsumers);
 constexpr int kMaxStages = 24;
 constexpr int kIssue = 4;                      // producer lanes issuing at once
 constexpr int kMergeThreads = 256;
+constexpr int kMergeWarps = kMergeThreads / 32;
 constexpr int kMergeBuf = 64 * 1024;           // merge: bytes of records per chunk
 constexpr int kMergeMaxRec = 256;              // merge: records per chunk at most
 
@@ -698,10 +699,11 @@ __device__ void anchor_tile(const uint4* kch, int n_valid, const float* qv, floa
 // ------------------------------------------------------------ split kernel
 // kDense: the ring carries full-rank pages (dense baseline) instead of latent
 // pages; KS / VB: rank class of the tensor-core tiles (bf16 only).
-// 200 registers: two warps per SM sub-partition, with room left for a q-fold
-// CTA beside the split CTA.
+// 168 registers: ten warps, three on two of the SM's four sub-partitions
+// (16K registers each).  More consumer warps hide more of each warp's
+// dependent latency; fewer registers spill in the wider rank classes.
 template <typename T, int G, bool kDense, int KS, int VB>
-__global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
+__global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   constexpr int CE = Elem<T>::CE;
   constexpr int NP = CE / 2;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -744,21 +746,25 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
   if (warp == kProducerWarp) {
     // ---------------- producer: lane l holds the slab address of tile base + l;
     // the next batch's block-table reads are in flight while this batch is
-    // issued, kIssue lanes at a time.
+    // issued, kIssue lanes at a time (fetch issues the read, addr consumes it).
     const uint64_t pol = l2_evict_first_policy();
-    auto addr = [&](int kk, const void*& src, uint32_t& bytes, int& good) {
+    auto fetch = [&](int kk, int& kvh, int& page) {
+      kvh = 0; page = -1;
+      if (kk >= N) return;
+      int b, i, tiles;
+      locate(rstart, a.B, a.H_kv, lo + kk, b, kvh, i, tiles);
+      page = rsp == 0 ? __ldg(a.bt_lat + (size_t)b * a.maxp_lat + i)
+                      : __ldg(a.bt_fr + (size_t)b * a.maxp_fr + i);
+    };
+    auto addr = [&](int kk, int kvh, int page, const void*& src, uint32_t& bytes, int& good) {
       src = nullptr; bytes = 0; good = 0;
       if (kk >= N) return;
-      int b, kvh, i, tiles;
-      locate(rstart, a.B, a.H_kv, lo + kk, b, kvh, i, tiles);
       if (rsp == 0) {
-        const int page = a.bt_lat[(size_t)b * a.maxp_lat + i];
         good = page >= 0 && page < a.num_pages_lat;
         const size_t slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
         bytes = kLatPage * (a.rk + a.rv) * sizeof(T);
         src = static_cast<const T*>(a.codes) + slab * kLatPage * (a.rk + a.rv);
       } else {
-        const int page = a.bt_fr[(size_t)b * a.maxp_fr + i];
         good = page >= 0 && page < a.num_pages_fr;
         const size_t slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
         bytes = 2 * kFrTile * kHeadDim * sizeof(T);
@@ -768,11 +774,13 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
     const void *csrc, *nsrc;
     uint32_t cbytes, nbytes;
     int cgood, ngood;
-    addr(lane, csrc, cbytes, cgood);
+    int fk, fp;
+    fetch(lane, fk, fp);
+    addr(lane, fk, fp, csrc, cbytes, cgood);
     int issued = 0;
     bool ok = true;
     for (int base = 0; base < N && ok; base += 32) {
-      addr(base + 32 + lane, nsrc, nbytes, ngood);
+      fetch(base + 32 + lane, fk, fp);
       const int cnt = min(32, N - base);
       for (int j0 = 0; j0 < cnt; j0 += kIssue) {
         int f = 0;
@@ -800,6 +808,7 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
         }
         issued = base + min(j0 + kIssue, cnt);
       }
+      addr(base + 32 + lane, fk, fp, nsrc, nbytes, ngood);
       csrc = nsrc; cbytes = nbytes; cgood = ngood;
     }
     // Drain: wait (bounded) for every copy this CTA issued before exiting.
@@ -937,8 +946,9 @@ __global__ void __maxnreg__(200) split_kernel(DecodeArgs a) {
 // ------------------------------------------------------------ merge kernel
 // Shared-memory plan of the merge kernel (byte offsets from the base).
 struct MergePlan {
-  int pvt, recb, fin, mh, lh, ah, mm, ll, wts, starts, bars, total;
+  int pv, recb, wts, latf, frf, lf, starts, bars, total;
 };
+__host__ __device__ inline int pv_row(int rv) { return rv + 4; }  // padded row of P_v
 __host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B) {
   MergePlan p;
   int off = 0;
@@ -948,31 +958,37 @@ __host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B) 
     off += bytes;
     return at;
   };
-  p.pvt = take(lat ? rv * (kHeadDim + 1) * 4 : 0, 16);
+  p.pv = take(lat ? kHeadDim * pv_row(rv) * 4 : 0, 16);
   p.recb = take(kMergeBuf, 128);
-  p.fin = take(G * kHeadDim * 4, 16);
-  p.mh = take(32, 16);
-  p.lh = take(32, 16);
-  p.ah = take(32, 16);
-  p.mm = take(kMergeMaxRec * G * 4, 16);
-  p.ll = take(kMergeMaxRec * G * 4, 16);
-  p.wts = take(kMergeMaxRec * G * 4, 16);
+  p.wts = take(kMergeWarps * (kMergeMaxRec + 4) * 4, 16);
+  p.latf = take(G * (lat ? rv : 0) * 4, 16);
+  p.frf = take(G * kHeadDim * 4, 16);
+  p.lf = take(G * 4, 16);
   p.starts = take(2 * (B + 1) * 4, 8);
   p.bars = take(8, 8);
   p.total = off;
   return p;
 }
 
-// sum over x < n of w[x * G] * col[x * S], eight loads in flight
-template <int G>
-__device__ __forceinline__ float weighted_column(const float* col, int S, const float* w, int n) {
+// sum over x < n of w[x] * col[x * S] (w 16-byte aligned); a record of
+// weight 0 adds nothing even if its words are stale.  Sixteen loads in flight.
+__device__ __forceinline__ float weighted_sum(const float* col, int S, const float* w, int n) {
   float s[4] = {0.f, 0.f, 0.f, 0.f};
   int x = 0;
 #pragma unroll 2
-  for (; x + 4 <= n; x += 4)
+  for (; x + 4 <= n; x += 4) {
+    const float4 w4 = *reinterpret_cast<const float4*>(w + x);
+    const float ww[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) s[u] = fmaf(w[(x + u) * G], col[(x + u) * S], s[u]);
-  for (; x < n; ++x) s[0] = fmaf(w[x * G], col[x * S], s[0]);
+    for (int u = 0; u < 4; ++u) {
+      const float c = col[(x + u) * S];
+      s[u] = fmaf(ww[u], ww[u] > 0.f ? c : 0.f, s[u]);
+    }
+  }
+  for (; x < n; ++x) {
+    const float c = col[x * S];
+    s[0] = fmaf(w[x], w[x] > 0.f ? c : 0.f, s[0]);
+  }
   return (s[0] + s[1]) + (s[2] + s[3]);
 }
 
@@ -981,24 +997,24 @@ __device__ __forceinline__ float weighted_column(const float* col, int S, const 
 //   lat = sum_latent w acc,  fr = sum_full-rank w acc,
 //   o = (P_v lat + fr) / L_g   (0 where L_g = 0: a sequence with no tokens).
 // A unit's records sit in consecutive slots of each space and arrive in
-// shared memory by bulk copies: both spaces at once when they fit in
-// kMergeBuf bytes (the usual case), else space by space in chunks merged
-// online with a running max.  Everything that does not depend on the split
-// grid (the sequence prefix, the record ranges, the unit's P_v block,
-// transposed for conflict-free reads) is done before waiting for it.
+// shared memory by bulk copies: both spaces at once when they fit (the usual
+// case), else space by space in chunks folded into running sums.  Warp w
+// owns head g = w % G and the share w / G of the latent and full-rank
+// columns; it folds every chunk on its own (warp shuffles, no block barrier),
+// so the path after the records land is short.  The product with P_v runs
+// once at the end, one thread per output row and several heads, so each
+// element of P_v is read from shared memory once per thread.  The sequence
+// prefix, the record ranges and P_v are staged before the split grid is
+// waited for.
 template <typename T, int G>
 __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const MergePlan mp = merge_plan(a.rv, a.codes != nullptr, G, a.B);
-  float* pvt = reinterpret_cast<float*>(smem + mp.pvt);      // [r_v][128 + 1]
-  float* recb = reinterpret_cast<float*>(smem + mp.recb);    // records of one chunk
-  float* fin_lat = reinterpret_cast<float*>(smem + mp.fin);  // [G][r_v]
-  float* Mh = reinterpret_cast<float*>(smem + mp.mh);        // running max per head
-  float* Lh = reinterpret_cast<float*>(smem + mp.lh);        // running denominator
-  float* Ah = reinterpret_cast<float*>(smem + mp.ah);        // rescale of this chunk
-  float* mm = reinterpret_cast<float*>(smem + mp.mm);        // [record][G]
-  float* ll = reinterpret_cast<float*>(smem + mp.ll);
-  float* wts = reinterpret_cast<float*>(smem + mp.wts);
+  float* pv = reinterpret_cast<float*>(smem + mp.pv);      // [128][r_v + 4]
+  float* recb = reinterpret_cast<float*>(smem + mp.recb);  // records of one chunk
+  float* latf = reinterpret_cast<float*>(smem + mp.latf);  // [G][r_v]
+  float* frf = reinterpret_cast<float*>(smem + mp.frf);    // [G][128]
+  float* Lf = reinterpret_cast<float*>(smem + mp.lf);      // [G]
   int* start_lat = reinterpret_cast<int*>(smem + mp.starts);
   int* start_fr = start_lat + (a.B + 1);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + mp.bars);
@@ -1006,20 +1022,18 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
 
   const int unit = blockIdx.x, b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  constexpr int kPT = kHeadDim + 1;  // padded row of the transposed basis
+  const int rv = a.codes ? a.rv : 0, PR = pv_row(a.rv);
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_fence_init();
   }
-  if (tid < G) {
-    Mh[tid] = -INFINITY;
-    Lh[tid] = 0.f;
-  }
-  if (a.codes) {
-    const float* P = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
-    for (int x = tid; x < kHeadDim * a.rv; x += kMergeThreads) {
-      const int d = x / a.rv, j = x - d * a.rv;
-      pvt[j * kPT + d] = __ldg(P + x);
+  if (rv) {
+    const float4* P = reinterpret_cast<const float4*>(a.P_v + (size_t)b * a.basis_bs +
+                                                      (size_t)kvh * kHeadDim * rv);
+    const int n4 = rv / 4;
+    for (int x = tid; x < kHeadDim * n4; x += kMergeThreads) {
+      const int d = x / n4, j4 = x - d * n4;
+      *reinterpret_cast<float4*>(pv + d * PR + 4 * j4) = __ldg(P + x);
     }
   }
   // seq_len was final before the q-fold started (an ordinary launch).
@@ -1039,23 +1053,29 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     c0[sp] = cta_of(us, total[sp], a.C);
     ncta[sp] = cta_of(us + tiles - 1, total[sp], a.C) - c0[sp] + 1;
   }
-  const int per[2] = {kConsumers, anchors ? 1 : kConsumers};
+  const int per0 = kConsumers, per1 = anchors ? 1 : kConsumers;
   const int S0 = H + G * a.rv, S1 = H + G * kHeadDim;  // floats per record
-  const int n0 = ncta[0] * per[0], n1 = ncta[1] * per[1];
-  const float* src0 = a.part_lat + (size_t)(unit + c0[0]) * per[0] * S0;
-  const float* src1 = a.part_fr + (size_t)(unit + c0[1]) * per[1] * S1;
+  const int n0 = ncta[0] * per0, n1 = ncta[1] * per1;
+  const float* src0 = a.part_lat + (size_t)(unit + c0[0]) * per0 * S0;
+  const float* src1 = a.part_fr + (size_t)(unit + c0[1]) * per1 * S1;
   const bool fused = n0 + n1 <= kMergeMaxRec && (n0 * S0 + n1 * S1) * 4 <= kMergeBuf;
+
+  // this warp: head g, columns [j0, j1) of the latent sums and [d0, d1) of
+  // the full-rank sums; lane owns columns j0 + lane + 32 i and d0 + lane + 32 i
+  constexpr int kParts = kMergeWarps / G;
+  const int g = warp % G, part = warp / G;
+  const int jn = (rv + kParts - 1) / kParts, j0 = min(rv, part * jn), j1 = min(rv, j0 + jn);
+  constexpr int dn = kHeadDim / kParts, kD = (dn + 31) / 32;
+  const int d0 = part * dn;
+  float* wts = reinterpret_cast<float*>(smem + mp.wts) + warp * (kMergeMaxRec + 4);
+  float M = -INFINITY, L = 0.f, lat[4], fr[kD];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lat[i] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kD; ++i) fr[i] = 0.f;
 
   pdl_wait();  // every record of the split kernel is visible
 
-  constexpr int kPer = (G * kHeadDim + kMergeThreads - 1) / kMergeThreads;
-  const int E_lat = a.codes ? G * a.rv : 0, E_fr = G * kHeadDim;
-  float lacc[kPer], facc[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    lacc[i] = 0.f;
-    facc[i] = 0.f;
-  }
   int chunk = 0, sp = 0, q0 = 0;
   bool ok = true;
   while (true) {
@@ -1095,55 +1115,45 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     }
     const int nq = nl + nf;
     const float* rf = recb + nl * S0;  // full-rank records of this chunk
-    // (1) (m, l) per record and head; a record whose CTA had an empty range
-    // was never written and counts as empty
-    for (int i = tid; i < nq * G; i += kMergeThreads) {
-      const int x = i / G, g = i - x * G;
-      const int s = x < nl ? 0 : 1, q = s ? f0 + x - nl : l0 + x;
-      const int cc = c0[s] + q / per[s];
-      const bool v = range_lo(cc, total[s], a.C) != range_lo(cc + 1, total[s], a.C);
-      const float* r = s ? rf + (x - nl) * S1 : recb + x * S0;
-      mm[i] = v ? r[g] : -INFINITY;
-      ll[i] = v ? r[G + g] : 0.f;
+    // max and weights of head g; a record whose CTA had an empty range was
+    // never written and gets weight 0
+    auto mval = [&](int x) -> float {
+      const bool isf = x >= nl;
+      const int q = isf ? f0 + x - nl : l0 + x;
+      const int cc = (isf ? c0[1] + q / per1 : c0[0] + q / per0);
+      const int tot = isf ? total[1] : total[0];
+      const bool v = range_lo(cc, tot, a.C) != range_lo(cc + 1, tot, a.C);
+      return v ? (isf ? rf + (x - nl) * S1 : recb + x * S0)[g] : -INFINITY;
+    };
+    float cm = -INFINITY;
+    for (int x = lane; x < nq; x += 32) cm = fmaxf(cm, mval(x));
+    const float Mn = fmaxf(M, warp_max(cm));
+    float ls = 0.f;
+    for (int x = lane; x < nq; x += 32) {
+      const float m = mval(x);
+      const float w = m > -INFINITY ? exp2f(m - Mn) : 0.f;
+      wts[x < nl ? x : x + ((4 - (nl & 3)) & 3)] = w;
+      if (w > 0.f) ls = fmaf(w, (x >= nl ? rf + (x - nl) * S1 : recb + x * S0)[G + g], ls);
     }
-    __syncthreads();
-    // (2) warp g: head g's running max, weights and denominator
-    if (warp < G) {
-      const int g = warp;
-      float cm = -INFINITY;
-      for (int x = lane; x < nq; x += 32) cm = fmaxf(cm, mm[x * G + g]);
-      cm = warp_max(cm);
-      const float Mo = Mh[g], Mn = fmaxf(Mo, cm);
-      float ls = 0.f;
-      for (int x = lane; x < nq; x += 32) {
-        const float m = mm[x * G + g];
-        const float w = m > -INFINITY ? exp2f(m - Mn) : 0.f;
-        wts[x * G + g] = w;
-        ls = fmaf(w, ll[x * G + g], ls);
-      }
-      ls = warp_sum(ls);
-      if (lane == 0) {
-        const float al = Mn > -INFINITY ? exp2f(Mo - Mn) : 1.f;
-        Ah[g] = al;
-        Mh[g] = Mn;
-        Lh[g] = fmaf(Lh[g], al, ls);
-      }
-    }
-    __syncthreads();
-    // (3) weighted sums of the accumulators
+    ls = warp_sum(ls);
+    __syncwarp();
+    const float* wts_f = wts + ((nl + 3) & ~3);  // full-rank weights, 16-byte aligned
+    const float al = Mn > -INFINITY ? exp2f(M - Mn) : 1.f;
+    M = Mn;
+    L = fmaf(L, al, ls);
+    // weighted sums; records of weight 0 are skipped (their words may be stale)
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = tid + i * kMergeThreads;
-      if (e < E_lat) {
-        const int g = e / a.rv;
-        lacc[i] = fmaf(lacc[i], Ah[g], weighted_column<G>(recb + H + e, S0, wts + g, nl));
-      }
-      if (e < E_fr) {
-        const int g = e / kHeadDim;
-        facc[i] = fmaf(facc[i], Ah[g], weighted_column<G>(rf + H + e, S1, wts + nl * G + g, nf));
-      }
+    for (int i = 0; i < 4; ++i) {
+      const int j = j0 + lane + 32 * i;
+      if (j < j1) lat[i] = fmaf(lat[i], al, weighted_sum(recb + H + g * a.rv + j, S0, wts, nl));
     }
-    __syncthreads();  // the next chunk overwrites recb, mm, ll and wts
+#pragma unroll
+    for (int i = 0; i < kD; ++i) {
+      const int d = d0 + lane + 32 * i;
+      if (lane + 32 * i < dn)
+        fr[i] = fmaf(fr[i], al, weighted_sum(rf + H + g * kHeadDim + d, S1, wts_f, nf));
+    }
+    __syncthreads();  // the next chunk overwrites recb
   }
   if (!ok) {
     if (tid == 0) {
@@ -1152,33 +1162,46 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     }
     return;
   }
-
-  // o = (P_v lat + fr) / L
+  // hand the sums over to the row-wise product with P_v
+  if (warp < kParts * G) {
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = tid + i * kMergeThreads;
-    if (e < E_lat) fin_lat[e] = lacc[i];
+    for (int i = 0; i < 4; ++i) {
+      const int j = j0 + lane + 32 * i;
+      if (j < j1) latf[g * rv + j] = lat[i];
+    }
+#pragma unroll
+    for (int i = 0; i < kD; ++i)
+      if (lane + 32 * i < dn) frf[g * kHeadDim + d0 + lane + 32 * i] = fr[i];
+    if (part == 0 && lane == 0) Lf[g] = L;
   }
   __syncthreads();
-  T* o = static_cast<T*>(a.o) + ((size_t)b * a.H_q + (size_t)kvh * G) * kHeadDim;
+  // o[g][d] = (sum_j P_v[d][j] lat[g][j] + fr[g][d]) / L_g: thread -> row d
+  // and heads [h0, h0 + kHT)
+  constexpr int kHT = (G * kHeadDim + kMergeThreads - 1) / kMergeThreads;
+  const int d = tid % kHeadDim, h0 = (tid / kHeadDim) * kHT;
+  if (h0 < G) {
+    float out[kHT];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int x = tid + i * kMergeThreads;
-    if (x >= G * kHeadDim) break;
-    const int g = x / kHeadDim, d = x - g * kHeadDim;
-    float out = facc[i];
-    if (a.codes) {
-      const float* lat = fin_lat + g * a.rv;
-      const float* col = pvt + d;
-      float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-      for (int j = 0; j < a.rv; j += 4)
+    for (int h = 0; h < kHT; ++h) out[h] = h0 + h < G ? frf[(h0 + h) * kHeadDim + d] : 0.f;
+    const float* prow = pv + d * PR;
+    for (int j = 0; j < rv; j += 4) {
+      const float4 p4 = *reinterpret_cast<const float4*>(prow + j);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) s[u] = fmaf(col[(j + u) * kPT], lat[j + u], s[u]);
-      out += (s[0] + s[1]) + (s[2] + s[3]);
+      for (int h = 0; h < kHT; ++h) {
+        if (h0 + h < G) {
+          const float4 l4 = *reinterpret_cast<const float4*>(latf + (h0 + h) * rv + j);
+          out[h] = fmaf(p4.x, l4.x, fmaf(p4.y, l4.y, fmaf(p4.z, l4.z, fmaf(p4.w, l4.w, out[h]))));
+        }
+      }
     }
-    const float L = Lh[g];
-    o[x] = from_f<T>(L > 0.f ? out / L : 0.f);
+    T* o = static_cast<T*>(a.o) + ((size_t)b * a.H_q + (size_t)kvh * G) * kHeadDim;
+#pragma unroll
+    for (int h = 0; h < kHT; ++h) {
+      if (h0 + h < G) {
+        const float Lg = Lf[h0 + h];
+        o[(h0 + h) * kHeadDim + d] = from_f<T>(Lg > 0.f ? out[h] / Lg : 0.f);
+      }
+    }
   }
 }
 
