@@ -118,14 +118,14 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
   // before reading anything (only the launch latency is hidden).
   pdl_wait();
   // 1. seq_len, and the basis into shared memory ([i][o]: P_k columns then P_v),
-  // eight 16-byte loads in flight per thread
+  // sixteen 16-byte loads in flight per thread (one round at r_k + r_v <= 128)
   const int L0 = __ldcg(a.seq_len + b);
-  if constexpr (kCluster) cluster_arrive();
   {
     const float* Pk = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rk;
     const float* Pv = a.P_v + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * a.rv;
     const int n4 = NJ / 4, total4 = kHeadDim * n4;
-    constexpr int kB = 8;
+    const uint64_t pol = l2_evict_last_policy();
+    constexpr int kB = 16;
     for (int x0 = tid; x0 < total4; x0 += kB * (int)blockDim.x) {
       float4 v[kB];
 #pragma unroll
@@ -134,8 +134,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
         v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (x < total4) {
           const int i = x / n4, o = 4 * (x - i * n4);
-          v[u] = o < a.rk ? __ldg(reinterpret_cast<const float4*>(Pk + i * a.rk + o))
-                          : __ldg(reinterpret_cast<const float4*>(Pv + i * a.rv + o - a.rk));
+          v[u] = ldg_f4_hint(reinterpret_cast<const float4*>(o < a.rk ? Pk + i * a.rk + o
+                                                               : Pv + i * a.rv + o - a.rk),
+                             pol);
         }
       }
 #pragma unroll
@@ -145,11 +146,37 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
       }
     }
   }
+  // This CTA has read seq_len: the cluster's rank 0 may advance it at the end.
+  // The arrive (release) comes after the basis loads, which are in flight
+  // together with the seq_len load, so it costs no round trip of its own.
+  if constexpr (kCluster) cluster_arrive();
   const int L1 = L0 + appended(a.n_new, a.n, b);
   const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
   const T* kin = static_cast<const T*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
   const T* vin = static_cast<const T*>(a.v) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
   const T* anc = static_cast<const T*>(a.anchors);
+
+  // Sink and window writes (step 3): token t of the input goes to slot
+  // slot_of(q) for q < wtotal.  The first 16-byte chunk of each thread is
+  // loaded now, together with the rows below, and stored after them.
+  const int w_lo = max(L0, max(a.n_sink, L1 - a.W));
+  const int n_sink_new = a.n_sink + a.W > 0 ? max(0, min(a.n_sink, L1) - L0) : 0;
+  const int n_win_new = a.n_sink + a.W > 0 ? max(0, L1 - w_lo) : 0;
+  const int wtotal = (n_sink_new + n_win_new) * 2 * NC;
+  auto wchunk = [&](int x, int& slot, int& isv, int& ch) -> const uint4* {
+    const int q = x / (2 * NC), rem = x - q * 2 * NC;
+    isv = rem / NC;
+    ch = rem - isv * NC;
+    int t;
+    if (q < n_sink_new) { t = L0 + q; slot = t; }
+    else { t = w_lo + (q - n_sink_new); slot = a.n_sink + (t - a.n_sink) % a.W; }
+    return reinterpret_cast<const uint4*>((isv ? vin : kin) + (size_t)(t - L0) * kHeadDim + ch * CE);
+  };
+  uint4 wfirst = make_uint4(0, 0, 0, 0);
+  if (tid < wtotal) {
+    int slot, isv, ch;
+    wfirst = __ldcg(wchunk(tid, slot, isv, ch));
+  }
 
   // 2. rows that become latent: evictions from the ring (token < L0, oldest
   // first), then input tokens that go straight to latent (small n only)
@@ -207,20 +234,14 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
     // before the window writes below)
   }
 
-  // 3. sink and window writes (full-rank, verbatim), 16-byte chunks
-  if (a.n_sink + a.W > 0) {
+  // 3. sink and window writes (full-rank, verbatim), 16-byte chunks; the
+  // ring slots they overwrite were read in step 2
+  {
     T* ancw = static_cast<T*>(a.anchors);
-    const int w_lo = max(L0, max(a.n_sink, L1 - a.W));
-    const int n_sink_new = max(0, min(a.n_sink, L1) - L0);
-    const int n_win_new = max(0, L1 - w_lo);
-    const int total = (n_sink_new + n_win_new) * 2 * NC;
-    for (int x = tid; x < total; x += blockDim.x) {
-      const int q = x / (2 * NC), rem = x - q * 2 * NC, isv = rem / NC, ch = rem - isv * NC;
-      int t, slot;
-      if (q < n_sink_new) { t = L0 + q; slot = t; }
-      else { t = w_lo + (q - n_sink_new); slot = a.n_sink + (t - a.n_sink) % a.W; }
-      const uint4 u = __ldcg(reinterpret_cast<const uint4*>((isv ? vin : kin) +
-                                                            (size_t)(t - L0) * kHeadDim + ch * CE));
+    for (int x = tid; x < wtotal; x += blockDim.x) {
+      int slot, isv, ch;
+      const uint4* src = wchunk(x, slot, isv, ch);
+      const uint4 u = x == tid ? wfirst : __ldcg(src);
       *reinterpret_cast<uint4*>(ancw + anchor_off<T>(a, b, kvh, slot, ch * CE, isv)) = u;
     }
   }

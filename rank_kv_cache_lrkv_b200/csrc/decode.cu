@@ -491,6 +491,7 @@ __global__ void __launch_bounds__(kFoldThreads) qfold_kernel(DecodeArgs a) {
   if (nc <= 0) return;
   const int nseg = max(1, kFoldThreads / nc), rows = (kHeadDim + nseg - 1) / nseg;
   const float* P = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * rk;
+  const uint64_t pol = l2_evict_last_policy();
   for (int col = tid; col < nseg * nc; col += kFoldThreads) {
     const int j = c0 + col % nc, seg = col / nc;
     float acc[G];
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(kFoldThreads) qfold_kernel(DecodeArgs a) {
     for (int ib = i0; ib < i1; ib += 32) {
       float pij[32];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) pij[u] = ib + u < i1 ? __ldg(P + (size_t)(ib + u) * rk + j) : 0.f;
+      for (int u = 0; u < 32; ++u) pij[u] = ib + u < i1 ? ldg_f_hint(P + (size_t)(ib + u) * rk + j, pol) : 0.f;
 #pragma unroll
       for (int u = 0; u < 32; ++u)
         if (ib + u < i1)
@@ -1031,9 +1032,10 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     const float4* P = reinterpret_cast<const float4*>(a.P_v + (size_t)b * a.basis_bs +
                                                       (size_t)kvh * kHeadDim * rv);
     const int n4 = rv / 4;
+    const uint64_t pol = l2_evict_last_policy();
     for (int x = tid; x < kHeadDim * n4; x += kMergeThreads) {
       const int d = x / n4, j4 = x - d * n4;
-      *reinterpret_cast<float4*>(pv + d * PR + 4 * j4) = __ldg(P + x);
+      *reinterpret_cast<float4*>(pv + d * PR + 4 * j4) = ldg_f4_hint(P + x, pol);
     }
   }
   // seq_len was final before the q-fold started (an ordinary launch).
