@@ -84,9 +84,9 @@ def step_bytes(wl, L):
 # context by the algorithmic bytes.
 TRAFFIC = {
     "llama3.1_8b_layer_T32768_anchors": {
-        "bytes": 205486080, "context": 32770,
-        "sources": {"decode.cu": "57ffd6ba13797a07643557fa430c9b3e330775fa31c810fee33f811d8a272b18",
-                    "common.cuh": "6ba106b4ff5a22865f4e61fe2d07c548923e766ab272fa646904ecccffe101a6"},
+        "bytes": 205418240, "context": 32769,
+        "sources": {"decode.cu": "cc5a270849cb6a21b4cedf3f1521d198ecf782dd1f47affdbadfb09c4e090c42",
+                    "common.cuh": "8dce2af1220e3508e414de083472ec6f7a22e0e1c2b9d523c5e212a703323cbc"},
     },
 }
 
