@@ -60,6 +60,20 @@ def reconstruct(P: np.ndarray, C: np.ndarray) -> np.ndarray:
     return np.asarray(C, np.float64) @ np.asarray(P, np.float64).T
 
 
+def rebase_codes(P_old: np.ndarray, P_new: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """Codes C [n, r] stored under basis P_old, re-expressed under P_new.
+
+    The pages adapt the basis online (OjaKV page, the question on online
+    subspace adaptation) but leave open what happens to codes stored under
+    the old basis.  Plain reading: a stored code stands for its rank-r
+    reconstruction x^ = P_old c (section 04's reconstruction), and re-basing
+    gives that vector's code in the new basis, c' = P_new^T x^; for an
+    orthonormal P_new this is the least-squares code of x^.  Written as the
+    two steps, reconstruct then project.
+    """
+    return project(P_new, reconstruct(P_old, C))
+
+
 def svd_basis(X: np.ndarray, r: int) -> np.ndarray:
     """Top-r right singular vectors of X [n, 128] as columns [128, r]
     (Half the Memory, section 05: plain SVD projections)."""
@@ -172,6 +186,20 @@ class LatentCacheOracle:
                         [self.codes_k[b][h], project(_basis_of(P_k, b, h), ek[h])])
                     self.codes_v[b][h] = np.concatenate(
                         [self.codes_v[b][h], project(_basis_of(P_v, b, h), ev[h])])
+
+    def rebase(self, P_k_old, P_k_new, P_v_old, P_v_new) -> None:
+        """Re-express every stored code under the new bases (rebase_codes);
+        a pair given as None leaves that side's codes as they are."""
+        for b in range(self.B):
+            for h in range(self.H_kv):
+                if P_k_old is not None:
+                    self.codes_k[b][h] = rebase_codes(_basis_of(P_k_old, b, h),
+                                                      _basis_of(P_k_new, b, h),
+                                                      self.codes_k[b][h])
+                if P_v_old is not None:
+                    self.codes_v[b][h] = rebase_codes(_basis_of(P_v_old, b, h),
+                                                      _basis_of(P_v_new, b, h),
+                                                      self.codes_v[b][h])
 
     def anchors(self, b: int, h: int):
         """Full-rank anchor rows (sink first, then window oldest first)."""

@@ -191,6 +191,71 @@ def test_evicted_tokens_use_the_basis_current_at_eviction():
     assert np.allclose(c.codes_k[0][0], exp, rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------------ re-basing
+
+def test_rebase_is_the_least_squares_code_of_the_reconstruction():
+    # pin against a different formulation: lstsq solves min ||P_new y - x^||
+    rng = np.random.default_rng(21)
+    P_old, P_new = _orth(rng, D, 16), _orth(rng, D, 16)
+    C = rng.standard_normal((9, 16))
+    got = orc.rebase_codes(P_old, P_new, C)
+    xhat = C @ P_old.T
+    want = np.linalg.lstsq(P_new, xhat.T, rcond=None)[0].T
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_rebase_onto_the_same_basis_is_the_identity():
+    rng = np.random.default_rng(22)
+    P = _orth(rng, D, 24)
+    C = rng.standard_normal((7, 24))
+    assert np.allclose(orc.rebase_codes(P, P, C), C, rtol=0, atol=1e-12)
+
+
+def test_rebase_within_the_same_span_keeps_reconstruction_and_attention():
+    # P_new = P_old Q spans the same subspace: every reconstruction, hence
+    # every score and output, is unchanged
+    rng = np.random.default_rng(23)
+    r = 12
+    P_k, P_v = _orth(rng, D, r)[None, None], _orth(rng, D, r)[None, None]
+    Qk, Qv = _orth(rng, r, r), _orth(rng, r, r)
+    P_k2, P_v2 = P_k @ Qk, P_v @ Qv
+    c = orc.LatentCacheOracle(1, 1, r, r, 1, 3)
+    k, v = rng.standard_normal((1, 1, 20, D)), rng.standard_normal((1, 1, 20, D))
+    c.append(k, v, P_k, P_v)
+    q = rng.standard_normal((1, 2, D))
+    before = c.attend(q, P_k, P_v, 1 / math.sqrt(D))
+    rec = c.codes_k[0][0] @ P_k[0, 0].T
+    c.rebase(P_k, P_k2, P_v, P_v2)
+    assert np.allclose(c.codes_k[0][0] @ P_k2[0, 0].T, rec, rtol=0, atol=1e-12)
+    after = c.attend(q, P_k2, P_v2, 1 / math.sqrt(D))
+    assert np.allclose(after, before, rtol=0, atol=1e-12)
+
+
+def test_rebase_residual_is_the_part_outside_the_new_span():
+    # ||P_new c' - x^||^2 = ||x^||^2 - ||c'||^2 for orthonormal P_new
+    # (orthogonal projection), and the residual is orthogonal to span(P_new)
+    rng = np.random.default_rng(24)
+    P_old, P_new = _orth(rng, D, 20), _orth(rng, D, 20)
+    C = rng.standard_normal((5, 20))
+    xhat = C @ P_old.T
+    c2 = orc.rebase_codes(P_old, P_new, C)
+    res = c2 @ P_new.T - xhat
+    assert np.allclose((res ** 2).sum(1), (xhat ** 2).sum(1) - (c2 ** 2).sum(1),
+                       rtol=1e-10, atol=1e-10)
+    assert np.abs(res @ P_new).max() < 1e-12
+
+
+def test_rebase_pin_catches_a_transposed_operand():
+    # a planted mistake in a copy of the oracle's arithmetic must fail the
+    # least-squares pin: projecting with P_old^T P_new instead
+    rng = np.random.default_rng(25)
+    P_old, P_new = _orth(rng, D, 16), _orth(rng, D, 16)
+    C = rng.standard_normal((9, 16))
+    wrong = C @ (P_old.T @ P_new).T
+    want = np.linalg.lstsq(P_new, (C @ P_old.T).T, rcond=None)[0].T
+    assert not np.allclose(wrong, want, rtol=0, atol=1e-6)
+
+
 # ------------------------------------------------------------ basis
 
 def test_eckart_young_tail_energy_with_planted_spectrum():
