@@ -184,6 +184,33 @@ int lrkv_oja_update(float *P, int32_t num_streams, int32_t rank,
 int lrkv_qr_orthonormalize(float *P, int32_t num_streams, int32_t rank,
                            int64_t basis_stride, void *stream);
 
+/* Re-basing of the stored codes after the bases changed.  The OjaKV page
+ * adapts the basis online (its question on online subspace adaptation) but
+ * does not say what becomes of codes stored under the old basis.  Here a
+ * stored code c stands for its rank-r reconstruction P_old c, and every
+ * latent code of every sequence and KV head is replaced by that vector's
+ * code under the new basis: c' = P_new^T (P_old c).  The sink and window
+ * anchors are full-rank and untouched; the decode calls that follow take
+ * P_new.
+ *   P_k_old, P_k_new : fp32 [Bp][H_kv][128][rank_k], 16-byte aligned, the
+ *       layout and basis_batch_stride of lrkv_compress (0: one basis shared
+ *       by every sequence).  Both NULL to leave the key codes as they are.
+ *   P_v_old, P_v_new : the same for the value codes.
+ *   workspace : at least lrkv_rebase_workspace_bytes, 16-byte aligned; the
+ *       first 4 bytes are an error word (2 = a block-table entry out of
+ *       range) that the library sets and never clears; zero it when the
+ *       workspace is allocated.
+ * Two stream-ordered launches: the per-unit r x r products P_new^T P_old in
+ * fp32, then one pass over the latent pages (read on the device from
+ * seq_len and the block table, so it follows the appends queued before it)
+ * that rounds each new code to the cache dtype once.  Returns
+ * LRKV_ERR_ARG for a half-given pair, a misaligned pointer or a short
+ * workspace. */
+size_t lrkv_rebase_workspace_bytes(const lrkv_cache *cache);
+int lrkv_rebase(const lrkv_cache *cache, const float *P_k_old, const float *P_k_new,
+                const float *P_v_old, const float *P_v_new, int64_t basis_batch_stride,
+                void *workspace, size_t workspace_bytes, void *stream);
+
 /* Dense full-rank paged KV cache: the baseline the latent cache replaces
  * (Half the Memory, section 08 compares against the full cache).  One slab
  * per (page, KV head), key chunks then value chunks:

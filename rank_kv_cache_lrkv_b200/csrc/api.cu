@@ -143,6 +143,28 @@ int lrkv_qr_orthonormalize(float* P, int32_t num_streams, int32_t rank, int64_t 
   return qr_launch(P, num_streams, rank, basis_stride, static_cast<cudaStream_t>(stream));
 }
 
+size_t lrkv_rebase_workspace_bytes(const lrkv_cache* cache) {
+  if (check_cache(cache) != LRKV_OK) return 0;
+  return rebase_workspace_bytes(cache->batch, cache->num_kv_heads, cache->rank_k, cache->rank_v);
+}
+
+int lrkv_rebase(const lrkv_cache* cache, const float* P_k_old, const float* P_k_new,
+                const float* P_v_old, const float* P_v_new, int64_t basis_batch_stride,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_cache(cache);
+  if (rc != LRKV_OK) return rc;
+  // a side is re-based when both of its bases are given
+  if (!P_k_old != !P_k_new || !P_v_old != !P_v_new) return LRKV_ERR_ARG;
+  if (!workspace || basis_batch_stride < 0 || basis_batch_stride % 4 != 0 ||
+      !aligned16(workspace) || !aligned16(P_k_old) || !aligned16(P_k_new) ||
+      !aligned16(P_v_old) || !aligned16(P_v_new))
+    return LRKV_ERR_ARG;
+  if (workspace_bytes < lrkv_rebase_workspace_bytes(cache)) return LRKV_ERR_WORKSPACE;
+  if (!P_k_old && !P_v_old) return LRKV_OK;
+  return rebase_launch(*cache, P_k_old, P_k_new, P_v_old, P_v_new, basis_batch_stride, workspace,
+                       static_cast<cudaStream_t>(stream));
+}
+
 int lrkv_dense_append(const lrkv_dense_cache* cache, const void* k, const void* v,
                       int32_t n_tokens, const int32_t* n_new, int64_t seq_stride, int64_t head_stride, void* stream) {
   int rc = check_dense(cache);

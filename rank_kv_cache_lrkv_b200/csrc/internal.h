@@ -43,4 +43,9 @@ int oja_launch(float* P, int S, int r, long long basis_stride, const void* x, in
                cudaStream_t st);
 int qr_launch(float* P, int S, int r, long long basis_stride, cudaStream_t st);
 
+size_t rebase_workspace_bytes(int B, int H_kv, int rk, int rv);
+int rebase_launch(const lrkv_cache& c, const float* Pk_old, const float* Pk_new,
+                  const float* Pv_old, const float* Pv_new, long long basis_bs, void* ws,
+                  cudaStream_t st);
+
 }  // namespace lrkv

@@ -55,7 +55,8 @@ class DenseDesc(ctypes.Structure):
 EXPORTS = ["lrkv_compress", "lrkv_decode_workspace_bytes", "lrkv_decode_attn",
            "lrkv_oja_update", "lrkv_qr_orthonormalize", "lrkv_dense_append",
            "lrkv_dense_decode_workspace_bytes", "lrkv_dense_decode_attn",
-           "lrkv_status_string", "lrkv_version", "lrkv_decode_attn_static"]
+           "lrkv_status_string", "lrkv_version", "lrkv_decode_attn_static",
+           "lrkv_rebase_workspace_bytes", "lrkv_rebase"]
 
 
 def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
@@ -75,6 +76,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "lrkv_dense_decode_workspace_bytes": (SZ, [P, I32]),
         "lrkv_dense_decode_attn": (ctypes.c_int, [P, P, I32, F32, P, P, SZ, P]),
         "lrkv_decode_attn_static": (ctypes.c_int, [P, P, I32, P, P, I64, F32, P, P]),
+        "lrkv_rebase_workspace_bytes": (SZ, [P]),
+        "lrkv_rebase": (ctypes.c_int, [P, P, P, P, P, I64, P, SZ, P]),
         "lrkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "lrkv_version": (ctypes.c_int, []),
     }
@@ -193,6 +196,26 @@ def decode_attn(cache: LatentCache, q: torch.Tensor, P_k: torch.Tensor, P_v: tor
         ctypes.byref(cache.desc), _ptr(q), q.shape[1], _ptr(P_k), _ptr(P_v), basis_batch_stride,
         float(scale), _ptr(o), _ptr(workspace), workspace.numel(), _stream(stream)))
     return o
+
+
+def rebase_workspace(cache: LatentCache, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace for lrkv_rebase."""
+    n = int(_lib.lrkv_rebase_workspace_bytes(ctypes.byref(cache.desc)))
+    if n == 0:
+        raise LrkvError("lrkv_rebase_workspace_bytes", -2)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def rebase(cache: LatentCache, P_k_old: Optional[torch.Tensor], P_k_new: Optional[torch.Tensor],
+           P_v_old: Optional[torch.Tensor], P_v_new: Optional[torch.Tensor],
+           workspace: torch.Tensor, basis_batch_stride: int = 0, stream=None) -> None:
+    """lrkv_rebase: re-express every stored latent code under the new bases,
+    c' = P_new^T (P_old c); a side whose pair is None is left as it is."""
+    for t in (P_k_old, P_k_new, P_v_old, P_v_new):
+        assert t is None or (t.dtype == torch.float32 and t.is_contiguous())
+    _check("lrkv_rebase", _lib.lrkv_rebase(
+        ctypes.byref(cache.desc), _ptr(P_k_old), _ptr(P_k_new), _ptr(P_v_old), _ptr(P_v_new),
+        basis_batch_stride, _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def decode_attn_static(cache: LatentCache, q: torch.Tensor, P_k: torch.Tensor,

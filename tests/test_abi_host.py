@@ -106,6 +106,27 @@ def test_decode_rejects_bad_calls(lrkv):
     assert L.lrkv_decode_workspace_bytes(ctypes.byref(d), 3) == 0
 
 
+def test_rebase_rejects_bad_calls(lrkv):
+    d = _desc(lrkv)
+    L = lrkv._lib
+    n = L.lrkv_rebase_workspace_bytes(ctypes.byref(d))
+    assert n == 256 + 2 * 2 * (64 * 64 + 32 * 32) * 4  # error word + R^T per unit and side
+
+    def call(pko, pkn, pvo, pvn, ws=FAKE, bs=0, nb=n):
+        return L.lrkv_rebase(ctypes.byref(d), pko, pkn, pvo, pvn, bs, ws, nb, None)
+
+    assert call(FAKE, None, None, None) == -1                        # half a pair
+    assert call(None, None, None, FAKE) == -1
+    assert call(FAKE, FAKE, None, None, ws=None) == -1
+    assert call(FAKE, FAKE, None, None, ws=ctypes.c_void_p(4100)) == -1  # misaligned
+    assert call(ctypes.c_void_p(4104), FAKE, None, None) == -1         # misaligned basis
+    assert call(FAKE, FAKE, None, None, bs=6) == -1                    # stride % 4
+    assert call(FAKE, FAKE, FAKE, FAKE, nb=n - 1) == -4                # short workspace
+    assert call(None, None, None, None) == 0                           # nothing to re-base
+    assert L.lrkv_rebase(None, FAKE, FAKE, None, None, 0, FAKE, n, None) == -1
+    assert L.lrkv_rebase_workspace_bytes(ctypes.byref(_desc(lrkv, rank_k=12))) == 0
+
+
 def test_oja_and_dense_reject_bad_calls(lrkv):
     L = lrkv._lib
     assert L.lrkv_oja_update(None, 1, 8, 1024, FAKE, 0, 0, 4, 0.1, 0, 0, None) == -1
