@@ -369,6 +369,32 @@ def run_ours(args, rank, world):
     attn_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / R
     L_now = wl.T + W + K
     abytes = step_bytes(wl, L_now)
+
+    # lrkv_rebase over the whole cache, timed as round trips to bases of the
+    # same span and back (the cache holds equivalent codes afterwards)
+    rb_ws = lrkv.rebase_workspace(cache, device=dev)
+    gq = torch.Generator().manual_seed(7)
+
+    def rotated(P):
+        Q = torch.linalg.qr(torch.randn(P.shape[-1], P.shape[-1], generator=gq,
+                                        dtype=torch.float64))[0]
+        return (P.double() @ Q.to(P.device)).float().contiguous()
+
+    Pk2, Pv2 = rotated(Pk), rotated(Pv)
+    RB = 4
+    for rep in range(RB + 1):
+        if rep == 1:
+            torch.cuda.synchronize()
+            e0.record()
+        lrkv.rebase(cache, Pk, Pk2, Pv, Pv2, rb_ws)
+        lrkv.rebase(cache, Pk2, Pk, Pv2, Pv, rb_ws)
+    e1.record()
+    torch.cuda.synchronize()
+    assert lrkv.workspace_error(rb_ws) == 0
+    rb_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / (2 * RB)
+    es = 2 if wl.dtype == "bf16" else 4
+    n_lat = max(0, L_now - wl.n_sink - wl.window)
+    rb_bytes = 2 * wl.B * wl.H_kv * n_lat * (wl.r_k + wl.r_v) * es
     pk = peaks()
     hbm = pk["hbm_gbs"] if pk else 6650.0
     achieved = abytes / (attn_ms * 1e-3) / 1e9
@@ -394,6 +420,10 @@ def run_ours(args, rank, world):
                              "achieved_GBs": round(prefill_bytes / (prefill_ms * 1e-3) / 1e9, 1),
                              "frac": round(prefill_bytes / (prefill_ms * 1e-3) / 1e9 / hbm, 4)},
         "clocks": clk.summary(),
+        "rebase": {"us_per_call": round(rb_ms * 1e3, 2), "bytes_per_call": rb_bytes,
+                   "achieved_GBs": round(rb_bytes / (rb_ms * 1e-3) / 1e9, 1),
+                   "frac": round(rb_bytes / (rb_ms * 1e-3) / 1e9 / hbm, 4),
+                   "note": "every latent code read and written once; per-unit r x r products"},
     }
 
     if not args.no_oja:

@@ -125,16 +125,27 @@ __global__ void __launch_bounds__(kRebaseThreads, 1) rebase_codes_kernel(RebaseA
     for (int w = tid; w < r * r / 4; w += kRebaseThreads)
       reinterpret_cast<float4*>(Rt)[w] = __ldcg(s4 + w);
     __syncthreads();
-    for (int q = tid; q < rows * r; q += kRebaseThreads) {
-      const int t = q / r, i = q - t * r;
-      const float* c = x + t * XS + off;
-      float s0 = 0.f, s1 = 0.f;
-      for (int j = 0; j < r; j += 2) {
-        s0 = fmaf(Rt[j * r + i], c[j], s0);
-        s1 = fmaf(Rt[(j + 1) * r + i], c[j + 1], s1);
+    // thread -> (group of kTok tokens, column i): one R^T load feeds kTok
+    // multiply-adds, the token rows are broadcast across the warp
+    constexpr int kTok = 8;
+    const int ng = (rows + kTok - 1) / kTok;
+    for (int q = tid; q < ng * r; q += kRebaseThreads) {
+      const int tg = q / r, i = q - tg * r, t0 = tg * kTok;
+      const float* c = x + t0 * XS + off;
+      float acc[kTok];
+#pragma unroll
+      for (int k = 0; k < kTok; ++k) acc[k] = 0.f;
+#pragma unroll 4
+      for (int j = 0; j < r; ++j) {
+        const float rj = Rt[j * r + i];
+#pragma unroll
+        for (int k = 0; k < kTok; ++k) acc[k] = fmaf(rj, c[k * XS + j], acc[k]);
       }
       const int col = off + i;
-      y[((size_t)(col / CE) * kLatPage + t) * CE + col % CE] = from_f<T>(s0 + s1);
+#pragma unroll
+      for (int k = 0; k < kTok; ++k)
+        if (t0 + k < rows)
+          y[((size_t)(col / CE) * kLatPage + t0 + k) * CE + col % CE] = from_f<T>(acc[k]);
     }
   }
   __syncthreads();
