@@ -407,3 +407,93 @@ def test_two_x_compression_halves_the_cache_and_values_at_quarter():
     q = g["values_at_quarter"]
     assert q["r_v"] / q["head_dim"] == q["fraction"]
     assert math.isclose(orc.compression_ratio(64, 32), 256 / 96)
+
+
+# ------------------------------------------------------------ decode from parts
+
+def _parts_case(rng, B, Hkv, G, rk, rv, lens, n_anc, per_seq_basis):
+    """Explicit per-(sequence, KV head) parts with ragged latent and anchor
+    counts, and per-sequence bases when asked."""
+    Bp = B if per_seq_basis else 1
+    Pk = rng.standard_normal((Bp, Hkv, D, rk)) * 0.3
+    Pv = rng.standard_normal((Bp, Hkv, D, rv)) * 0.3
+    Ck = [[rng.standard_normal((lens[b][h], rk)) for h in range(Hkv)] for b in range(B)]
+    Cv = [[rng.standard_normal((lens[b][h], rv)) for h in range(Hkv)] for b in range(B)]
+    Ka = [[rng.standard_normal((n_anc[b][h], D)) for h in range(Hkv)] for b in range(B)]
+    Va = [[rng.standard_normal((n_anc[b][h], D)) for h in range(Hkv)] for b in range(B)]
+    q = rng.standard_normal((B, Hkv * G, D))
+    return q, Pk, Pv, Ck, Cv, Ka, Va
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_decode_from_parts_matches_independent_loops(G):
+    """Half the Memory, section 08 (attention on the codes) with OjaKV
+    anchors: every (sequence, q head) output of decode_from_parts must equal
+    the pure-Python loop over reconstructed rows of KV head h // G, with the
+    basis of its own sequence.  Ragged latent and anchor counts per unit, one
+    unit with no latent tokens, and r_k == r_v so that a swap of the key and
+    value codes would still run (and must fail here)."""
+    rng = np.random.default_rng(300 + G)
+    B, Hkv, rk, rv = 2, 2, 6, 6
+    lens = [[5, 0], [3, 7]]
+    n_anc = [[2, 3], [0, 1]]
+    q, Pk, Pv, Ck, Cv, Ka, Va = _parts_case(rng, B, Hkv, G, rk, rv, lens, n_anc, True)
+    o = orc.decode_from_parts(q, Pk, Pv, Ck, Cv, Ka, Va, G, 0.2)
+    assert o.shape == (B, Hkv * G, D)
+    for b in range(B):
+        for h in range(Hkv * G):
+            g = h // G
+            ref = bf.attention(q[b, h].tolist(), Pk[b, g].tolist(), Pv[b, g].tolist(),
+                               Ck[b][g].tolist(), Cv[b][g].tolist(), Ka[b][g].tolist(),
+                               Va[b][g].tolist(), 0.2)
+            ref = np.array(ref)
+            assert np.max(np.abs(o[b, h] - ref)) < 1e-12 * np.max(np.abs(ref)), (b, h)
+
+
+def test_decode_from_parts_pin_catches_planted_mistakes():
+    """The loop comparison above is discriminating: the plausible mistakes
+    (head map h % G, key and value codes swapped, the shared basis of
+    sequence 0 used for every sequence) each move the output far beyond
+    the 1e-12 bar on the same data."""
+    rng = np.random.default_rng(310)
+    B, Hkv, G, r = 2, 2, 2, 6
+    lens = [[5, 4], [3, 7]]
+    n_anc = [[2, 3], [1, 1]]
+    q, Pk, Pv, Ck, Cv, Ka, Va = _parts_case(rng, B, Hkv, G, r, r, lens, n_anc, True)
+    o = orc.decode_from_parts(q, Pk, Pv, Ck, Cv, Ka, Va, G, 0.2)
+    b, h = 1, 1                      # h % G = 1 but h // G = 0
+    good = orc.latent_attention(q[b, h], Pk[b, 0], Pv[b, 0], Ck[b][0], Cv[b][0],
+                                Ka[b][0], Va[b][0], 0.2)
+    wrong = [
+        orc.latent_attention(q[b, h], Pk[b, 1], Pv[b, 1], Ck[b][1], Cv[b][1], Ka[b][1],
+                             Va[b][1], 0.2),
+        orc.latent_attention(q[b, h], Pk[b, 0], Pv[b, 0], Cv[b][0], Ck[b][0], Ka[b][0],
+                             Va[b][0], 0.2),
+        orc.latent_attention(q[b, h], Pk[0, 0], Pv[0, 0], Ck[b][0], Cv[b][0], Ka[b][0],
+                             Va[b][0], 0.2),
+    ]
+    scale = np.max(np.abs(good))
+    assert np.max(np.abs(o[b, h] - good)) < 1e-12 * scale
+    for w in wrong:
+        assert np.max(np.abs(w - good)) > 1e-3 * scale
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_decode_from_parts_equals_cache_attend(G):
+    """Parts read out of a LatentCacheOracle (sink + window + codes, per
+    sequence bases) decode to exactly what the cache's own attend gives."""
+    rng = np.random.default_rng(320 + G)
+    B, Hkv, rk, rv = 2, 2, 8, 4
+    c = orc.LatentCacheOracle(B, Hkv, rk, rv, n_sink=1, window=3)
+    Pk = rng.standard_normal((B, Hkv, D, rk)) * 0.3
+    Pv = rng.standard_normal((B, Hkv, D, rv)) * 0.3
+    k, v = rng.standard_normal((B, Hkv, 13, D)), rng.standard_normal((B, Hkv, 13, D))
+    c.append(k, v, Pk, Pv)
+    q = rng.standard_normal((B, Hkv * G, D))
+    Ck = [[c.codes_k[b][h] for h in range(Hkv)] for b in range(B)]
+    Cv = [[c.codes_v[b][h] for h in range(Hkv)] for b in range(B)]
+    Ka = [[c.anchors(b, h)[0] for h in range(Hkv)] for b in range(B)]
+    Va = [[c.anchors(b, h)[1] for h in range(Hkv)] for b in range(B)]
+    o = orc.decode_from_parts(q, Pk, Pv, Ck, Cv, Ka, Va, G, 0.15)
+    ref = c.attend(q, Pk, Pv, 0.15)
+    assert np.max(np.abs(o - ref)) < 1e-13 * np.max(np.abs(ref))
