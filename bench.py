@@ -47,9 +47,13 @@ def parse():
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-oja", action="store_true",
                    help="skip the Oja-update timing of the 28-layer stack")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the other workloads (tiny, Qwen3 8K, the rank x batch sweep, "
+                        "the 28-layer stack)")
     p.add_argument("--profile", type=int, default=0,
                    help="profiling run: prefill, then this many eager decode steps "
-                        "(append + decode attention), no timing and no JSON line")
+                        "(append + decode attention) and one re-basing, no timing and no "
+                        "JSON line")
     return p.parse_args()
 
 
@@ -137,12 +141,236 @@ def time_oja(lrkv, dev, world):
     torch.cuda.synchronize()
     ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
     ok = bool(torch.isfinite(P).all().item())
-    del x, P, P0
+    # the chunked form (P frozen within 64-token chunks) on the same rows
+    Pc = P0.clone().contiguous()
+    lrkv.oja_update_chunked(Pc[:4].clone(), x[:4, :512], wl.oja_eta, wl.oja_qr_every, 0, 64)
+    torch.cuda.synchronize()
+    e0.record()
+    lrkv.oja_update_chunked(Pc, x, wl.oja_eta, wl.oja_qr_every, 0, 64)
+    e1.record()
+    torch.cuda.synchronize()
+    cms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    # how far the chunked bases are from the sequential ones (projector gap)
+    gap = float(torch.linalg.matrix_norm(P @ P.transpose(1, 2) - Pc @ Pc.transpose(1, 2),
+                                         ord=2).max().item())
+    del x, P, P0, Pc
     torch.cuda.empty_cache()
     return {"workload": wl.name, "streams": S, "tokens_per_stream": n, "rank": r,
             "eta": wl.oja_eta, "qr_every": wl.oja_qr_every, "ms": round(ms, 3),
             "stream_steps_per_s": round(S * n / (ms * 1e-3), 1),
-            "us_per_token_step": round(ms * 1e3 / n, 4), "finite": ok}
+            "us_per_token_step": round(ms * 1e3 / n, 4), "finite": ok,
+            "chunked": {"chunk": 64, "ms": round(cms, 3), "speedup": round(ms / cms, 2),
+                        "max_projector_gap_to_sequential": round(gap, 6)}}
+
+
+def device_kv(dev, g, B, H_kv, n, dtype):
+    """Timing inputs drawn on the device: keys and values [B, H_kv, n, 128]
+    with the workload recipe's spectra (exp(-i/16) keys, exp(-i/8) values)
+    under a random rotation per KV head.  Decode and compress time do not
+    depend on the values; parity is tested on the oracle's own draws."""
+    import torch
+    out = []
+    for decay in (16.0, 8.0):
+        spec = torch.exp(-torch.arange(HEAD_DIM, device=dev, dtype=torch.float32) / decay)
+        Q = torch.linalg.qr(torch.randn(H_kv, HEAD_DIM, HEAD_DIM, device=dev, generator=g))[0]
+        x = torch.empty((B, H_kv, n, HEAD_DIM), device=dev, dtype=dtype)
+        for b in range(B):
+            z = torch.randn((H_kv, n, HEAD_DIM), device=dev, generator=g)
+            x[b] = torch.bmm(z * spec, Q).to(dtype)
+            del z
+        out.append(x)
+    return out
+
+
+def device_basis(dev, g, lead, r):
+    """Random orthonormal bases [*lead, 128, r] in fp32."""
+    import torch
+    z = torch.randn(tuple(lead) + (HEAD_DIM, r), device=dev, generator=g)
+    return torch.linalg.qr(z)[0].contiguous()
+
+
+def time_layer_decode(lrkv, dev, wl, steps, calls, world, clk, seed):
+    """One layer of workload wl on device draws: prefill compress, then
+    `steps` decode steps (append + decode attention) captured in a CUDA graph
+    and timed, then `calls` decode-attention calls alone (the roofline)."""
+    import torch
+    from rank_kv_cache_lrkv_b200 import replicas
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    n = wl.T + steps + 1
+    Kd, Vd = device_kv(dev, g, wl.B, wl.H_kv, n, dt)
+    Pk, Pv = device_basis(dev, g, (wl.H_kv,), wl.r_k), device_basis(dev, g, (wl.H_kv,), wl.r_v)
+    qs = (torch.randn((steps + 1, wl.B, wl.H_q, HEAD_DIM), device=dev, generator=g)
+          / HEAD_DIM ** 0.5).to(dt)
+    cache = lrkv.LatentCache(wl.B, wl.H_kv, wl.r_k, wl.r_v, n, wl.n_sink, wl.window, dtype=dt,
+                             device=dev)
+    lrkv.compress(cache, Kd[:, :, :wl.T], Vd[:, :, :wl.T], Pk, Pv)
+    ws = lrkv.decode_workspace(cache, wl.H_q, device=dev)
+    o = torch.empty_like(qs[0])
+
+    def step(s):
+        t = wl.T + s
+        lrkv.compress(cache, Kd[:, :, t:t + 1], Vd[:, :, t:t + 1], Pk, Pv)
+        lrkv.decode_attn(cache, qs[s], Pk, Pv, wl.scale, o, ws)
+
+    step(0)  # warm: module loading, attributes
+    torch.cuda.synchronize()
+    gs = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gs, capture_error_mode="relaxed"):
+        for s in range(1, steps + 1):
+            step(s)
+    saved = cache.seq_len.clone()
+    gs.replay()
+    torch.cuda.synchronize()
+    cache.seq_len.copy_(saved)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        gs.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ga = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ga, capture_error_mode="relaxed"):
+        for _ in range(calls):
+            lrkv.decode_attn(cache, qs[0], Pk, Pv, wl.scale, o, ws)
+    ga.replay()
+    torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        ga.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    attn_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / calls
+    assert lrkv.workspace_error(ws) == 0
+    L = wl.T + steps + 1
+    nbytes = step_bytes(wl, L)
+    del gs, ga, cache, Kd, Vd
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(wl.B * steps * world / (ms * 1e-3), 1),
+            "us_per_step": round(ms * 1e3 / steps, 3),
+            "attn_us": round(attn_ms * 1e3, 3), "bytes_per_call": nbytes,
+            "attn_GBs": round(nbytes / (attn_ms * 1e-3) / 1e9, 1), "context": L}
+
+
+def time_sweep(lrkv, dev, world, clk, hbm, steps, calls):
+    """Rank x batch sweep on the Qwen3-1.7B-shaped layer at T=16384: decode
+    tokens/s and the roofline fraction of decode attention per point."""
+    from rank_kv_cache_lrkv_b200 import workloads as wk
+    pts = []
+    for B in wk.SWEEP_BATCHES:
+        for r_k, r_v in wk.SWEEP_RANKS:
+            wl = wk.qwen3_sweep_point(r_k, r_v, B)
+            res = time_layer_decode(lrkv, dev, wl, steps, calls, world, clk,
+                                    seed=1000 + 7 * B + r_k + r_v)
+            res.update({"B": B, "r_k": r_k, "r_v": r_v,
+                        "frac": round(res["attn_GBs"] / hbm, 4)})
+            pts.append(res)
+    return {"workload": "qwen3_1.7b_layer_T16384 rank x batch sweep", "T": 16384, "H_q": 16,
+            "H_kv": 8, "steps": steps, "calls": calls,
+            "inputs": "device draws with the recipe's spectra; random orthonormal bases",
+            "points": pts}
+
+
+def time_stack(lrkv, dev, world, clk, steps):
+    """The 28-layer Qwen3-1.7B-shaped stack (B=2, T=32768, r 48/48, bases per
+    sequence): decode tokens/s over all layers (a step appends one token and
+    attends at every layer), then one decode-time basis update of the whole
+    stack: Oja over 512 generated tokens for every (layer, K|V, sequence, KV
+    head) stream (896 streams) followed by re-basing every layer's codes."""
+    import torch
+    from rank_kv_cache_lrkv_b200 import replicas
+    from rank_kv_cache_lrkv_b200 import workloads as wk
+    wl = wk.QWEN3_STACK_OJA
+    B, H, r, T, Lyr = wl.B, wl.H_kv, wl.r_k, wl.T, wl.layers
+    g = torch.Generator(device=dev)
+    g.manual_seed(2828)
+    P = device_basis(dev, g, (Lyr, 2, B, H), r)        # [layer][K|V][b][h][128][r]
+    bs = H * HEAD_DIM * r
+    caches, news = [], []
+    for layer in range(Lyr):
+        Kd, Vd = device_kv(dev, g, B, H, T + steps + 1, torch.bfloat16)
+        c = lrkv.LatentCache(B, H, r, r, T + steps + 1, dtype=torch.bfloat16, device=dev)
+        lrkv.compress(c, Kd[:, :, :T], Vd[:, :, :T], P[layer, 0], P[layer, 1],
+                      basis_batch_stride=bs)
+        caches.append(c)
+        news.append((Kd[:, :, T:].clone(), Vd[:, :, T:].clone()))
+        del Kd, Vd
+    qs = (torch.randn((steps + 1, Lyr, B, wl.H_q, HEAD_DIM), device=dev, generator=g)
+          / HEAD_DIM ** 0.5).to(torch.bfloat16)
+    ws = [lrkv.decode_workspace(c, wl.H_q, device=dev) for c in caches]
+    o = torch.empty_like(qs[0, 0])
+
+    def step(s):
+        for layer in range(Lyr):
+            kn, vn = news[layer]
+            lrkv.compress(caches[layer], kn[:, :, s:s + 1], vn[:, :, s:s + 1], P[layer, 0],
+                          P[layer, 1], basis_batch_stride=bs)
+            lrkv.decode_attn(caches[layer], qs[s, layer], P[layer, 0], P[layer, 1], wl.scale, o,
+                             ws[layer], basis_batch_stride=bs)
+
+    step(0)
+    torch.cuda.synchronize()
+    gs = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gs, capture_error_mode="relaxed"):
+        for s in range(1, steps + 1):
+            step(s)
+    saved = [c.seq_len.clone() for c in caches]
+    gs.replay()
+    torch.cuda.synchronize()
+    for c, sv in zip(caches, saved):
+        c.seq_len.copy_(sv)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        gs.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    assert all(lrkv.workspace_error(w) == 0 for w in ws)
+    del gs
+    stack_bytes = Lyr * step_bytes(wl, T + steps + 1)
+    out = {"workload": wl.name, "layers": Lyr, "B": B, "T": T, "r_k": r, "r_v": r,
+           "steps": steps, "tokens_per_s": round(B * steps * world / (ms * 1e-3), 1),
+           "us_per_step": round(ms * 1e3 / steps, 2),
+           "GBs_per_step": round(stack_bytes / (ms * 1e-3 / steps) / 1e9, 1)}
+    # decode-time update of the whole stack (eta 1e-3, QR every 256, tokens
+    # counted on from the prompt), then every layer's codes re-based
+    n_upd = wl.oja_decode_every
+    S = Lyr * 2 * B * H
+    x = torch.empty((S, n_upd, HEAD_DIM), device=dev, dtype=torch.bfloat16)
+    for s0 in range(0, S, 64):
+        x[s0:s0 + 64] = device_kv(dev, g, 1, min(64, S - s0), n_upd, torch.bfloat16)[0][0]
+    Pflat = P.view(S, HEAD_DIM, r)
+    rws = [lrkv.rebase_workspace(c, device=dev) for c in caches]
+    P_old = torch.empty_like(P)
+
+    def update():
+        P_old.copy_(P)
+        lrkv.oja_update(Pflat, x, wl.oja_eta, wl.oja_qr_every, T)
+        for layer in range(Lyr):
+            lrkv.rebase(caches[layer], P_old[layer, 0], P[layer, 0], P_old[layer, 1],
+                        P[layer, 1], rws[layer], basis_batch_stride=bs)
+
+    update()  # warm
+    torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        update()
+        e1.record()
+        torch.cuda.synchronize()
+    ums = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    assert all(lrkv.workspace_error(w) == 0 for w in rws)
+    out["decode_oja"] = {"streams": S, "tokens": n_upd, "rank": r, "ms": round(ums, 3),
+                         "note": "Oja over the last 512 generated tokens of every stream, "
+                                 "then lrkv_rebase of all 28 layers; once per 512 steps",
+                         "share_of_512_steps": round(ums / (512 * ms / steps), 4)}
+    del caches, news, x, P, P_old
+    torch.cuda.empty_cache()
+    return out
 
 
 def dense_step_bytes(wl, L):
@@ -167,6 +395,8 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = None
         self.max_mhz = None
+        self.active = False     # set around each timed region
+        self.regions = 0
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -179,13 +409,28 @@ class ClockSampler:
     def _run(self):
         nv = self.nv
         while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append((mhz, rs))
-            except Exception:
-                pass
+            if self.active:
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    if self.active:
+                        self.samples.append((mhz, rs))
+                except Exception:
+                    pass
             time.sleep(self.period)
+
+    def region(self):
+        """Context manager marking one timed region (sampled while open)."""
+        clk = self
+
+        class _Region:
+            def __enter__(self_inner):
+                clk.active = True
+                clk.regions += 1
+
+            def __exit__(self_inner, *a):
+                clk.active = False
+        return _Region()
 
     def __enter__(self):
         if self.nv:
@@ -217,7 +462,8 @@ class ClockSampler:
                 if rs & bit and n != "gpu_idle":
                     seen.add(n)
         return {"sm_mhz": mhz[len(mhz) // 2] if mhz else None, "sm_max_mhz": self.max_mhz,
-                "samples": len(mhz), "reasons": sorted(seen)}
+                "samples": len(mhz), "timed_regions": self.regions, "reasons": sorted(seen),
+                "note": "NVML polled every 2 ms while any timed region of this run was open"}
 
 
 # ------------------------------------------------------------------ oracle
@@ -293,16 +539,19 @@ def run_ours(args, rank, world):
                              dtype=Kd.dtype, device=dev)
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(dev.index)
+    clk.__enter__()
     # warm the prefill kernels (module loading) on a small cache first
     small = lrkv.LatentCache(wl.B, wl.H_kv, wl.r_k, wl.r_v, 1024, wl.n_sink, wl.window,
                              dtype=Kd.dtype, device=dev)
     lrkv.compress(small, Kd[:, :, :1024], Vd[:, :, :1024], Pk, Pv)
     torch.cuda.synchronize()
     del small
-    e0.record()
-    lrkv.compress(cache, Kd[:, :, :wl.T], Vd[:, :, :wl.T], Pk, Pv)
-    e1.record()
-    torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        lrkv.compress(cache, Kd[:, :, :wl.T], Vd[:, :, :wl.T], Pk, Pv)
+        e1.record()
+        torch.cuda.synchronize()
     prefill_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
     # prefill bytes: K and V rows read, codes and anchors written
     n_lat = wl.T - wl.n_sink - wl.window
@@ -320,9 +569,25 @@ def run_ours(args, rank, world):
     if args.profile:
         for s in range(min(args.profile, wl.n_decode)):
             step(s)
+        # one re-basing onto a rotated basis of the same span (a profiler
+        # selects it by kernel name)
+        g = torch.Generator().manual_seed(7)
+        Qk = torch.linalg.qr(torch.randn(wl.r_k, wl.r_k, generator=g, dtype=torch.float64))[0]
+        Pk2 = (Pk.double() @ Qk.to(dev)).float().contiguous()
+        rb_ws = lrkv.rebase_workspace(cache, device=dev)
+        lrkv.rebase(cache, Pk, Pk2, Pv, Pv, rb_ws)
+        # a chunked and a sequential Oja update, 64 streams x 2048 tokens, r 48
+        g2 = torch.Generator(device=dev)
+        g2.manual_seed(11)
+        xo = (torch.randn(64, 2048, HEAD_DIM, device=dev, generator=g2) * 0.3).to(torch.bfloat16)
+        Po = torch.linalg.qr(torch.randn(64, HEAD_DIM, 48, device=dev, generator=g2))[0]
+        lrkv.oja_update_chunked(Po.contiguous(), xo, 1e-3, 256, 0, 64)
+        lrkv.oja_update(Po.contiguous(), xo, 1e-3, 256, 0)
         torch.cuda.synchronize()
-        assert lrkv.workspace_error(ws) == 0
-        print(f"profile run: {wl.name}, prefill + {args.profile} decode steps")
+        assert lrkv.workspace_error(ws) == 0 and lrkv.workspace_error(rb_ws) == 0
+        clk.__exit__()
+        print(f"profile run: {wl.name}, prefill + {args.profile} decode steps, one re-basing, "
+              "a chunked and a sequential Oja update")
         return None
 
     for s in range(W):
@@ -340,11 +605,10 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     cache.seq_len.copy_(saved_len)
     torch.cuda.synchronize()
-    L_mid = wl.T + W + K // 2
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clk:
+    with clk.region():
         e0.record()
         g.replay()
         e1.record()
@@ -362,10 +626,11 @@ def run_ours(args, rank, world):
             lrkv.decode_attn(cache, qs[0], Pk, Pv, wl.scale, o, ws)
     g2.replay()
     torch.cuda.synchronize()
-    e0.record()
-    g2.replay()
-    e1.record()
-    torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        g2.replay()
+        e1.record()
+        torch.cuda.synchronize()
     attn_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / R
     L_now = wl.T + W + K
     abytes = step_bytes(wl, L_now)
@@ -382,14 +647,16 @@ def run_ours(args, rank, world):
 
     Pk2, Pv2 = rotated(Pk), rotated(Pv)
     RB = 4
-    for rep in range(RB + 1):
-        if rep == 1:
-            torch.cuda.synchronize()
-            e0.record()
-        lrkv.rebase(cache, Pk, Pk2, Pv, Pv2, rb_ws)
-        lrkv.rebase(cache, Pk2, Pk, Pv2, Pv, rb_ws)
-    e1.record()
+    lrkv.rebase(cache, Pk, Pk2, Pv, Pv2, rb_ws)
+    lrkv.rebase(cache, Pk2, Pk, Pv2, Pv, rb_ws)
     torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        for rep in range(RB):
+            lrkv.rebase(cache, Pk, Pk2, Pv, Pv2, rb_ws)
+            lrkv.rebase(cache, Pk2, Pk, Pv2, Pv, rb_ws)
+        e1.record()
+        torch.cuda.synchronize()
     assert lrkv.workspace_error(rb_ws) == 0
     rb_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / (2 * RB)
     es = 2 if wl.dtype == "bf16" else 4
@@ -419,7 +686,6 @@ def run_ours(args, rank, world):
                              "bytes": prefill_bytes,
                              "achieved_GBs": round(prefill_bytes / (prefill_ms * 1e-3) / 1e9, 1),
                              "frac": round(prefill_bytes / (prefill_ms * 1e-3) / 1e9 / hbm, 4)},
-        "clocks": clk.summary(),
         "rebase": {"us_per_call": round(rb_ms * 1e3, 2), "bytes_per_call": rb_bytes,
                    "achieved_GBs": round(rb_bytes / (rb_ms * 1e-3) / 1e9, 1),
                    "frac": round(rb_bytes / (rb_ms * 1e-3) / 1e9 / hbm, 4),
@@ -427,7 +693,8 @@ def run_ours(args, rank, world):
     }
 
     if not args.no_oja:
-        out["oja_update"] = time_oja(lrkv, dev, world)
+        with clk.region():
+            out["oja_update"] = time_oja(lrkv, dev, world)
 
     if not args.no_dense:
         dc = lrkv.DenseCache(wl.B, wl.H_kv, cap, dtype=Kd.dtype, device=dev)
@@ -440,10 +707,11 @@ def run_ours(args, rank, world):
                 lrkv.dense_append(dc, Kd[:, :, t:t + 1], Vd[:, :, t:t + 1])
                 lrkv.dense_decode_attn(dc, qs[s], wl.scale, o, dws)
         torch.cuda.synchronize()
-        e0.record()
-        g3.replay()
-        e1.record()
-        torch.cuda.synchronize()
+        with clk.region():
+            e0.record()
+            g3.replay()
+            e1.record()
+            torch.cuda.synchronize()
         dms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
         g4 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g4, capture_error_mode="relaxed"):
@@ -451,10 +719,11 @@ def run_ours(args, rank, world):
                 lrkv.dense_decode_attn(dc, qs[0], wl.scale, o, dws)
         g4.replay()
         torch.cuda.synchronize()
-        e0.record()
-        g4.replay()
-        e1.record()
-        torch.cuda.synchronize()
+        with clk.region():
+            e0.record()
+            g4.replay()
+            e1.record()
+            torch.cuda.synchronize()
         dattn = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / R
         db = dense_step_bytes(wl, L_now)
         out["dense_baseline"] = {
@@ -465,32 +734,56 @@ def run_ours(args, rank, world):
 
     if E:
         # End to end through the public API with host buffers: per step the
-        # new k, v and q are copied from pinned host memory, and o read back.
+        # new k, v and q (packed in one pinned host buffer) are copied to the
+        # device in one transfer, and o is read back.
         a0 = wl.T + W + K
-        kh = inp["K"][:, :, a0:a0 + E].permute(2, 0, 1, 3).unsqueeze(3).contiguous().pin_memory()
-        vh = inp["V"][:, :, a0:a0 + E].permute(2, 0, 1, 3).unsqueeze(3).contiguous().pin_memory()
-        qh = wk.layer_queries(wl)[W + K:W + K + E].contiguous().pin_memory()
+        nk = wl.B * wl.H_kv * HEAD_DIM
+        nq = wl.B * wl.H_q * HEAD_DIM
+        host_in = torch.empty((E, 2 * nk + nq), dtype=Kd.dtype).pin_memory()
+        host_in[:, :nk] = inp["K"][:, :, a0:a0 + E].permute(2, 0, 1, 3).reshape(E, nk)
+        host_in[:, nk:2 * nk] = inp["V"][:, :, a0:a0 + E].permute(2, 0, 1, 3).reshape(E, nk)
+        host_in[:, 2 * nk:] = wk.layer_queries(wl)[W + K:W + K + E].reshape(E, nq)
         oh = torch.empty((E,) + tuple(o.shape), dtype=o.dtype).pin_memory()
-        kd = torch.empty((wl.B, wl.H_kv, 1, HEAD_DIM), dtype=Kd.dtype, device=dev)
-        vd = torch.empty_like(kd)
-        qd = torch.empty_like(qs[0])
+        dev_in = torch.empty((2 * nk + nq,), dtype=Kd.dtype, device=dev)
+        kd = dev_in[:nk].view(wl.B, wl.H_kv, 1, HEAD_DIM)
+        vd = dev_in[nk:2 * nk].view(wl.B, wl.H_kv, 1, HEAD_DIM)
+        qd = dev_in[2 * nk:].view(wl.B, wl.H_q, HEAD_DIM)
         torch.cuda.synchronize()
-        e0.record()
-        for s in range(E):
-            kd.copy_(kh[s], non_blocking=True)
-            vd.copy_(vh[s], non_blocking=True)
-            qd.copy_(qh[s], non_blocking=True)
-            lrkv.compress(cache, kd, vd, Pk, Pv)
-            lrkv.decode_attn(cache, qd, Pk, Pv, wl.scale, o, ws)
-            oh[s].copy_(o, non_blocking=True)
-        e1.record()
-        torch.cuda.synchronize()
+        with clk.region():
+            e0.record()
+            for s in range(E):
+                dev_in.copy_(host_in[s], non_blocking=True)
+                lrkv.compress(cache, kd, vd, Pk, Pv)
+                lrkv.decode_attn(cache, qd, Pk, Pv, wl.scale, o, ws)
+                oh[s].copy_(o, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
         ems = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
-        es = kd.element_size()
+        es = Kd.element_size()
         out["e2e"] = {"value": round(replicas.aggregate_tokens_per_s(wl.B, E, world, ems), 2),
                       "unit": "tokens/s",
-                      "h2d_bytes_per_step": 2 * kd.numel() * es + qd.numel() * es,
+                      "h2d_bytes_per_step": (2 * nk + nq) * es,
                       "d2h_bytes_per_step": o.numel() * es, "steps": E}
+
+    # the other workloads: decode tokens/s and roofline fraction of each
+    if not args.no_workloads:
+        S2, C2 = min(max(K, 8), 32), 50
+        del g, g2
+        torch.cuda.empty_cache()
+        extra = {}
+        for key, w in (("tiny_single_head_fp32", wk.TINY_SINGLE_HEAD),
+                       ("qwen3_1.7b_layer_T8192", wk.QWEN3_LAYER_8K)):
+            shard = replicas.shard(w, rank, world)
+            res = time_layer_decode(lrkv, dev, shard, S2, C2, world, clk, seed=77)
+            res.update({"B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "T": w.T, "r_k": w.r_k,
+                        "r_v": w.r_v, "dtype": w.dtype,
+                        "frac": round(res["attn_GBs"] / hbm, 4)})
+            extra[key] = res
+        out["workloads"] = extra
+        out["sweep"] = time_sweep(lrkv, dev, world, clk, hbm, S2, C2)
+        out["stack"] = time_stack(lrkv, dev, world, clk, min(max(K, 4), 16))
+    clk.__exit__()
+    out["clocks"] = clk.summary()
     if rank == 0 and world == 1 and not args.no_cpu:
         n, per_unit = OracleUnit(wl, inp).run(args.cpu_seconds)
         rate = wl.B / (per_unit * wl.B * wl.H_kv)

@@ -44,8 +44,31 @@ enum {
   LRKV_ERR_CUDA = -5         /* a CUDA runtime call or launch failed        */
 };
 
-/* Element type of K/V inputs, codes, anchors, q and o. */
-enum { LRKV_BF16 = 0, LRKV_F32 = 1 };
+/* Element type of K/V inputs, codes, anchors, q and o.  LRKV_BF16_Q8: K/V
+ * inputs, anchors, q and o are bf16, and the latent codes are stored as
+ * per-token int8 with one fp32 scale per (token, KV head, side): the Palu
+ * abstract (low-rank codes are quantisation-friendly) and the LowRAM
+ * abstract (low-rank compression composes with quantisation) combine the
+ * two; the pages give no scheme, and this one is symmetric per token,
+ * s = max_j |c_j| / 127 and q_j = round-half-even(c_j / s), decided in fp32.
+ * Attention reads the dequantised codes q_j s. */
+enum { LRKV_BF16 = 0, LRKV_F32 = 1, LRKV_BF16_Q8 = 2, LRKV_BF16_VA = 3 };
+
+/* LRKV_BF16_VA: value amortisation (LowRAM abstract: within a head, values
+ * are largely predictable from their keys; a light per-head predictor is
+ * fitted at test time and residuals are stored only for the tokens it
+ * reconstructs worst).  The pages give neither the predictor's form nor the
+ * selection rule; here, per (sequence, KV head), a linear map A (rank_k x
+ * rank_v, fp32) predicts the value code from the key code, c_v ~ A^T c_k,
+ * fitted by least squares over the prompt's latent tokens, and each 64-token
+ * page keeps the value residual c_v - A^T c_k of its LRKV_VA_KEEP tokens
+ * with the largest residual norm (ties: the earlier token).  No value codes
+ * are stored; attention reads A^T c_k (+ the kept residual).  A slab holds
+ *   [rank_k / 8][64][8] bf16 key codes, [rank_v / 8][16][8] bf16 residuals,
+ *   int32 [16] page row of each residual slot (-1 empty), fp32 [16] squared
+ *   residual norm of each slot,
+ * 128 * rank_k + 32 * rank_v + 128 bytes in all. */
+#define LRKV_VA_KEEP 16
 
 #define LRKV_HEAD_DIM 128
 #define LRKV_PAGE_TOKENS 64    /* tokens per latent code page */
@@ -63,6 +86,10 @@ enum { LRKV_BF16 = 0, LRKV_F32 = 1 };
  *   codes[num_pages][num_kv_heads][(rank_k + rank_v) / CE][LRKV_PAGE_TOKENS][CE]
  * Latent token j of sequence b (the j-th token that left the window) lives
  * in page block_table[b * max_pages_per_seq + j / 64], row j % 64.
+ * With LRKV_BF16_Q8 a chunk holds 16 int8 codes and the slab ends with the
+ * scales: [(rank_k + rank_v) / 16][64][16] int8, then [64][2] fp32 (key
+ * scale, value scale per token); one slab is 64 * (rank_k + rank_v) + 512
+ * bytes, and both ranks must be multiples of 16.
  *
  * Anchors (full-rank sink + window ring), chunk-major tiles of 32 slots with
  * the key's 128 dims first, then the value's:
@@ -71,6 +98,11 @@ enum { LRKV_BF16 = 0, LRKV_F32 = 1 };
  * when n_sink == 1; token t >= n_sink of the window sits in slot
  * n_sink + (t - n_sink) % window.  The valid slots of a sequence of L tokens
  * are the first min(L, n_sink) + min(L - sink, window) slots.
+ *
+ * The block table may scatter pages over the pool in any order.  Entries
+ * out of [0, num_pages) are never dereferenced: writes to them are skipped
+ * and decode and re-basing set error word 2.  lrkv_compress and lrkv_rebase
+ * write pages, so two entries naming one page must not both be written.
  *
  * seq_len[b] counts the tokens appended to sequence b so far; the library
  * advances it.  append_counter[b] is scratch the append kernels use to
@@ -81,8 +113,8 @@ typedef struct lrkv_cache {
   int32_t batch;             /* B, 1..LRKV_MAX_BATCH                       */
   int32_t num_kv_heads;      /* H_kv                                       */
   int32_t head_dim;          /* must be 128                                */
-  int32_t rank_k, rank_v;    /* 8..128, multiples of CE                    */
-  int32_t dtype;             /* LRKV_BF16 or LRKV_F32                      */
+  int32_t rank_k, rank_v;    /* 8..128, multiples of CE (16 for Q8)        */
+  int32_t dtype;             /* LRKV_BF16, LRKV_F32 or LRKV_BF16_Q8        */
   int32_t n_sink;            /* 0 or 1                                     */
   int32_t window;            /* W >= 0 full-rank recent tokens             */
   int32_t num_pages;         /* pages in the code pool                     */
@@ -160,7 +192,14 @@ int lrkv_decode_attn(const lrkv_cache *cache, const void *q, int32_t num_q_heads
  *   All calls share the one array: calls whose work overlaps on the GPU
  *     (other streams, other host threads) race and give wrong results;
  *     keep them ordered on one stream.  Each call clears the parts that must
- *     start at zero.  The error word is not reported by this entry point. */
+ *     start at zero.  The error word is not reported by this entry point, so
+ *     its outputs are unchecked: with a block-table entry out of range or a
+ *     timed-out wait it still returns LRKV_OK and o holds wrong values.
+ *     Callers that need that check use lrkv_decode_attn with a workspace.
+ *   The stream must belong to the current device; a device reset while the
+ *     library is loaded is not supported (the kept address goes stale).
+ *   A configuration the regular entry point rejects returns the same
+ *     status here (bad cache or heads, or LRKV_ERR_UNSUPPORTED). */
 #define LRKV_STATIC_WORKSPACE_BYTES (4u << 20)
 int lrkv_decode_attn_static(const lrkv_cache *cache, const void *q,
                             int32_t num_q_heads, const float *P_k,
@@ -179,6 +218,25 @@ int lrkv_oja_update(float *P, int32_t num_streams, int32_t rank,
                     int64_t basis_stride, const void *x, int32_t x_dtype,
                     int64_t x_stream_stride, int32_t n_tokens, float eta,
                     int32_t qr_every, int64_t tokens_seen, void *stream);
+
+/* Chunked form of the Oja update, for the prompt pass (OjaKV article: the
+ * basis adapts comprehensively during prompt prefilling; done token by token
+ * that pass is one long chain of dependent steps).  The tokens of each
+ * stream are taken in chunks of `chunk` (1..64); within a chunk every token's
+ * update uses the basis of the chunk's start, so a chunk is
+ *   Y = X P,  Z = X - Y P^T,  P <- P + eta Z^T Y,
+ * the sum of the rule's per-token updates with P frozen (chunk = 1 is the
+ * sequential rule; the two differ by a term of order eta^2 * chunk per
+ * chunk).  A chunk ends early where (tokens_seen + tokens so far) reaches a
+ * multiple of qr_every, and P is then replaced by the Q of its QR with
+ * diag(R) > 0.  Same arguments as lrkv_oja_update, plus chunk; rank <= 64
+ * and a multiple of 8 (LRKV_ERR_UNSUPPORTED otherwise); x 16-byte aligned
+ * with x_stream_stride a multiple of 16 bytes (LRKV_ERR_ARG otherwise). */
+int lrkv_oja_update_chunked(float *P, int32_t num_streams, int32_t rank,
+                            int64_t basis_stride, const void *x, int32_t x_dtype,
+                            int64_t x_stream_stride, int32_t n_tokens, float eta,
+                            int32_t qr_every, int64_t tokens_seen, int32_t chunk,
+                            void *stream);
 
 /* Replace each basis by the Q factor of its thin QR with diag(R) > 0. */
 int lrkv_qr_orthonormalize(float *P, int32_t num_streams, int32_t rank,
@@ -203,9 +261,12 @@ int lrkv_qr_orthonormalize(float *P, int32_t num_streams, int32_t rank,
  * Two stream-ordered launches: the per-unit r x r products P_new^T P_old in
  * fp32, then one pass over the latent pages (read on the device from
  * seq_len and the block table, so it follows the appends queued before it)
- * that rounds each new code to the cache dtype once.  Returns
- * LRKV_ERR_ARG for a half-given pair, a misaligned pointer or a short
- * workspace. */
+ * that rounds each new code to the cache dtype once (LRKV_BF16_Q8 caches:
+ * LRKV_ERR_UNSUPPORTED).  Pages are rewritten in
+ * place per (sequence, page), so no two block-table entries may name the
+ * same page (no shared-prefix aliasing): an aliased page would be re-based
+ * twice, or by two CTAs at once.  Returns LRKV_ERR_ARG for a half-given
+ * pair, a misaligned pointer or a short workspace. */
 size_t lrkv_rebase_workspace_bytes(const lrkv_cache *cache);
 int lrkv_rebase(const lrkv_cache *cache, const float *P_k_old, const float *P_k_new,
                 const float *P_v_old, const float *P_v_new, int64_t basis_batch_stride,

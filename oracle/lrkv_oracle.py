@@ -28,6 +28,23 @@ What it computes, and where the pages state it:
   online subspace adaptation): for each token x in order, y = P^T x and
   P <- P + eta (x - P y) y^T; after every qr_every-th token P is replaced by
   the Q factor of its QR decomposition with diag(R) > 0.
+* Value amortisation (the LowRAM abstract: within a head values are largely
+  predictable from their keys; a light per-head predictor is fitted at test
+  time and residuals are stored only for the tokens it reconstructs worst).
+  The pages give no predictor form or selection rule; the plain reading
+  taken here, in the codes' space: per (sequence, KV head) a linear map A
+  (r_k x r_v) fitted by least squares over the prompt's latent tokens,
+  C_k A ~ C_v; residual e_t = c_v,t - A^T c_k,t; in each 64-token page the
+  `keep` tokens with the largest ||e_t|| (ties: the earlier token) keep
+  their residual, and attention reads the value code A^T c_k,t (+ e_t).
+* Quantised codes.  Low-rank codes compose with quantisation (the Palu
+  abstract: quantisation-friendly low-rank codes; the LowRAM abstract: the
+  pipeline composes with quantisation).  The pages give no scheme; the plain
+  reading taken here is symmetric per-token integer codes: for each stored
+  token and side, s = max_j |c_j| / (2^(bits-1) - 1) and q_j = round(c_j / s)
+  (round half to even), and attention reads the dequantised code q s.  The
+  decision q is an integer decided from floating point, so it is taken in
+  fp32, the precision the CUDA path takes it in.
 
 Every pin that checks this file lives in tests/test_oracle_pins.py.
 """
@@ -72,6 +89,56 @@ def rebase_codes(P_old: np.ndarray, P_new: np.ndarray, C: np.ndarray) -> np.ndar
     two steps, reconstruct then project.
     """
     return project(P_new, reconstruct(P_old, C))
+
+
+def quantize_codes(C: np.ndarray, bits: int = 8):
+    """Symmetric per-token integer codes of C [n, r] (one scale per row).
+
+    s = max_j |c_j| / (2^(bits-1) - 1) and q_j = round(c_j / s), round half
+    to even, both in fp32 (the quantisation decision is taken in the
+    precision of the CUDA path); a row of zeros gets s = 0 and q = 0.
+    Returns (q as int8 [n, r], s as float32 [n]).
+    """
+    qmax = np.float32(2 ** (bits - 1) - 1)
+    C32 = np.asarray(C, np.float64).astype(np.float32)
+    amax = np.max(np.abs(C32), axis=1) if C32.shape[1] else np.zeros(C32.shape[0], np.float32)
+    s = (amax / qmax).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    q = np.rint((C32 / safe[:, None]).astype(np.float32))
+    q = np.clip(q, -qmax, qmax)
+    q[s == 0] = 0
+    return q.astype(np.int8), s
+
+
+def dequantize_codes(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """The codes a quantised row stands for: q_j s, in float64."""
+    return np.asarray(q, np.float64) * np.asarray(s, np.float64)[:, None]
+
+
+def fit_value_predictor(C_k: np.ndarray, C_v: np.ndarray) -> np.ndarray:
+    """Least-squares linear predictor of value codes from key codes:
+    A = argmin ||C_k A - C_v||_F, shape [r_k, r_v] (LowRAM abstract: a
+    lightweight per-head predictor fitted at test time)."""
+    return np.linalg.lstsq(np.asarray(C_k, np.float64), np.asarray(C_v, np.float64),
+                           rcond=None)[0]
+
+
+def amortised_value_codes(C_k: np.ndarray, C_v: np.ndarray, A: np.ndarray, keep: int,
+                          page: int = 64):
+    """Value codes as an amortised cache holds them: the prediction A^T c_k
+    for every token, plus the residual c_v - A^T c_k for the `keep` tokens of
+    each `page`-token page with the largest residual norm (ties: the earlier
+    token).  Returns (value codes [n, r_v], kept mask [n])."""
+    C_k = np.asarray(C_k, np.float64)
+    C_v = np.asarray(C_v, np.float64)
+    pred = C_k @ np.asarray(A, np.float64)
+    E = C_v - pred
+    norms = np.linalg.norm(E, axis=1)
+    kept = np.zeros(C_k.shape[0], bool)
+    for p0 in range(0, C_k.shape[0], page):
+        idx = sorted(range(p0, min(p0 + page, C_k.shape[0])), key=lambda t: (-norms[t], t))
+        kept[idx[:keep]] = True
+    return pred + np.where(kept[:, None], E, 0.0), kept
 
 
 def svd_basis(X: np.ndarray, r: int) -> np.ndarray:
@@ -149,9 +216,17 @@ class LatentCacheOracle:
     """
 
     def __init__(self, B: int, H_kv: int, r_k: int, r_v: int,
-                 n_sink: int = 0, window: int = 0):
+                 n_sink: int = 0, window: int = 0, quant_bits: int = 0,
+                 value_keep: int = 0):
         self.B, self.H_kv, self.r_k, self.r_v = B, H_kv, r_k, r_v
         self.n_sink, self.W = n_sink, window
+        # 0: codes kept as computed; 8: every stored code row is replaced by
+        # its dequantised per-token int8 form (quantize_codes)
+        self.quant_bits = quant_bits
+        # value amortisation: residuals kept per 64-token page once amortise()
+        # has fitted the predictors (None until then)
+        self.value_keep = value_keep
+        self.A = None
         self.seq_len = [0] * B
         self.sink_k = [[] for _ in range(B)]   # list of [H_kv, 128]
         self.sink_v = [[] for _ in range(B)]
@@ -183,9 +258,15 @@ class LatentCacheOracle:
                 ek, ev = np.stack(evict_k, 1), np.stack(evict_v, 1)  # [H, n, 128]
                 for h in range(self.H_kv):
                     self.codes_k[b][h] = np.concatenate(
-                        [self.codes_k[b][h], project(_basis_of(P_k, b, h), ek[h])])
+                        [self.codes_k[b][h], self._stored(project(_basis_of(P_k, b, h), ek[h]))])
                     self.codes_v[b][h] = np.concatenate(
-                        [self.codes_v[b][h], project(_basis_of(P_v, b, h), ev[h])])
+                        [self.codes_v[b][h], self._stored(project(_basis_of(P_v, b, h), ev[h]))])
+
+    def _stored(self, C: np.ndarray) -> np.ndarray:
+        """What the cache keeps of freshly computed codes C."""
+        if not self.quant_bits:
+            return C
+        return dequantize_codes(*quantize_codes(C, self.quant_bits))
 
     def rebase(self, P_k_old, P_k_new, P_v_old, P_v_new) -> None:
         """Re-express every stored code under the new bases (rebase_codes);
@@ -200,6 +281,20 @@ class LatentCacheOracle:
                     self.codes_v[b][h] = rebase_codes(_basis_of(P_v_old, b, h),
                                                       _basis_of(P_v_new, b, h),
                                                       self.codes_v[b][h])
+
+    def amortise(self) -> None:
+        """Fit every unit's value predictor over its latent tokens so far
+        (the prompt) and from now on attend over amortised value codes
+        (fit_value_predictor, amortised_value_codes)."""
+        self.A = [[fit_value_predictor(self.codes_k[b][h], self.codes_v[b][h])
+                   for h in range(self.H_kv)] for b in range(self.B)]
+
+    def value_codes(self, b: int, h: int) -> np.ndarray:
+        """The value codes attention reads for unit (b, h)."""
+        if self.A is None:
+            return self.codes_v[b][h]
+        return amortised_value_codes(self.codes_k[b][h], self.codes_v[b][h], self.A[b][h],
+                                     self.value_keep)[0]
 
     def anchors(self, b: int, h: int):
         """Full-rank anchor rows (sink first, then window oldest first)."""
@@ -223,7 +318,7 @@ class LatentCacheOracle:
                 Ka, Va = self.anchors(b, g)
                 o[b, h] = latent_attention(
                     q[b, h], _basis_of(P_k, b, g), _basis_of(P_v, b, g),
-                    self.codes_k[b][g], self.codes_v[b][g], Ka, Va, scale)
+                    self.codes_k[b][g], self.value_codes(b, g), Ka, Va, scale)
         return o
 
 
@@ -281,6 +376,39 @@ def oja_update(P: np.ndarray, X: np.ndarray, eta: float, qr_every: int,
         y = P.T @ x
         P += eta * np.outer(x - P @ y, y)
         if qr_every > 0 and (tokens_seen + j + 1) % qr_every == 0:
+            P = qr_positive(P)
+    return P
+
+
+def oja_update_blocked(P: np.ndarray, X: np.ndarray, eta: float, qr_every: int,
+                       tokens_seen: int = 0, chunk: int = 64) -> np.ndarray:
+    """Chunked form of the Oja rule: the tokens are taken in chunks of
+    `chunk`, and within a chunk every token's update uses the basis of the
+    chunk's start.
+
+    The OjaKV page adapts the basis over the prompt token by token; done so,
+    the prompt pass is one long chain of dependent steps.  Freezing P within
+    a chunk keeps Oja's per-token update, y = P^T x and (x - P y) y^T, and
+    sums it over the chunk, so a chunk is three matrix products:
+    Y = X P, Z = X - Y P^T, P <- P + eta Z^T Y.  With chunk = 1 this is the
+    sequential rule.  A chunk never straddles a QR point: chunks end where the
+    running token count (tokens_seen + tokens so far) reaches a multiple of
+    qr_every, and P is then replaced by the Q of its QR with diag(R) > 0.
+    Returns a new array.
+    """
+    P = np.array(P, np.float64, copy=True)
+    X = np.asarray(X, np.float64)
+    j = 0
+    while j < X.shape[0]:
+        n = min(chunk, X.shape[0] - j)
+        if qr_every > 0:
+            n = min(n, qr_every - (tokens_seen + j) % qr_every)
+        Xc = X[j:j + n]
+        Y = Xc @ P
+        Z = Xc - Y @ P.T
+        P = P + eta * (Z.T @ Y)
+        j += n
+        if qr_every > 0 and (tokens_seen + j) % qr_every == 0:
             P = qr_positive(P)
     return P
 

@@ -9,17 +9,21 @@ using namespace lrkv;
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-int chunk_elems(int dtype) { return dtype == LRKV_BF16 ? 8 : 4; }
+// Elements per 16-byte chunk of the K/V inputs, anchors, q and o.
+int chunk_elems(int dtype) { return dtype == LRKV_F32 ? 4 : 8; }
+// Code elements per 16-byte chunk of a latent page.
+int code_chunk_elems(int dtype) { return dtype == LRKV_BF16_Q8 ? 16 : chunk_elems(dtype); }
 
 int check_rank(int r, int dtype) {
-  if (r < chunk_elems(dtype) || r > kHeadDim || r % chunk_elems(dtype) != 0)
-    return LRKV_ERR_UNSUPPORTED;
+  const int ce = code_chunk_elems(dtype);
+  if (r < ce || r > kHeadDim || r % ce != 0) return LRKV_ERR_UNSUPPORTED;
   return LRKV_OK;
 }
 
 int check_cache(const lrkv_cache* c) {
   if (!c) return LRKV_ERR_ARG;
-  if (c->dtype != LRKV_BF16 && c->dtype != LRKV_F32) return LRKV_ERR_UNSUPPORTED;
+  if (c->dtype != LRKV_BF16 && c->dtype != LRKV_F32 && c->dtype != LRKV_BF16_Q8)
+    return LRKV_ERR_UNSUPPORTED;
   if (c->head_dim != kHeadDim) return LRKV_ERR_UNSUPPORTED;
   if (c->batch < 1 || c->batch > LRKV_MAX_BATCH || c->num_kv_heads < 1) return LRKV_ERR_ARG;
   int rc = check_rank(c->rank_k, c->dtype);
@@ -52,6 +56,20 @@ int check_heads(int H_kv, int H_q) {
 }
 
 }  // namespace
+
+namespace lrkv {
+// Why lrkv_decode_workspace_bytes returned 0: the argument check's status, or
+// the planning status (LRKV_ERR_UNSUPPORTED when the ring does not fit in
+// shared memory, LRKV_ERR_CUDA when the device query failed).
+int decode_plan_status(const lrkv_cache* cache, int H_q) {
+  int rc = check_cache(cache);
+  if (rc == LRKV_OK) rc = check_heads(cache->num_kv_heads, H_q);
+  if (rc != LRKV_OK) return rc;
+  return decode_plan_check(cache->batch, cache->num_kv_heads, H_q, cache->rank_k,
+                           cache->rank_v, true, cache->n_sink + cache->window > 0,
+                           cache->dtype);
+}
+}  // namespace lrkv
 
 extern "C" {
 
@@ -135,6 +153,22 @@ int lrkv_oja_update(float* P, int32_t num_streams, int32_t rank, int64_t basis_s
                     eta, qr_every, tokens_seen, static_cast<cudaStream_t>(stream));
 }
 
+int lrkv_oja_update_chunked(float* P, int32_t num_streams, int32_t rank, int64_t basis_stride,
+                            const void* x, int32_t x_dtype, int64_t x_stream_stride,
+                            int32_t n_tokens, float eta, int32_t qr_every, int64_t tokens_seen,
+                            int32_t chunk, void* stream) {
+  if (!P || num_streams < 1 || rank < 1 || rank > kHeadDim || n_tokens < 0 || qr_every < 0 ||
+      tokens_seen < 0 || basis_stride < (int64_t)kHeadDim * rank || chunk < 1 || chunk > 64)
+    return LRKV_ERR_ARG;
+  if (x_dtype != LRKV_BF16 && x_dtype != LRKV_F32) return LRKV_ERR_UNSUPPORTED;
+  if (rank > 64 || rank % 8 != 0) return LRKV_ERR_UNSUPPORTED;
+  if (n_tokens > 0 && !x) return LRKV_ERR_ARG;
+  if (n_tokens == 0) return LRKV_OK;
+  return oja_blocked_launch(P, num_streams, rank, basis_stride, x, x_dtype, x_stream_stride,
+                            n_tokens, eta, qr_every, tokens_seen, chunk,
+                            static_cast<cudaStream_t>(stream));
+}
+
 int lrkv_qr_orthonormalize(float* P, int32_t num_streams, int32_t rank, int64_t basis_stride,
                            void* stream) {
   if (!P || num_streams < 1 || rank < 1 || rank > kHeadDim ||
@@ -160,6 +194,7 @@ int lrkv_rebase(const lrkv_cache* cache, const float* P_k_old, const float* P_k_
       !aligned16(P_v_old) || !aligned16(P_v_new))
     return LRKV_ERR_ARG;
   if (workspace_bytes < lrkv_rebase_workspace_bytes(cache)) return LRKV_ERR_WORKSPACE;
+  if (cache->dtype == LRKV_BF16_Q8) return LRKV_ERR_UNSUPPORTED;
   if (!P_k_old && !P_v_old) return LRKV_OK;
   return rebase_launch(*cache, P_k_old, P_k_new, P_v_old, P_v_new, basis_batch_stride, workspace,
                        static_cast<cudaStream_t>(stream));

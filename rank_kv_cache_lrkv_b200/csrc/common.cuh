@@ -23,6 +23,14 @@ constexpr int kLatPage = LRKV_PAGE_TOKENS;     // tokens per latent page
 constexpr int kFrTile = LRKV_FULL_RANK_TILE;   // tokens per full-rank tile
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Value-amortised slabs (LRKV_BF16_VA): key codes [rk / 8][64][8] bf16,
+// residual rows [rv / 8][kVaKeep][8] bf16, slot rows int32 [kVaKeep], slot
+// squared norms fp32 [kVaKeep].
+constexpr int kVaKeep = LRKV_VA_KEEP;
+__host__ __device__ inline int va_slab_bytes(int rk, int rv) {
+  return kLatPage * rk * 2 + kVaKeep * rv * 2 + kVaKeep * 8;
+}
+
 // Error word values written to the first 4 bytes of a decode workspace.
 constexpr int kErrNone = 0;
 constexpr int kErrTimeout = 1;

@@ -18,6 +18,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "compress.cuh"
 #include "internal.h"
 
 namespace lrkv {
@@ -25,74 +26,13 @@ namespace lrkv {
 constexpr int kSmallN = 16;       // input tokens handled by append_kernel
 constexpr int kBulkRows = 64;     // tokens per bulk_compress CTA
 
-// Tokens sequence b appends in this call.
-__device__ inline int appended(const int* n_new, int n, int b) {
-  if (!n_new) return n;
-  const int x = n_new[b];
-  return x < 0 ? 0 : (x < n ? x : n);
-}
-
-struct AppendArgs {
-  int B, H_kv, rk, rv, n_sink, W, maxp, num_pages, n, anchor_tiles;
-  void *codes, *anchors;
-  const int* bt;
-  int* seq_len;
-  int* counter;
-  const int* n_new;  // optional per-sequence counts (<= n)
-  const void *k, *v;
-  long long seq_stride, head_stride;
-  const float *P_k, *P_v;
-  long long basis_bs;
-};
-
-// Element offset of (slot, dim d) of the key (isv = 0) or value (isv = 1)
-// in the anchor tiles of unit (b, kvh).
-template <typename T>
-__device__ inline size_t anchor_off(const AppendArgs& a, int b, int kvh, int slot, int d, int isv) {
-  constexpr int CE = Elem<T>::CE;
-  const size_t tile = ((size_t)b * a.H_kv + kvh) * a.anchor_tiles + slot / kFrTile;
-  const int chunk = isv * (kHeadDim / CE) + d / CE;
-  return (tile * (2 * kHeadDim / CE) + chunk) * kFrTile * CE + (slot % kFrTile) * CE + d % CE;
-}
-
-// Element offset of (latent index j, code dim jj) of the key (isv = 0) or
-// value (isv = 1) codes in the code pool; -1 if the page is out of range.
-template <typename T>
-__device__ inline long long code_off(const AppendArgs& a, int b, int kvh, int j, int jj, int isv) {
-  constexpr int CE = Elem<T>::CE;
-  const int pi = j / kLatPage;
-  if (pi >= a.maxp) return -1;
-  const int page = a.bt[(size_t)b * a.maxp + pi];
-  if (page < 0 || page >= a.num_pages) return -1;
-  const int nch = (a.rk + a.rv) / CE;
-  const int chunk = isv * (a.rk / CE) + jj / CE;
-  return ((((long long)page * a.H_kv + kvh) * nch + chunk) * kLatPage + j % kLatPage) * CE +
-         jj % CE;
-}
-
-// Page of latent index j of sequence b (-1 when past the block table or
-// out of the pool), and the element offset of code dim jj of that token.
-__device__ inline int latent_page(const AppendArgs& a, int b, int j) {
-  const int pi = j / kLatPage;
-  if (pi >= a.maxp) return -1;
-  const int page = a.bt[(size_t)b * a.maxp + pi];
-  return page >= 0 && page < a.num_pages ? page : -1;
-}
-template <typename T>
-__device__ inline long long code_off_in(const AppendArgs& a, int page, int kvh, int j, int jj,
-                                        int isv) {
-  constexpr int CE = Elem<T>::CE;
-  const int nch = (a.rk + a.rv) / CE;
-  const int chunk = isv * (a.rk / CE) + jj / CE;
-  return ((((long long)page * a.H_kv + kvh) * nch + chunk) * kLatPage + j % kLatPage) * CE +
-         jj % CE;
-}
-
 constexpr int kRowBatch = 16;  // token rows projected per pass
 // Dynamic shared memory of append_kernel: the unit's basis [128][r_k + r_v]
 // fp32, rows [kRowBatch][k, v][128] fp32, partial sums [256], and a page per row.
+// (+ one row of codes [256] and two scales for int8 codes)
 inline size_t append_smem_bytes(int rk, int rv) {
-  return ((size_t)kHeadDim * (rk + rv) + (size_t)kRowBatch * 2 * kHeadDim + 256 + kRowBatch) * 4;
+  return ((size_t)kHeadDim * (rk + rv) + (size_t)kRowBatch * 2 * kHeadDim + 256 + kRowBatch +
+          256 + 4) * 4;
 }
 
 // One CTA per (KV head, sequence).  Latency matters here (a decode step
@@ -112,6 +52,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
   float* xs = Ps + kHeadDim * NJ;                                      // [row][k, v][128]
   float* red = xs + kRowBatch * 2 * kHeadDim;                          // [seg][NJ]
   int* pg = reinterpret_cast<int*>(red + 256);                         // [row]
+  float* crow = red + 256 + kRowBatch;                                 // [NJ] one row's codes
+  float* qscale = crow + 256;                                          // [2] its scales
   const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
 
   // Launched with programmatic dependent launch: wait for the previous grid
@@ -221,7 +163,33 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
         red[seg * NJ + o] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       __syncthreads();
-      if (tid < NJ && pg[rr] >= 0) {
+      if (a.q8) {
+        // per-token int8: the row's codes, then one scale per side
+        // (max |c| / 127), then the codes under it
+        if (tid < NJ) {
+          float c = 0.f;
+          for (int seg = 0; seg < nseg; ++seg) c += red[seg * NJ + tid];
+          crow[tid] = c;
+        }
+        __syncthreads();
+        if (tid < 64) {
+          const int isv = tid >> 5, lo_c = isv ? a.rk : 0, hi_c = isv ? NJ : a.rk;
+          float m = 0.f;
+          for (int o = lo_c + (tid & 31); o < hi_c; o += 32) m = fmaxf(m, fabsf(crow[o]));
+          m = warp_max(m);
+          if ((tid & 31) == 0) qscale[isv] = __fdiv_rn(m, 127.f);
+        }
+        __syncthreads();
+        if (tid < NJ && pg[rr] >= 0) {
+          const int isv = tid < a.rk ? 0 : 1, jj = isv ? tid - a.rk : tid;
+          const int j = token_of(r0 + rr) - a.n_sink;
+          uint8_t* cb = static_cast<uint8_t*>(a.codes);
+          cb[q8_code_off(a, pg[rr], kvh, j, jj, isv)] =
+              static_cast<uint8_t>(static_cast<int8_t>(q8_code(crow[tid], qscale[isv])));
+          if (jj == 0)
+            *reinterpret_cast<float*>(cb + q8_scale_off(a, pg[rr], kvh, j, isv)) = qscale[isv];
+        }
+      } else if (tid < NJ && pg[rr] >= 0) {
         float c = 0.f;
         for (int seg = 0; seg < nseg; ++seg) c += red[seg * NJ + tid];
         const int isv = tid < a.rk ? 0 : 1, jj = isv ? tid - a.rk : tid;
@@ -313,26 +281,10 @@ __global__ void __launch_bounds__(256) bulk_compress_kernel(AppendArgs a) {
 // a new unit, so ldmatrix reads both operands without bank conflicts.
 constexpr int kPadRow = kHeadDim + 8;  // bf16 elements per staged row
 
-__host__ __device__ inline int round16(int x) { return (x + 15) / 16 * 16; }
 // Shared memory of bulk_compress_mma for tiles of TT tokens and B sequences.
 inline size_t bulk_mma_smem_bytes(int rk, int rv, int TT, int B) {
   return ((size_t)2 * (round16(rk) + round16(rv)) + (size_t)2 * 2 * TT) * kPadRow * 2 +
          (size_t)4 * (B + 1) * 4;
-}
-
-// First tile of CTA c when `total` tiles are split evenly over C CTAs.
-__device__ inline int bulk_range_lo(int c, int total, int C) {
-  const int q = total / C, r = total - q * C;
-  return c * q + (c * r) / C;
-}
-
-// Input rows of sequence b that go straight to latent: [in_lo, in_hi), relative to L0.
-__device__ inline void bulk_rows(const AppendArgs& a, int b, int& L0, int& in_lo, int& in_hi) {
-  L0 = __ldcg(a.seq_len + b);
-  const int L1 = L0 + appended(a.n_new, a.n, b);
-  const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
-  in_lo = max(L0, a.n_sink + s0.lat) - L0;
-  in_hi = max(in_lo, a.n_sink + s1.lat - L0);
 }
 
 template <int TT>
@@ -516,41 +468,49 @@ __global__ void __launch_bounds__(TT * 2) bulk_compress_mma(AppendArgs a) {
   }
 }
 
+// Input tokens that go straight to the latent pages (only for large n).
+// bf16: the tensor-memory kernel, or the warp-MMA kernel where the former's
+// shared memory does not fit; fp32: the SIMT kernel.
+template <typename T>
+static int bulk_launch(const AppendArgs& a, cudaStream_t st) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    int dev = 0;
+    DevInfo info;
+    int rc = current_device_info(dev, info);
+    if (rc != LRKV_OK) return rc;
+    const int sms = info.sms, optin = info.optin;
+    rc = bulk_compress_tc_launch(a, sms, optin, st);
+    if (rc != LRKV_ERR_UNSUPPORTED || a.q8) return rc;
+    // persistent: one CTA per SM; 128-token tiles (8 warps) when they fit
+    const bool big = bulk_mma_smem_bytes(a.rk, a.rv, 128, a.B) <= (size_t)optin;
+    const size_t smem = bulk_mma_smem_bytes(a.rk, a.rv, big ? 128 : 64, a.B);
+    if (smem > (size_t)optin) return LRKV_ERR_UNSUPPORTED;
+    const void* fn = big ? (const void*)bulk_compress_mma<128> : (const void*)bulk_compress_mma<64>;
+    rc = prepare_kernel(fn, false);
+    if (rc != LRKV_OK) return rc;
+    if (big)
+      bulk_compress_mma<128><<<sms, 256, smem, st>>>(a);
+    else
+      bulk_compress_mma<64><<<sms, 128, smem, st>>>(a);
+  } else {
+    dim3 g((a.n + kBulkRows - 1) / kBulkRows, a.H_kv, a.B);
+    bulk_compress_kernel<T><<<g, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+}
+
 template <typename T>
 static int compress_t(const AppendArgs& a, cudaStream_t st) {
   const bool small = a.n <= kSmallN;
   if (!small) {
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-      // persistent: one CTA per SM; 128-token tiles (8 warps) when they fit
-      int dev = 0, sms = 0, optin = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-              cudaSuccess)
-        return LRKV_ERR_CUDA;
-      const bool big = bulk_mma_smem_bytes(a.rk, a.rv, 128, a.B) <= (size_t)optin;
-      const size_t smem = bulk_mma_smem_bytes(a.rk, a.rv, big ? 128 : 64, a.B);
-      if (smem > (size_t)optin) return LRKV_ERR_UNSUPPORTED;
-      const void* fn = big ? (const void*)bulk_compress_mma<128> : (const void*)bulk_compress_mma<64>;
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-        return LRKV_ERR_CUDA;
-      if (big)
-        bulk_compress_mma<128><<<sms, 256, smem, st>>>(a);
-      else
-        bulk_compress_mma<64><<<sms, 128, smem, st>>>(a);
-    } else {
-      dim3 g((a.n + kBulkRows - 1) / kBulkRows, a.H_kv, a.B);
-      bulk_compress_kernel<T><<<g, 256, 0, st>>>(a);
-    }
-    if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
+    const int rc = bulk_launch<T>(a, st);
+    if (rc != LRKV_OK) return rc;
   }
   const size_t smem = append_smem_bytes(a.rk, a.rv);
   const bool cluster = a.H_kv <= 8;
   const void* fn = cluster ? (const void*)append_kernel<T, true> : (const void*)append_kernel<T, false>;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return LRKV_ERR_CUDA;
+  const int prc = prepare_kernel(fn, false);
+  if (prc != LRKV_OK) return prc;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.H_kv, a.B);
   cfg.blockDim = dim3(256);
@@ -578,11 +538,12 @@ int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, co
   a.B = c.batch; a.H_kv = c.num_kv_heads; a.rk = c.rank_k; a.rv = c.rank_v;
   a.n_sink = c.n_sink; a.W = c.window; a.maxp = c.max_pages_per_seq; a.num_pages = c.num_pages;
   a.n = n; a.anchor_tiles = (c.n_sink + c.window + kFrTile - 1) / kFrTile;
+  a.q8 = c.dtype == LRKV_BF16_Q8 ? 1 : 0;
   a.codes = c.codes; a.anchors = c.anchors;
   a.bt = c.block_table; a.seq_len = c.seq_len; a.counter = c.append_counter; a.n_new = n_new;
   a.k = k; a.v = v; a.seq_stride = seq_stride; a.head_stride = head_stride;
   a.P_k = P_k; a.P_v = P_v; a.basis_bs = basis_bs;
-  return c.dtype == LRKV_BF16 ? compress_t<__nv_bfloat16>(a, st) : compress_t<float>(a, st);
+  return c.dtype == LRKV_F32 ? compress_t<float>(a, st) : compress_t<__nv_bfloat16>(a, st);
 }
 
 // ------------------------------------------------------------ dense baseline

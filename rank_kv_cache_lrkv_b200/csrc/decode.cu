@@ -75,6 +75,7 @@ struct DecodeArgs {
   int C;               // CTAs of the split grid
   int NS;              // ring stages
   int stage_bytes;
+  int dq_bytes;        // int8 codes: per-consumer dequantised half page (bytes)
 };
 
 __host__ __device__ inline int hdr_floats(int G) { return ((2 * G + 3) / 4) * 4; }
@@ -87,6 +88,20 @@ __device__ inline int tiles_fr(int n) { return (n + kFrTile - 1) / kFrTile; }
 __device__ inline int range_lo(int c, int total, int C) {
   const int q = total / C, r = total - q * C;
   return c * q + (c * r) / C;
+}
+// CTAs a space of `total` tiles is spread over: at most one tile per CTA
+// short of the grid, so a small space keeps its records in few CTAs' slots
+// (the merge folds fewer records).  CTAs c >= ctas_for(...) own no tile.
+__device__ inline int ctas_for(int total, int C) { return total < C ? total : C; }
+// Tiles [lo, hi) of CTA c in a space of `total` tiles over a grid of C CTAs.
+__device__ inline void cta_range(int c, int total, int C, int& lo, int& hi) {
+  const int Ce = ctas_for(total, C);
+  if (c >= Ce) {
+    lo = hi = total;
+    return;
+  }
+  lo = range_lo(c, total, Ce);
+  hi = range_lo(c + 1, total, Ce);
 }
 // CTA whose range holds tile t (0 <= t < total).
 __device__ inline int cta_of(int t, int total, int C) {
@@ -539,11 +554,13 @@ __host__ __device__ inline bool anchor_mode(const void* fr, const int* bt_fr) {
 
 // Shared-memory plan of the split kernel (byte offsets from the base).
 struct SmemPlan {
-  int ring, full, empty, tag, start_lat, start_fr, pbuf, qown, flags, total;
+  int ring, full, empty, tag, start_lat, start_fr, pbuf, qown, flags, dq, total;
 };
 // tc: the consumers run on the tensor cores and keep their query fragments in
 // registers, so only the anchor warp needs probability and query slices.
-__host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, int G, bool tc) {
+// dq_bytes: per consumer warp, the bf16 form of half an int8 page.
+__host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, int G, bool tc,
+                                              int dq_bytes = 0) {
   const int slots = tc ? 1 : kConsumers + 1;
   SmemPlan p;
   int off = 0;
@@ -564,6 +581,7 @@ __host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, in
   p.pbuf = take(slots * kLatPage * G * 8, 16);
   p.qown = take(slots * G * kHeadDim * 4, 16);
   p.flags = take(16, 16);
+  p.dq = take(kConsumers * dq_bytes, 128);
   p.total = off;
   return p;
 }
@@ -697,19 +715,52 @@ __device__ void anchor_tile(const uint4* kch, int n_valid, const float* qv, floa
   __syncwarp();
 }
 
+// Half `half` (32 tokens) of an int8 latent slab -> bf16 chunk-major tile
+// [rk / 8 + rv / 8][32][8] in dst (the layout process_tile_mma reads), each
+// code multiplied by its token's scale and rounded to bf16 once.  Lane =
+// token; tokens at or past n are written as zeros.
+__device__ __forceinline__ void dequant_half(const uint4* slab, int half, int rk, int rv, int n,
+                                             uint4* dst, int lane) {
+  const int t = half * kFrTile + lane;
+  const float* scales = reinterpret_cast<const float*>(slab + (rk + rv) / 16 * kLatPage);
+  const bool ok = lane < n;
+  const float sk = ok ? scales[2 * t] : 0.f, sv = ok ? scales[2 * t + 1] : 0.f;
+  const int nk16 = rk / 16, n16 = (rk + rv) / 16;
+  for (int c = 0; c < n16; ++c) {
+    const float s = c < nk16 ? sk : sv;
+    const uint4 w = ok ? slab[c * kLatPage + t] : make_uint4(0, 0, 0, 0);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+      // the four int8 codes of word e4, sign-extended, times the scale
+      const int x0 = (int)(ws[e4] << 24) >> 24, x1 = (int)(ws[e4] << 16) >> 24;
+      const int x2 = (int)(ws[e4] << 8) >> 24, x3 = (int)ws[e4] >> 24;
+      o[2 * e4] = pack_bf16x2((float)x0 * s, (float)x1 * s);
+      o[2 * e4 + 1] = pack_bf16x2((float)x2 * s, (float)x3 * s);
+    }
+    dst[(2 * c) * kFrTile + lane] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[(2 * c + 1) * kFrTile + lane] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------ split kernel
 // kDense: the ring carries full-rank pages (dense baseline) instead of latent
 // pages; KS / VB: rank class of the tensor-core tiles (bf16 only).
 // 168 registers: ten warps, three on two of the SM's four sub-partitions
 // (16K registers each).  More consumer warps hide more of each warp's
 // dependent latency; fewer registers spill in the wider rank classes.
-template <typename T, int G, bool kDense, int KS, int VB>
+// kQ8: the latent pages hold per-token int8 codes and fp32 scales; each
+// consumer dequantises a page half by half into its own bf16 buffer and
+// runs the bf16 tensor-core tile on it.
+template <typename T, int G, bool kDense, int KS, int VB, bool kQ8 = false>
 __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   constexpr int CE = Elem<T>::CE;
   constexpr int NP = CE / 2;
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr bool kTC = std::is_same<T, __nv_bfloat16>::value;
-  const SmemPlan sp_ = smem_plan(a.NS, a.stage_bytes, a.B, G, kTC);
+  const SmemPlan sp_ = smem_plan(a.NS, a.stage_bytes, a.B, G, kTC, a.dq_bytes);
   uint8_t* ring = smem + sp_.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp_.full);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + sp_.empty);
@@ -742,7 +793,9 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   constexpr int rsp = kDense ? 1 : 0;
   const int* rstart = rsp == 0 ? start_lat : start_fr;
   const int rtot = rstart[a.B];
-  const int lo = range_lo(c, rtot, a.C), hi = range_lo(c + 1, rtot, a.C), N = hi - lo;
+  int lo, hi;
+  cta_range(c, rtot, a.C, lo, hi);
+  const int N = hi - lo;
 
   if (warp == kProducerWarp) {
     // ---------------- producer: lane l holds the slab address of tile base + l;
@@ -763,8 +816,8 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
       if (rsp == 0) {
         good = page >= 0 && page < a.num_pages_lat;
         const size_t slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
-        bytes = kLatPage * (a.rk + a.rv) * sizeof(T);
-        src = static_cast<const T*>(a.codes) + slab * kLatPage * (a.rk + a.rv);
+        bytes = a.stage_bytes;  // one latent slab (bf16, fp32 or int8 + scales)
+        src = static_cast<const uint8_t*>(a.codes) + slab * a.stage_bytes;
       } else {
         good = page >= 0 && page < a.num_pages_fr;
         const size_t slab = (size_t)(good ? page : 0) * a.H_kv + kvh;
@@ -833,7 +886,8 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
     } else {
     if (!anchor_mode(a.fr, a.bt_fr)) return;
     const int tot = start_fr[a.B];
-    const int flo = range_lo(c, tot, a.C), fhi = range_lo(c + 1, tot, a.C);
+    int flo, fhi;
+    cta_range(c, tot, a.C, flo, fhi);
     const int rec_stride = hdr_floats(G) + G * kHeadDim;
     int t = flo;
     while (t < fhi) {
@@ -868,7 +922,7 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   // ---------------- consumers (bf16 pages on the tensor cores, fp32 on SIMT)
   constexpr bool kTensorTiles = std::is_same<T, __nv_bfloat16>::value;
   const int w = warp - kFirstConsumer;
-  const int nck = rsp == 0 ? a.rk / CE : kHeadDim / CE;
+  const int nck = rsp == 0 ? a.rk / CE : kHeadDim / CE;  // (int8 pages: of the bf16 buffer)
   const int ncv = rsp == 0 ? a.rv / CE : kHeadDim / CE;
   const int rvd = rsp == 0 ? a.rv : kHeadDim;
   const int qdim = rsp == 0 ? a.rk : kHeadDim;
@@ -911,12 +965,32 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
         for (int vb = 0; vb < VB; ++vb)
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[hl][vb][i] = 0.f;
-      for (int tt = first; tt < ce; tt += kConsumers) {
-        const uint4* st = acquire(tt);
-        if (!st) break;
-        process_tile_mma<TT, KS, VB>(st, min(TT, ntok - (tt - ustart) * TT), nck, ncv, qf, m, l,
-                                     acc, lane);
-        release(tt);
+      if constexpr (kQ8 && !kDense) {
+        // int8 pages: each half of 32 tokens is dequantised into this warp's
+        // buffer, then run on the tensor cores as a 32-token tile
+        uint4* dq = reinterpret_cast<uint4*>(smem + sp_.dq + (size_t)w * a.dq_bytes);
+        for (int tt = first; tt < ce; tt += kConsumers) {
+          const uint4* st = acquire(tt);
+          if (!st) break;
+          const int nv = min(TT, ntok - (tt - ustart) * TT);
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            const int nh = min(kFrTile, nv - half * kFrTile);
+            if (nh <= 0) break;
+            dequant_half(st, half, a.rk, a.rv, nh, dq, lane);
+            if (half == 1 || nv <= kFrTile) release(tt);
+            process_tile_mma<kFrTile, KS, VB>(dq, nh, nck, ncv, qf, m, l, acc, lane);
+          }
+          if (nv <= 0) release(tt);
+        }
+      } else {
+        for (int tt = first; tt < ce; tt += kConsumers) {
+          const uint4* st = acquire(tt);
+          if (!st) break;
+          process_tile_mma<TT, KS, VB>(st, min(TT, ntok - (tt - ustart) * TT), nck, ncv, qf, m,
+                                       l, acc, lane);
+          release(tt);
+        }
       }
       // This warp's record for (unit, CTA); m = -inf when it had no tile.
       write_record_mma<G, VB>(rec, rvd, m, l, acc, lane);
@@ -1052,8 +1126,9 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     const int tiles = (starts[sp][b + 1] - starts[sp][b]) / a.H_kv;
     if (total[sp] == 0 || tiles == 0) continue;
     const int us = starts[sp][b] + kvh * tiles;
-    c0[sp] = cta_of(us, total[sp], a.C);
-    ncta[sp] = cta_of(us + tiles - 1, total[sp], a.C) - c0[sp] + 1;
+    const int Ce = ctas_for(total[sp], a.C);
+    c0[sp] = cta_of(us, total[sp], Ce);
+    ncta[sp] = cta_of(us + tiles - 1, total[sp], Ce) - c0[sp] + 1;
   }
   const int per0 = kConsumers, per1 = anchors ? 1 : kConsumers;
   const int S0 = H + G * a.rv, S1 = H + G * kHeadDim;  // floats per record
@@ -1124,7 +1199,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
       const int q = isf ? f0 + x - nl : l0 + x;
       const int cc = (isf ? c0[1] + q / per1 : c0[0] + q / per0);
       const int tot = isf ? total[1] : total[0];
-      const bool v = range_lo(cc, tot, a.C) != range_lo(cc + 1, tot, a.C);
+      const int Ce = ctas_for(tot, a.C);
+      const bool v = range_lo(cc, tot, Ce) != range_lo(cc + 1, tot, Ce);
       return v ? (isf ? rf + (x - nl) * S1 : recb + x * S0)[g] : -INFINITY;
     };
     float cm = -INFINITY;
@@ -1209,28 +1285,32 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
 
 // ------------------------------------------------------------ host side
 struct Plan {
-  int C, NS, stage_bytes, smem, merge_smem;
+  int C, NS, stage_bytes, dq_bytes, smem, merge_smem;
   size_t off_qlat, off_qfr, off_lat, off_fr, total;
 };
 
 static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, bool has_fr,
-                       bool anchors, int esize, Plan& p) {
-  int dev = 0, sms = 0, optin = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LRKV_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return LRKV_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-    return LRKV_ERR_CUDA;
+                       bool anchors, int esize, Plan& p, bool q8 = false) {
+  int dev = 0;
+  DevInfo info;
+  const int rc = current_device_info(dev, info);
+  if (rc != LRKV_OK) return rc;
+  const int sms = info.sms, optin = info.optin;
   const int G = H_q / H_kv;
   // the ring holds latent pages, or dense full-rank pages (no latent space)
   p.stage_bytes = has_lat ? kLatPage * (rk + rv) * esize : 2 * kFrTile * kHeadDim * esize;
+  p.dq_bytes = 0;
+  if (has_lat && q8) {  // int8 codes + scales; a bf16 half page per consumer
+    p.stage_bytes = kLatPage * (rk + rv) + 512;
+    p.dq_bytes = kFrTile * (rk + rv) * 2;
+  }
   // Leave room for a q-fold CTA beside each split CTA.
   const int budget = optin - 8 * 1024;
   const bool tc = esize == 2;  // bf16: tensor-core consumers
-  const int fixed = smem_plan(0, p.stage_bytes, B, G, tc).total + 1024;
+  const int fixed = smem_plan(0, p.stage_bytes, B, G, tc, p.dq_bytes).total + 1024;
   p.NS = std::min(kMaxStages, (budget - fixed) / p.stage_bytes);
   if (p.NS < 2) return LRKV_ERR_UNSUPPORTED;
-  p.smem = smem_plan(p.NS, p.stage_bytes, B, G, tc).total;
+  p.smem = smem_plan(p.NS, p.stage_bytes, B, G, tc, p.dq_bytes).total;
   p.C = sms;
   p.merge_smem = merge_plan(rv, has_lat, G, B).total;
   const int U = B * H_kv;
@@ -1248,12 +1328,19 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   return LRKV_OK;
 }
 
+int decode_plan_check(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, bool has_fr,
+                      int dtype) {
+  Plan p;
+  return plan_decode(B, H_kv, H_q, rk, rv, has_lat, has_fr, has_lat && has_fr,
+                     dtype == LRKV_F32 ? 4 : 2, p, dtype == LRKV_BF16_Q8);
+}
+
 size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has_lat,
                               bool has_fr, int dtype) {
   Plan p;
   // anchors: full-rank space present next to a latent one (no block table)
   if (plan_decode(B, H_kv, H_q, rk, rv, has_lat, has_fr, has_lat && has_fr,
-                  dtype == LRKV_BF16 ? 2 : 4, p) != LRKV_OK)
+                  dtype == LRKV_F32 ? 4 : 2, p, dtype == LRKV_BF16_Q8) != LRKV_OK)
     return 0;
   return p.total;
 }
@@ -1278,8 +1365,13 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
 template <typename T, int G>
 static const void* split_fn(const DecodeArgs& a) {
   if (!a.codes) return (const void*)split_kernel<T, G, true, 8, 8>;
-  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (a.dq_bytes) {  // int8 codes
+      if (a.rk <= 64 && a.rv <= 32) return (const void*)split_kernel<T, G, false, 4, 2, true>;
+      return (const void*)split_kernel<T, G, false, 8, 8, true>;
+    }
     if (a.rk <= 64 && a.rv <= 32) return (const void*)split_kernel<T, G, false, 4, 2>;
+  }
   return (const void*)split_kernel<T, G, false, 8, 8>;
 }
 
@@ -1287,21 +1379,16 @@ template <typename T, int G>
 static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st) {
   // Keep SMs in the large-shared-memory configuration while the q-fold runs,
   // so the split kernel's CTAs can start beside it without a reconfiguration.
-  cudaFuncSetAttribute(qfold_kernel<T, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                       (int)cudaSharedmemCarveoutMaxShared);
+  // (Kernel attributes are set once per device; see prepare_kernel.)
+  const void* split = split_fn<T, G>(a);
+  int rc = prepare_kernel((const void*)qfold_kernel<T, G>, true);
+  if (rc == LRKV_OK) rc = prepare_kernel(split, true);
+  if (rc == LRKV_OK) rc = prepare_kernel((const void*)merge_kernel<T, G>, false);
+  if (rc != LRKV_OK) return rc;
   qfold_kernel<T, G><<<a.B * a.H_kv * kFoldSplit, kFoldThreads, 0, st>>>(a);
   if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
-  const void* split = split_fn<T, G>(a);
-  if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) !=
-      cudaSuccess)
-    return LRKV_ERR_CUDA;
-  cudaFuncSetAttribute(split, cudaFuncAttributePreferredSharedMemoryCarveout,
-                       (int)cudaSharedmemCarveoutMaxShared);
   void* args[] = {&a};
   if (launch_pdl(split, dim3(p.C), dim3(kThreads), p.smem, st, args) != cudaSuccess)
-    return LRKV_ERR_CUDA;
-  if (cudaFuncSetAttribute(merge_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           p.merge_smem) != cudaSuccess)
     return LRKV_ERR_CUDA;
   if (launch_pdl((const void*)merge_kernel<T, G>, dim3(a.B * a.H_kv), dim3(kMergeThreads),
                  p.merge_smem, st, args) != cudaSuccess)
@@ -1322,10 +1409,10 @@ static int launch_decode_g(const DecodeArgs& a, const Plan& p, cudaStream_t st) 
 
 int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
   const bool has_lat = L.codes != nullptr, has_fr = L.fr != nullptr;
-  const int es = L.dtype == LRKV_BF16 ? 2 : 4;
+  const int es = L.dtype == LRKV_F32 ? 4 : 2;
   Plan p;
   int rc = plan_decode(L.B, L.H_kv, L.H_q, L.rk, L.rv, has_lat, has_fr,
-                       anchor_mode(L.fr, L.bt_fr), es, p);
+                       anchor_mode(L.fr, L.bt_fr), es, p, L.dtype == LRKV_BF16_Q8);
   if (rc != LRKV_OK) return rc;
   if (L.ws_bytes < p.total) return LRKV_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(L.ws);
@@ -1343,9 +1430,9 @@ int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
   a.qfr = reinterpret_cast<float*>(ws + p.off_qfr);
   a.part_lat = reinterpret_cast<float*>(ws + p.off_lat);
   a.part_fr = reinterpret_cast<float*>(ws + p.off_fr);
-  a.C = p.C; a.NS = p.NS; a.stage_bytes = p.stage_bytes;
-  if (L.dtype == LRKV_BF16) return launch_decode_g<__nv_bfloat16>(a, p, st);
-  return launch_decode_g<float>(a, p, st);
+  a.C = p.C; a.NS = p.NS; a.stage_bytes = p.stage_bytes; a.dq_bytes = p.dq_bytes;
+  if (L.dtype == LRKV_F32) return launch_decode_g<float>(a, p, st);
+  return launch_decode_g<__nv_bfloat16>(a, p, st);
 }
 
 }  // namespace lrkv

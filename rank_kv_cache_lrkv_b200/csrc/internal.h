@@ -8,6 +8,17 @@
 
 namespace lrkv {
 
+// SM count and opt-in shared memory per block of a device.
+struct DevInfo {
+  int sms, optin;
+};
+// The current device and its DevInfo, queried once per device per process.
+int current_device_info(int& dev, DevInfo& info);
+// Once per (kernel, device): allow the device's full opt-in dynamic shared
+// memory for fn and, when max_carveout, prefer the largest shared-memory
+// carveout.  Later calls return at once.
+int prepare_kernel(const void* fn, bool max_carveout);
+
 struct DecodeLaunch {
   int B, H_kv, H_q, dtype;
   const int* seq_len;
@@ -29,6 +40,11 @@ struct DecodeLaunch {
 
 size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has_lat,
                               bool has_fr, int dtype);
+// Status of planning that decode (LRKV_OK when decode_workspace_bytes > 0).
+int decode_plan_check(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, bool has_fr,
+                      int dtype);
+// Status explaining a zero lrkv_decode_workspace_bytes for this cache.
+int decode_plan_status(const lrkv_cache* cache, int H_q);
 int decode_launch(const DecodeLaunch& L, cudaStream_t st);
 
 int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, const int* n_new,
@@ -42,6 +58,14 @@ int oja_launch(float* P, int S, int r, long long basis_stride, const void* x, in
                long long x_stride, int n, float eta, int qr_every, long long tokens_seen,
                cudaStream_t st);
 int qr_launch(float* P, int S, int r, long long basis_stride, cudaStream_t st);
+int oja_blocked_launch(float* P, int S, int r, long long basis_stride, const void* x,
+                       int x_dtype, long long x_stride, int n, float eta, int qr_every,
+                       long long tokens_seen, int chunk, cudaStream_t st);
+
+size_t amortise_workspace_bytes(int B, int H_kv, int rk, int rv);
+int amortise_launch(const lrkv_cache& c, const void* v, int n, long long seq_stride,
+                    long long head_stride, const float* P_v, long long basis_bs, float* A,
+                    void* ws, cudaStream_t st);
 
 size_t rebase_workspace_bytes(int B, int H_kv, int rk, int rv);
 int rebase_launch(const lrkv_cache& c, const float* Pk_old, const float* Pk_new,

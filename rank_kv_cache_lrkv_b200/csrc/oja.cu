@@ -323,14 +323,202 @@ __global__ void __launch_bounds__(kOja2Threads, 6) oja2_kernel(float* P, int r, 
   }
 }
 
+// ---- chunked Oja (P frozen within a chunk)
+// One CTA of 128 threads per stream, r <= 64.  Per chunk of nc <= 64 tokens
+// (a chunk ends early at a QR point):
+//   Y = X P        [nc][r]    thread -> 4 tokens x r/8 columns
+//   Z = X - Y P^T  [nc][128]  in place over X; thread -> 8 tokens x 8 rows
+//   P += eta Z^T Y [128][r]   thread -> 4 rows x r/4 columns
+// in fp32 from shared memory, register-blocked so each loaded value feeds
+// several multiply-adds.  The next chunk's rows arrive by cp.async while
+// the current one is processed.  QR every qr_every tokens seen, as in the
+// sequential kernel.
+constexpr int kBlkRows = 64;     // tokens per chunk at most
+constexpr int kBlkLdX = 132;     // fp32 row stride of X / Z
+
+inline size_t oja_blocked_smem_bytes(int r, int esize) {
+  return (size_t)(kBlkRows * kBlkLdX + kBlkRows * (r + 1) + kHeadDim * (r + 1) + 2 * kHeadDim) *
+             4 +
+         (size_t)2 * kBlkRows * kHeadDim * esize;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kOjaThreads) oja_blocked_kernel(
+    float* P, int r, long long bstride, const T* __restrict__ x, long long xstride, int n,
+    float eta, int qr_every, long long seen, int chunk) {
+  extern __shared__ __align__(16) float bsm[];
+  const int ldp = r + 1;
+  float* X = bsm;                                   // [64][132] fp32, becomes Z
+  float* Y = X + kBlkRows * kBlkLdX;                // [64][r + 1]
+  float* Ps = Y + kBlkRows * ldp;                   // [128][r + 1]
+  float* col = Ps + kHeadDim * ldp;                 // [128] QR scratch
+  float* h = col + kHeadDim;                        // [128]
+  T* stg = reinterpret_cast<T*>(h + kHeadDim);      // [2][64][128] raw rows
+  __shared__ float red[4];
+  const int tid = threadIdx.x;
+  constexpr int CE = Elem<T>::CE;
+  float* Pg = P + (size_t)blockIdx.x * bstride;
+  const T* xg = x + (size_t)blockIdx.x * xstride;
+  for (int e = tid; e < kHeadDim * r; e += kOjaThreads) Ps[(e / r) * ldp + e % r] = Pg[e];
+
+  // length of the chunk starting at token j
+  auto chunk_len = [&](int j) {
+    int nc = min(min(chunk, kBlkRows), n - j);
+    if (qr_every > 0) {
+      const long long to_qr = qr_every - (seen + j) % qr_every;
+      if (to_qr < nc) nc = (int)to_qr;
+    }
+    return nc;
+  };
+  auto stage = [&](int j, int buf) {
+    const int nc = chunk_len(j);
+    T* dst = stg + (size_t)buf * kBlkRows * kHeadDim;
+    for (int e = tid; e < nc * (kHeadDim / CE); e += kOjaThreads) {
+      const int t = e / (kHeadDim / CE), c = e - t * (kHeadDim / CE);
+      cp_async16(dst + t * kHeadDim + c * CE, xg + (size_t)(j + t) * kHeadDim + c * CE, 16u);
+    }
+    cp_async_commit();
+  };
+  if (n > 0) stage(0, 0);
+  int buf = 0;
+  for (int j = 0; j < n;) {
+    const int nc = chunk_len(j);
+    cp_async_wait<0>();
+    __syncthreads();  // rows of this chunk landed; P and the buffers are free
+    {
+      const T* src = stg + (size_t)buf * kBlkRows * kHeadDim;
+      for (int e = tid; e < kBlkRows * kHeadDim; e += kOjaThreads) {
+        const int t = e >> 7, i = e & 127;
+        X[t * kBlkLdX + i] = t < nc ? to_f<T>(src[e]) : 0.f;
+      }
+    }
+    if (j + nc < n) stage(j + nc, buf ^ 1);
+    __syncthreads();
+    // Y = X P: thread -> tokens 4 tb .. 4 tb + 3, columns jb * (r / 8) ..
+    {
+      const int tb = tid >> 3, jb = tid & 7, rj = r >> 3, j0 = jb * rj;
+      float acc[4][8];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < kHeadDim; ++k) {
+        float xv[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) xv[a] = X[(4 * tb + a) * kBlkLdX + k];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c < rj) {
+            const float pv = Ps[k * ldp + j0 + c];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) acc[a][c] = fmaf(xv[a], pv, acc[a][c]);
+          }
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (c < rj) Y[(4 * tb + a) * ldp + j0 + c] = acc[a][c];
+    }
+    __syncthreads();
+    // Z = X - Y P^T, in place: thread -> tokens 8 tb .. + 7, rows ib + 16 m
+    {
+      const int tb = tid >> 4, ib = tid & 15;
+      float acc[8][8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int m = 0; m < 8; ++m) acc[a][m] = X[(8 * tb + a) * kBlkLdX + ib + 16 * m];
+      for (int k = 0; k < r; ++k) {
+        float yv[8], pv[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) yv[a] = Y[(8 * tb + a) * ldp + k];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) pv[m] = Ps[(ib + 16 * m) * ldp + k];
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+          for (int m = 0; m < 8; ++m) acc[a][m] = fmaf(-yv[a], pv[m], acc[a][m]);
+      }
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int m = 0; m < 8; ++m) X[(8 * tb + a) * kBlkLdX + ib + 16 * m] = acc[a][m];
+    }
+    __syncthreads();
+    // P += eta Z^T Y: thread -> rows ib + 32 m, columns jb * (r / 4) ..
+    {
+      const int ib = tid & 31, jb = tid >> 5, rj = r >> 2, j0 = jb * rj;
+      float acc[4][16];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) acc[m][c] = 0.f;
+      for (int t = 0; t < nc; ++t) {
+        float zv[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) zv[m] = X[t * kBlkLdX + ib + 32 * m];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          if (c < rj) {
+            const float yv = Y[t * ldp + j0 + c];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) acc[m][c] = fmaf(zv[m], yv, acc[m][c]);
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if (c < rj) {
+            float& pp = Ps[(ib + 32 * m) * ldp + j0 + c];
+            pp = fmaf(eta, acc[m][c], pp);
+          }
+    }
+    j += nc;
+    buf ^= 1;
+    __syncthreads();
+    if (qr_every > 0 && (seen + j) % qr_every == 0) qr_shared(Ps, r, ldp, col, h, red);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int e = tid; e < kHeadDim * r; e += kOjaThreads) Pg[e] = Ps[(e / r) * ldp + e % r];
+}
+
+int oja_blocked_launch(float* P, int S, int r, long long basis_stride, const void* x,
+                       int x_dtype, long long x_stride, int n, float eta, int qr_every,
+                       long long tokens_seen, int chunk, cudaStream_t st) {
+  const int es = x_dtype == LRKV_BF16 ? 2 : 4;
+  // rows are copied in 16-byte pieces
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0 || (x_stride * es) % 16 != 0)
+    return LRKV_ERR_ARG;
+  if (r > 64 || r % 8 != 0) return LRKV_ERR_UNSUPPORTED;
+  const size_t sm = oja_blocked_smem_bytes(r, es);
+  const void* fn = x_dtype == LRKV_BF16 ? (const void*)oja_blocked_kernel<__nv_bfloat16>
+                                        : (const void*)oja_blocked_kernel<float>;
+  const int rc = prepare_kernel(fn, false);
+  if (rc != LRKV_OK) return rc;
+  if (x_dtype == LRKV_BF16)
+    oja_blocked_kernel<__nv_bfloat16><<<S, kOjaThreads, sm, st>>>(
+        P, r, basis_stride, static_cast<const __nv_bfloat16*>(x), x_stride, n, eta, qr_every,
+        tokens_seen, chunk);
+  else
+    oja_blocked_kernel<float><<<S, kOjaThreads, sm, st>>>(P, r, basis_stride,
+                                                          static_cast<const float*>(x), x_stride,
+                                                          n, eta, qr_every, tokens_seen, chunk);
+  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+}
+
 template <typename T>
 static int oja2_launch_t(float* P, int S, int r, long long bs, const T* x, long long xs, int n,
                          float eta, int qr_every, long long seen, cudaStream_t st) {
   const size_t sm = oja2_smem_bytes(r, (int)sizeof(T));
   auto go = [&](auto kern) -> int {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-        cudaSuccess)
-      return LRKV_ERR_CUDA;
+    const int rc = prepare_kernel((const void*)kern, false);
+    if (rc != LRKV_OK) return rc;
     kern<<<S, kOja2Threads, sm, st>>>(P, r, bs, x, xs, n, eta, qr_every, seen);
     return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
   };
@@ -358,14 +546,14 @@ int oja_launch(float* P, int S, int r, long long basis_stride, const void* x, in
   const size_t sm = oja_smem(r);
   if (x_dtype == LRKV_BF16) {
     auto k = oja_kernel<__nv_bfloat16>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
-      return LRKV_ERR_CUDA;
+    const int rc = prepare_kernel((const void*)k, false);
+    if (rc != LRKV_OK) return rc;
     k<<<S, kOjaThreads, sm, st>>>(P, r, basis_stride, static_cast<const __nv_bfloat16*>(x),
                                    x_stride, n, eta, qr_every, tokens_seen);
   } else {
     auto k = oja_kernel<float>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
-      return LRKV_ERR_CUDA;
+    const int rc = prepare_kernel((const void*)k, false);
+    if (rc != LRKV_OK) return rc;
     k<<<S, kOjaThreads, sm, st>>>(P, r, basis_stride, static_cast<const float*>(x), x_stride, n,
                                    eta, qr_every, tokens_seen);
   }
@@ -374,9 +562,8 @@ int oja_launch(float* P, int S, int r, long long basis_stride, const void* x, in
 
 int qr_launch(float* P, int S, int r, long long basis_stride, cudaStream_t st) {
   const size_t sm = oja_smem(r);
-  if (cudaFuncSetAttribute(qr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-      cudaSuccess)
-    return LRKV_ERR_CUDA;
+  const int rc = prepare_kernel((const void*)qr_kernel, false);
+  if (rc != LRKV_OK) return rc;
   qr_kernel<<<S, kOjaThreads, sm, st>>>(P, r, basis_stride);
   return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
 }

@@ -19,6 +19,8 @@
 //     The work is small next to a decode step's stream (every latent byte
 //     is read and written once, plus r multiply-adds per code element), so
 //     it runs on the CUDA cores.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -157,19 +159,335 @@ __global__ void __launch_bounds__(kRebaseThreads, 1) rebase_codes_kernel(RebaseA
   }
 }
 
+// ---- bf16 codes on the tensor cores
+// rebase_codes_mma: persistent, several CTAs per SM.  The latent pages of
+// every (sequence, KV head) unit are laid end to end and each CTA takes an
+// equal contiguous range.  A producer warp streams one slab per page into a
+// ring of shared-memory stages with bulk copies (block-table entries
+// resolved a batch of 32 pages ahead).  Four consumer warps share each
+// page: warp w owns the 16 tokens of m-block w and every code column, and
+// computes c'[t][n] = sum_k c[t][k] R[n][k] with warp-level bf16 MMAs
+// (m16n8k16, fp32 accumulation), R split into hi + lo bf16 halves so the
+// products keep about 16 mantissa bits.  A fragments come by ldmatrix
+// straight from the chunk-major slab; a warp reads and rewrites only its own
+// rows, so it writes its new codes in place and copies its latent rows back
+// with 16-byte stores without waiting for the other warps; the stage is
+// released when all four have arrived.  R sits in padded rows [n][k] in
+// shared memory, rebuilt by the four warps together (a named barrier on
+// each side) when the range enters a new unit.
+constexpr int kRbConsumers = 4;
+constexpr int kRbThreads = 32 * (kRbConsumers + 1);
+constexpr int kRbMaxStages = 4;
+
+__host__ __device__ inline int rb_r16(int r) { return (r + 15) / 16 * 16; }
+__host__ __device__ inline int rb_row(int r) { return rb_r16(r) + 8; }  // padded R row (bf16)
+
+struct RbPlan {
+  int ring, rk_hi, rk_lo, rv_hi, rv_lo, full, empty, meta, start, flag, total;
+};
+__host__ __device__ inline RbPlan rb_plan(int NS, int rk, int rv, int B) {
+  RbPlan p;
+  int off = 0;
+  auto take = [&](int bytes, int align) {
+    off = (off + align - 1) / align * align;
+    const int at = off;
+    off += bytes;
+    return at;
+  };
+  const int slab = kLatPage * (rk + rv) * 2;
+  p.ring = take(NS * slab, 128);
+  p.rk_hi = take(rb_r16(rk) * rb_row(rk) * 2, 16);
+  p.rk_lo = take(rb_r16(rk) * rb_row(rk) * 2, 16);
+  p.rv_hi = take(rb_r16(rv) * rb_row(rv) * 2, 16);
+  p.rv_lo = take(rb_r16(rv) * rb_row(rv) * 2, 16);
+  p.full = take(NS * 8, 8);
+  p.empty = take(NS * 8, 8);
+  p.meta = take(NS * 2 * 4, 4);      // per stage: page (-1 bad), latent rows
+  p.start = take((B + 1) * 4, 4);
+  p.flag = take(8, 4);               // producer's and consumers' failure flags
+  p.total = off;
+  return p;
+}
+
+// Pages of sequence b's latent tokens (capped by the block-table row).
+__device__ inline int rb_pages(const RebaseArgs& a, int b) {
+  const int L = max(0, __ldcg(a.seq_len + b));
+  const int n_lat = split_tokens(L, a.n_sink, a.W).lat;
+  return min((n_lat + kLatPage - 1) / kLatPage, a.maxp);
+}
+
+// Bounded wait by lane 0 that also gives up once fail is set, its result
+// given to the warp.
+__device__ inline bool rb_wait_warp(uint64_t* bar, uint32_t parity, volatile int* fail,
+                                    int lane) {
+  int ok = 1;
+  if (lane == 0) {
+    ok = 0;
+    if (!*fail) {
+      if (mbar_try_wait(bar, parity)) {
+        ok = 1;
+      } else {
+        const uint64_t t0 = global_ns();
+        while (!*fail) {
+          if (mbar_try_wait(bar, parity)) { ok = 1; break; }
+          if (global_ns() - t0 > 2000000000ull) { *fail = 1; break; }
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__global__ void __launch_bounds__(kRbThreads) rebase_codes_mma(RebaseArgs a, int NS) {
+  using bf16 = __nv_bfloat16;
+  extern __shared__ __align__(128) uint8_t rsm[];
+  const RbPlan pl = rb_plan(NS, a.rk, a.rv, a.B);
+  uint64_t* full = reinterpret_cast<uint64_t*>(rsm + pl.full);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(rsm + pl.empty);
+  int* meta = reinterpret_cast<int*>(rsm + pl.meta);
+  int* start = reinterpret_cast<int*>(rsm + pl.start);
+  volatile int* fail = reinterpret_cast<volatile int*>(rsm + pl.flag);
+  volatile int* cfail = fail + 1;  // set only by consumer waits
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NJ = a.rk + a.rv, slab_bytes = kLatPage * NJ * 2;
+
+  // page prefix over sequences, one warp
+  if (warp == 0) {
+    const int per = (a.B + 31) / 32;
+    const int b0 = min(a.B, lane * per), b1 = min(a.B, b0 + per);
+    int own = 0;
+    for (int b = b0; b < b1; ++b) own += rb_pages(a, b) * a.H_kv;
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int e = incl - own;
+    for (int b = b0; b < b1; ++b) {
+      start[b] = e;
+      e += rb_pages(a, b) * a.H_kv;
+    }
+    if (lane == 31) start[a.B] = incl;
+  }
+  if (tid == 32) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kRbConsumers);
+    }
+    *fail = 0;
+    *cfail = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  const int total = start[a.B];
+  const int q = total / (int)gridDim.x, rem = total - q * (int)gridDim.x;
+  const int lo = blockIdx.x * q + (blockIdx.x * rem) / gridDim.x;
+  const int hi = (blockIdx.x + 1) * q + ((blockIdx.x + 1) * rem) / gridDim.x;
+  const int N = hi - lo;
+  if (N <= 0) return;
+  auto locate = [&](int k, int& b, int& kvh, int& p) {
+    int l = 0, h = a.B;
+    while (h - l > 1) {
+      const int mid = (l + h) >> 1;
+      if (start[mid] <= k) l = mid; else h = mid;
+    }
+    b = l;
+    const int pages = (start[b + 1] - start[b]) / a.H_kv;
+    const int r = k - start[b];
+    kvh = r / pages;
+    p = r - kvh * pages;
+  };
+
+  if (warp == 0) {
+    // ---------------- producer: lane l resolves page base + l of each batch
+    int issued = 0;
+    for (int base = 0; base < N; base += 32) {
+      int page = -1, rows = 0, kvh = 0;
+      if (base + lane < N) {
+        int b, p;
+        locate(lo + base + lane, b, kvh, p);
+        const int L = max(0, __ldcg(a.seq_len + b));
+        rows = min(kLatPage, split_tokens(L, a.n_sink, a.W).lat - p * kLatPage);
+        page = __ldg(a.bt + (size_t)b * a.maxp + p);
+        if (page < 0 || page >= a.num_pages) page = -1;
+      }
+      const int cnt = min(32, N - base);
+      bool ok = true;
+      for (int jj = 0; jj < cnt; ++jj) {
+        int f = 0;
+        if (lane == jj) {
+          const int k = base + jj, s = k % NS, n = k / NS;
+          if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) {
+            f = 1;
+          } else {
+            meta[2 * s] = page;
+            meta[2 * s + 1] = rows;
+            if (page >= 0) {
+              mbar_arrive_expect_tx(&full[s], slab_bytes);
+              bulk_g2s(rsm + pl.ring + (size_t)s * slab_bytes,
+                       static_cast<const bf16*>(a.codes) +
+                           ((size_t)page * a.H_kv + kvh) * kLatPage * NJ,
+                       slab_bytes, &full[s]);
+            } else {
+              *a.err = kErrBadPage;
+              mbar_arrive(&full[s]);
+            }
+            issued = k + 1;
+          }
+        }
+        if (__any_sync(0xffffffffu, f) || *fail || *cfail) {
+          *fail = 1;
+          ok = false;
+          break;
+        }
+      }
+      issued = __reduce_max_sync(0xffffffffu, issued);
+      if (!ok) break;
+    }
+    // every copy issued has landed before the CTA may exit
+    if (lane == 0)
+      for (int s = 0; s < NS && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / NS) * NS;
+        mbar_wait_bounded(&full[s], (last / NS) & 1);
+      }
+    return;
+  }
+
+  // ---------------- consumers: warp cw owns rows 16 cw .. 16 cw + 15
+  const int cw = warp - 1, ctid = tid - 32;
+  const int g = lane >> 2, t = lane & 3;
+  auto Rh = [&](int sd) { return reinterpret_cast<bf16*>(rsm + (sd ? pl.rv_hi : pl.rk_hi)); };
+  auto Rl = [&](int sd) { return reinterpret_cast<bf16*>(rsm + (sd ? pl.rv_lo : pl.rk_lo)); };
+  auto side_on = [&](int sd) { return (sd ? a.Pv_old : a.Pk_old) != nullptr; };
+  int cur_unit = -1;
+  for (int k = 0; k < N; ++k) {
+    const int s = k % NS;
+    int b, kvh, p;
+    locate(lo + k, b, kvh, p);
+    const int unit = b * a.H_kv + kvh;
+    if (unit != cur_unit) {
+      // R of the new unit as padded [n][k] rows, hi + lo, zero past the rank.
+      // Every consumer takes this branch at the same page (the page order is
+      // fixed), so the barriers always meet, even after a failed wait.
+      named_bar(1, 32 * kRbConsumers);  // no warp still reads the old R
+#pragma unroll 1
+      for (int sd = 0; sd < 2; ++sd) {
+        if (!side_on(sd)) continue;
+        const int r = sd ? a.rv : a.rk, R16 = rb_r16(r), RS = rb_row(r);
+        const float* Rt = (sd ? a.Rv : a.Rk) + (size_t)unit * r * r;  // Rt[k][n] = R[n][k]
+        bf16* rh = Rh(sd);
+        bf16* rl = Rl(sd);
+        for (int x = ctid; x < R16 * R16; x += 32 * kRbConsumers) {
+          const int kk = x / R16, n = x - kk * R16;
+          const float v = (kk < r && n < r) ? __ldcg(Rt + (size_t)kk * r + n) : 0.f;
+          const bf16 h = __float2bfloat16_rn(v);
+          rh[n * RS + kk] = h;
+          rl[n * RS + kk] = __float2bfloat16_rn(v - __bfloat162float(h));
+        }
+      }
+      cur_unit = unit;
+      named_bar(1, 32 * kRbConsumers);
+    }
+    if (!rb_wait_warp(&full[s], (k / NS) & 1, cfail, lane)) continue;  // skip work, keep pace
+    const int page = meta[2 * s], rows = meta[2 * s + 1];
+    uint8_t* st = rsm + pl.ring + (size_t)s * slab_bytes;
+    if (page >= 0) {
+      const uint32_t sbase = smem_u32(st);
+      bf16* sb = reinterpret_cast<bf16*>(st);
+#pragma unroll 1
+      for (int sd = 0; sd < 2; ++sd) {
+        if (!side_on(sd)) continue;
+        const int r = sd ? a.rv : a.rk, nch = r / 8, cb = sd ? a.rk / 8 : 0;
+        const int NP = rb_r16(r) / 16;            // n-block pairs = k-steps of 16
+        const uint32_t rh = smem_u32(Rh(sd)), rl = smem_u32(Rl(sd));
+        const int RS = rb_row(r);
+        float acc[16][4];
+#pragma unroll
+        for (int nb = 0; nb < 16; ++nb)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[nb][i] = 0.f;
+        for (int ks = 0; ks < NP; ++ks) {
+          const int c = min(2 * ks + (lane >> 4), nch - 1);
+          uint32_t af[4];
+          ldsm_x4(sbase + (uint32_t)(((cb + c) * kLatPage + cw * 16 + (lane & 15)) * 16), af);
+#pragma unroll
+          for (int pr = 0; pr < 8; ++pr) {
+            if (pr < NP) {
+              const int o = 16 * pr + (lane & 7) + ((lane >> 4) << 3);
+              const int koff = 16 * ks + ((lane >> 3) & 1) * 8;
+              uint32_t bh[4], bl[4];
+              ldsm_x4(rh + (uint32_t)((o * RS + koff) * 2), bh);
+              ldsm_x4(rl + (uint32_t)((o * RS + koff) * 2), bl);
+              mma_bf16_16816(acc[2 * pr], af, bh[0], bh[1]);
+              mma_bf16_16816(acc[2 * pr + 1], af, bh[2], bh[3]);
+              mma_bf16_16816(acc[2 * pr], af, bl[0], bl[1]);
+              mma_bf16_16816(acc[2 * pr + 1], af, bl[2], bl[3]);
+            }
+          }
+        }
+        __syncwarp();  // every lane's reads of this side's old codes are done
+#pragma unroll
+        for (int nb = 0; nb < 16; ++nb) {
+          if (nb < nch) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int row = cw * 16 + g + 8 * h2;
+              *reinterpret_cast<uint32_t*>(sb + ((size_t)(cb + nb) * kLatPage + row) * 8 + 2 * t) =
+                  pack_bf16x2(acc[nb][2 * h2], acc[nb][2 * h2 + 1]);
+            }
+          }
+        }
+      }
+      __syncwarp();  // the warp's new codes are in place
+      // this warp's latent rows of the re-based sides go back, 16 bytes at a time
+      const uint4* src = reinterpret_cast<const uint4*>(st);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(a.codes) +
+                                            ((size_t)page * a.H_kv + kvh) * kLatPage * NJ);
+      const int c0 = side_on(0) ? 0 : a.rk / 8, c1 = side_on(1) ? NJ / 8 : a.rk / 8;
+      for (int x = lane; x < (c1 - c0) * 16; x += 32) {
+        const int c = c0 + x / 16, row = cw * 16 + (x & 15);
+        if (row < rows) dst[c * kLatPage + row] = src[c * kLatPage + row];
+      }
+    }
+    __syncwarp();  // the warp is done with the stage
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
 template <typename T>
 int launch_rebase_t(const RebaseArgs& a, cudaStream_t st) {
   const int rmax = a.rk > a.rv ? a.rk : a.rv;
   const size_t ms = matrix_smem_bytes(rmax);
-  if (cudaFuncSetAttribute(rebase_matrix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)ms) != cudaSuccess)
-    return LRKV_ERR_CUDA;
+  int rc = prepare_kernel((const void*)rebase_matrix_kernel, false);
+  if (rc == LRKV_OK) rc = prepare_kernel((const void*)rebase_codes_kernel<T>, false);
+  if (rc != LRKV_OK) return rc;
   rebase_matrix_kernel<<<dim3(a.H_kv, a.B, 2), kRebaseThreads, ms, st>>>(a);
   if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // tensor-core pass: as many ring stages as fit beside R and the prefix
+    int dev = 0;
+    DevInfo info;
+    rc = current_device_info(dev, info);
+    if (rc != LRKV_OK) return rc;
+    int NS = kRbMaxStages;
+    while (NS >= 2 && rb_plan(NS, a.rk, a.rv, a.B).total > info.optin) --NS;
+    if (NS >= 2) {
+      rc = prepare_kernel((const void*)rebase_codes_mma, false);
+      if (rc != LRKV_OK) return rc;
+      const int smem = rb_plan(NS, a.rk, a.rv, a.B).total;
+      int per_sm = 1;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rebase_codes_mma, kRbThreads,
+                                                        smem) != cudaSuccess ||
+          per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+      }
+      rebase_codes_mma<<<info.sms * per_sm, kRbThreads, smem, st>>>(a, NS);
+      return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+    }
+  }
   const size_t cs = codes_smem_bytes<T>(a.rk, a.rv);
-  if (cudaFuncSetAttribute(rebase_codes_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)cs) != cudaSuccess)
-    return LRKV_ERR_CUDA;
   rebase_codes_kernel<T><<<dim3(a.maxp, a.H_kv, a.B), kRebaseThreads, cs, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
 }

@@ -11,7 +11,10 @@
 // it names a host-side stand-in).  The first call on a device, with that
 // device current, looks up the array's device address once with
 // cudaGetSymbolAddress and keeps it; that first call should therefore come
-// before any stream capture.  Every later call on the device reuses it.
+// before any stream capture.  Every later call on the device reuses it, so
+// the stream passed must belong to the current device, and a device reset
+// (cudaDeviceReset) while the library is loaded is not supported: the kept
+// address would be stale.
 #include <mutex>
 
 #include "common.cuh"
@@ -48,9 +51,9 @@ extern "C" int lrkv_decode_attn_static(const lrkv_cache* cache, const void* q,
                                        void* stream) {
   const size_t need = lrkv_decode_workspace_bytes(cache, num_q_heads);
   if (need == 0) {
-    // invalid arguments: let the regular entry point report which
-    return lrkv_decode_attn(cache, q, num_q_heads, P_k, P_v, basis_batch_stride, scale, o,
-                            nullptr, 0, stream);
+    // the cache, the head counts or the plan were rejected: report why
+    const int rc = lrkv::decode_plan_status(cache, num_q_heads);
+    return rc != LRKV_OK ? rc : LRKV_ERR_ARG;
   }
   if (need > (size_t)LRKV_STATIC_WORKSPACE_BYTES) return LRKV_ERR_WORKSPACE;
   void* ws = nullptr;

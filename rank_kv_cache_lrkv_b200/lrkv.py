@@ -17,7 +17,7 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblrkv.so")
 
-LRKV_BF16, LRKV_F32 = 0, 1
+LRKV_BF16, LRKV_F32, LRKV_BF16_Q8 = 0, 1, 2
 HEAD_DIM = 128
 PAGE_TOKENS = 64
 FULL_RANK_TILE = 32
@@ -56,7 +56,7 @@ EXPORTS = ["lrkv_compress", "lrkv_decode_workspace_bytes", "lrkv_decode_attn",
            "lrkv_oja_update", "lrkv_qr_orthonormalize", "lrkv_dense_append",
            "lrkv_dense_decode_workspace_bytes", "lrkv_dense_decode_attn",
            "lrkv_status_string", "lrkv_version", "lrkv_decode_attn_static",
-           "lrkv_rebase_workspace_bytes", "lrkv_rebase"]
+           "lrkv_rebase_workspace_bytes", "lrkv_rebase", "lrkv_oja_update_chunked"]
 
 
 def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
@@ -72,6 +72,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "lrkv_decode_attn": (ctypes.c_int, [P, P, I32, P, P, I64, F32, P, P, SZ, P]),
         "lrkv_oja_update": (ctypes.c_int, [P, I32, I32, I64, P, I32, I64, I32, F32, I32, I64, P]),
         "lrkv_qr_orthonormalize": (ctypes.c_int, [P, I32, I32, I64, P]),
+        "lrkv_oja_update_chunked": (ctypes.c_int,
+                                    [P, I32, I32, I64, P, I32, I64, I32, F32, I32, I64, I32, P]),
         "lrkv_dense_append": (ctypes.c_int, [P, P, P, I32, P, I64, I64, P]),
         "lrkv_dense_decode_workspace_bytes": (SZ, [P, I32]),
         "lrkv_dense_decode_attn": (ctypes.c_int, [P, P, I32, F32, P, P, SZ, P]),
@@ -126,16 +128,25 @@ class LatentCache:
 
     def __init__(self, B: int, H_kv: int, r_k: int, r_v: int, max_tokens: int,
                  n_sink: int = 0, window: int = 0, dtype=torch.bfloat16,
-                 device="cuda", page_perm: Optional[torch.Tensor] = None):
+                 device="cuda", page_perm: Optional[torch.Tensor] = None,
+                 int8_codes: bool = False):
         ce = chunk_elems(dtype)
         self.B, self.H_kv, self.r_k, self.r_v = B, H_kv, r_k, r_v
         self.n_sink, self.window, self.dtype = n_sink, window, dtype
+        self.int8_codes = int8_codes
         max_lat = max(1, max_tokens - n_sink - window)
         self.max_pages = math.ceil(max_lat / PAGE_TOKENS)
         self.num_pages = B * self.max_pages
-        # one slab per (page, kv head): key-code chunks, then value-code chunks
-        self.codes = torch.zeros((self.num_pages, H_kv, (r_k + r_v) // ce, PAGE_TOKENS, ce),
-                                 dtype=dtype, device=device)
+        if int8_codes:
+            # one slab per (page, kv head): int8 code chunks of 16, key codes
+            # then value codes, then [64][2] fp32 scales (bf16 inputs)
+            assert dtype == torch.bfloat16
+            self.codes = torch.zeros((self.num_pages, H_kv, PAGE_TOKENS * (r_k + r_v) + 512),
+                                     dtype=torch.uint8, device=device)
+        else:
+            # one slab per (page, kv head): key-code chunks, then value-code chunks
+            self.codes = torch.zeros((self.num_pages, H_kv, (r_k + r_v) // ce, PAGE_TOKENS, ce),
+                                     dtype=dtype, device=device)
         ids = torch.arange(self.num_pages, dtype=torch.int32) if page_perm is None else \
             torch.as_tensor(page_perm, dtype=torch.int32)
         self.block_table = ids.reshape(B, self.max_pages).to(device)
@@ -145,7 +156,8 @@ class LatentCache:
                                    dtype=dtype, device=device)
         self.seq_len = torch.zeros(B, dtype=torch.int32, device=device)
         self.append_counter = torch.zeros(B, dtype=torch.int32, device=device)
-        self.desc = CacheDesc(B, H_kv, HEAD_DIM, r_k, r_v, _dtype_code(dtype), n_sink, window,
+        code = LRKV_BF16_Q8 if int8_codes else _dtype_code(dtype)
+        self.desc = CacheDesc(B, H_kv, HEAD_DIM, r_k, r_v, code, n_sink, window,
                               self.num_pages, self.max_pages, self.codes.data_ptr(),
                               self.block_table.data_ptr(), self.anchors.data_ptr(),
                               self.seq_len.data_ptr(), self.append_counter.data_ptr())
@@ -240,6 +252,19 @@ def oja_update(P: torch.Tensor, x: torch.Tensor, eta: float, qr_every: int, toke
     _check("lrkv_oja_update", _lib.lrkv_oja_update(
         _ptr(P), P.shape[0], P.shape[2], P.stride(0), _ptr(x), _dtype_code(x.dtype), x.stride(0),
         x.shape[1], float(eta), int(qr_every), int(tokens_seen), _stream(stream)))
+
+
+def oja_update_chunked(P: torch.Tensor, x: torch.Tensor, eta: float, qr_every: int,
+                       tokens_seen: int, chunk: int = 64, stream=None) -> None:
+    """lrkv_oja_update_chunked: the Oja update with P frozen within chunks of
+    `chunk` tokens; P [S, 128, r] fp32 in place, x [S, n, 128] rows."""
+    assert P.dtype == torch.float32 and P.dim() == 3 and P.shape[1] == HEAD_DIM
+    assert P.stride(2) == 1 and P.stride(1) == P.shape[2]
+    assert x.dim() == 3 and x.shape[2] == HEAD_DIM and x.stride(2) == 1 and \
+        (x.shape[1] <= 1 or x.stride(1) == HEAD_DIM)
+    _check("lrkv_oja_update_chunked", _lib.lrkv_oja_update_chunked(
+        _ptr(P), P.shape[0], P.shape[2], P.stride(0), _ptr(x), _dtype_code(x.dtype), x.stride(0),
+        x.shape[1], float(eta), int(qr_every), int(tokens_seen), int(chunk), _stream(stream)))
 
 
 def qr_orthonormalize(P: torch.Tensor, stream=None) -> None:

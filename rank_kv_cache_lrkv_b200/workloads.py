@@ -126,6 +126,18 @@ QWEN3_STACK_OJA = Workload(
     basis="random", layers=28, oja_eta=1e-3, oja_qr_every=256,
     oja_decode_every=512, prefill_oja=True)
 
+# Small variant of the Oja workload whose decode-time update fires: the basis
+# of every (sequence, KV head) is adapted over the prompt, then every 32
+# generated tokens over those 32 tokens, with a QR every 64 tokens seen.
+# Sink + window anchors make evictions cross basis updates.  The rate is
+# larger than the stack's 1e-3 so that a 32-token update moves the basis
+# visibly (eta * |x|^2 stays below 0.2, well inside Oja's stable range).
+QWEN3_DECODE_OJA_SMALL = Workload(
+    name="qwen3_1.7b_layer_T512_decode_oja32", wid=5, B=2, H_q=8, H_kv=2,
+    T=512, r_k=32, r_v=32, dtype="bf16", rope_theta=1e6, n_sink=1, window=32,
+    n_decode=96, basis="random", oja_eta=2e-2, oja_qr_every=64,
+    oja_decode_every=32, prefill_oja=True)
+
 ALL = {w.name: w for w in [TINY_SINGLE_HEAD, QWEN3_LAYER_8K,
                            LLAMA31_LAYER_32K_ANCHORS, QWEN3_STACK_OJA]}
 

@@ -51,6 +51,29 @@ def gather_codes(cache, b, kvh, n, kind="k"):
     return x.reshape(n, r).double().cpu().numpy()
 
 
+def gather_q8(cache, b, kvh, n, kind="k"):
+    """int8 codes [n, r] and fp32 scales [n] of latent tokens 0..n-1 of
+    (b, kvh) in an int8-code cache (16 codes per chunk, key chunks first,
+    then the value chunks, then [64][2] scales per page)."""
+    r = cache.r_k if kind == "k" else cache.r_v
+    c0 = 0 if kind == "k" else cache.r_k // 16
+    side = 0 if kind == "k" else 1
+    nj = cache.r_k + cache.r_v
+    slabs = cache.codes.cpu()
+    bt = cache.block_table[b].long().cpu()
+    q = np.zeros((n, r), np.int8)
+    s = np.zeros(n, np.float32)
+    for j in range(n):
+        slab = slabs[bt[j // 64], kvh]
+        row = j % 64
+        for c in range(r // 16):
+            off = ((c0 + c) * 64 + row) * 16
+            q[j, 16 * c:16 * c + 16] = slab[off:off + 16].numpy().view(np.int8)
+        so = 64 * nj + (row * 2 + side) * 4
+        s[j] = slab[so:so + 4].numpy().view(np.float32)[0]
+    return q, s
+
+
 def gather_anchor_slots(cache, b, kvh, slots, kind="k"):
     ce = cache.anchors.shape[-1]
     h = 128 // ce
@@ -79,12 +102,13 @@ class Inputs:
         self.q = wk.layer_queries(wl, layer)
 
 
-def run_gpu(wl, inp, n_steps=None, page_perm=None, lrkv=None, prefill_chunks=None):
+def run_gpu(wl, inp, n_steps=None, page_perm=None, lrkv=None, prefill_chunks=None,
+            int8_codes=False):
     """Prefill + decode steps through the C ABI; returns (cache, [o per step])."""
     n_steps = wl.n_decode if n_steps is None else n_steps
     dt = torch_dtype(wl)
     cache = lrkv.LatentCache(wl.B, wl.H_kv, wl.r_k, wl.r_v, wl.T + n_steps, wl.n_sink,
-                             wl.window, dtype=dt, page_perm=page_perm)
+                             wl.window, dtype=dt, page_perm=page_perm, int8_codes=int8_codes)
     K, V = inp.K.cuda(), inp.V.cuda()
     Pk, Pv = inp.Pk.cuda(), inp.Pv.cuda()
     chunks = prefill_chunks or [wl.T]
@@ -108,7 +132,7 @@ def run_gpu(wl, inp, n_steps=None, page_perm=None, lrkv=None, prefill_chunks=Non
     return cache, outs
 
 
-def run_oracle(wl, inp, n_steps=None, units=None):
+def run_oracle(wl, inp, n_steps=None, units=None, quant_bits=0):
     """The same schedule in the float64 oracle.  units: optional list of
     (b, kvh) pairs; then only those units are simulated (each as its own
     single-sequence, single-head cache) and outputs are returned per unit as
@@ -120,7 +144,8 @@ def run_oracle(wl, inp, n_steps=None, units=None):
         V = inp.V.double().numpy()
         Pk = inp.Pk.double().numpy()[None]
         Pv = inp.Pv.double().numpy()[None]
-        oc = orc.LatentCacheOracle(wl.B, wl.H_kv, wl.r_k, wl.r_v, wl.n_sink, wl.window)
+        oc = orc.LatentCacheOracle(wl.B, wl.H_kv, wl.r_k, wl.r_v, wl.n_sink, wl.window,
+                                   quant_bits=quant_bits)
         oc.append(K[:, :, :wl.T], V[:, :, :wl.T], Pk, Pv)
         outs = []
         for s in range(n_steps):
@@ -135,7 +160,8 @@ def run_oracle(wl, inp, n_steps=None, units=None):
         V = inp.V[b:b + 1, h:h + 1].double().numpy()
         Pk = inp.Pk[h:h + 1].double().numpy()[None]
         Pv = inp.Pv[h:h + 1].double().numpy()[None]
-        oc = orc.LatentCacheOracle(1, 1, wl.r_k, wl.r_v, wl.n_sink, wl.window)
+        oc = orc.LatentCacheOracle(1, 1, wl.r_k, wl.r_v, wl.n_sink, wl.window,
+                                   quant_bits=quant_bits)
         oc.append(K[:, :, :wl.T], V[:, :, :wl.T], Pk, Pv)
         outs = []
         for s in range(n_steps):
@@ -148,8 +174,9 @@ def run_oracle(wl, inp, n_steps=None, units=None):
     return res
 
 
-def check_state(wl, inp, cache, oc, L):
+def check_state(wl, inp, cache, oc, L, tol_code=None):
     """Codes and anchors on the GPU vs the oracle's cache (same schedule)."""
+    tol_code = TOL_CODE[wl.dtype] if tol_code is None else tol_code
     for b in range(wl.B):
         for h in range(wl.H_kv):
             n = oc.codes_k[b][h].shape[0]
@@ -159,7 +186,7 @@ def check_state(wl, inp, cache, oc, L):
                 got = gather_codes(cache, b, h, n, kind)
                 den = np.maximum(np.max(np.abs(ref), axis=1), 1e-30)
                 err = np.max(np.max(np.abs(got - ref), axis=1) / den)
-                assert err < TOL_CODE[wl.dtype], (b, h, kind, err)
+                assert err < tol_code, (b, h, kind, err)
             Ka, Va = oc.anchors(b, h)
             if Ka.shape[0]:
                 slots = window_slots(L, wl.n_sink, wl.window)

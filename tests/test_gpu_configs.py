@@ -12,6 +12,7 @@ import torch
 from oracle import lrkv_oracle as orc
 from rank_kv_cache_lrkv_b200 import workloads as wk
 from tests import lrkv_testutil as tu
+from tests.test_tolerances import TOL_P_STACK
 
 pytestmark = pytest.mark.gpu
 
@@ -23,9 +24,10 @@ def lrkv():
     return m
 
 
-def _sampled(lrkv, wl, units, page_perm=None):
-    inp = tu.Inputs(wl)
-    cache, outs = tu.run_gpu(wl, inp, lrkv=lrkv, page_perm=page_perm)
+def _sampled(lrkv, wl, units, page_perm=None, inp=None, inp_gpu=None):
+    inp = tu.Inputs(wl) if inp is None else inp
+    cache, outs = tu.run_gpu(wl, inp if inp_gpu is None else inp_gpu, lrkv=lrkv,
+                             page_perm=page_perm)
     res = tu.run_oracle(wl, inp, units=units)
     G = wl.G
     worst = 0.0
@@ -57,10 +59,42 @@ def test_llama31_layer_32k_anchors_sampled(lrkv):
     _sampled(lrkv, wl, [(0, 0), (1, 3), (3, 7)], page_perm=perm)
 
 
-@pytest.mark.parametrize("r_k,r_v,B", [(96, 64, 8), (32, 32, 32), (64, 32, 1)])
-def test_qwen3_rank_batch_sweep_points(lrkv, r_k, r_v, B):
+class _Slice:
+    """Inputs of a sweep point cut from the largest point's draws."""
+
+    def __init__(self, K, V, Pk, Pv, q):
+        self.K, self.V, self.Pk, self.Pv, self.q = K, V, Pk, Pv, q
+
+
+@pytest.fixture(scope="module")
+def sweep_inputs():
+    """The sweep's seeded draws at the largest batch and ranks.  A stream
+    depends only on its (sequence, KV head) seed and a basis of rank r is the
+    first r columns of the rank-96 (keys) or rank-64 (values) SVD basis, so
+    every point's inputs are slices of these."""
+    rk_max = max(r for r, _ in wk.SWEEP_RANKS)
+    rv_max = max(r for _, r in wk.SWEEP_RANKS)
+    wl = wk.qwen3_sweep_point(rk_max, rv_max, max(wk.SWEEP_BATCHES)).with_(n_decode=2)
+    cpu = tu.Inputs(wl)
+    gpu = _Slice(cpu.K.cuda(), cpu.V.cuda(), cpu.Pk, cpu.Pv, cpu.q)
+    return cpu, gpu
+
+
+@pytest.mark.parametrize("r_k,r_v", wk.SWEEP_RANKS)
+@pytest.mark.parametrize("B", wk.SWEEP_BATCHES)
+def test_qwen3_rank_batch_sweep_points(lrkv, sweep_inputs, r_k, r_v, B):
+    """Every point of the rank x batch sweep at T=16384: two decode steps;
+    the first and last (sequence, KV head) units and one in the middle are
+    replayed by the oracle."""
     wl = wk.qwen3_sweep_point(r_k, r_v, B).with_(n_decode=2)
-    _sampled(lrkv, wl, [(0, 0), (B - 1, 7)])
+    cpu, gpu = sweep_inputs
+    Pk = cpu.Pk[:, :, :r_k].contiguous()
+    Pv = cpu.Pv[:, :, :r_v].contiguous()
+    assert torch.equal(Pk[0], torch.from_numpy(wk.basis(wl, "k", 0, 0)))
+    inp = _Slice(cpu.K[:B], cpu.V[:B], Pk, Pv, cpu.q[:, :B])
+    inp_gpu = _Slice(gpu.K[:B], gpu.V[:B], Pk, Pv, cpu.q[:, :B])
+    units = sorted({(0, 0), (B // 2, 3), (B - 1, 7)})
+    _sampled(lrkv, wl, units, inp=inp, inp_gpu=inp_gpu)
 
 
 def test_qwen3_28_layer_stack_with_oja():
@@ -122,5 +156,9 @@ def test_qwen3_28_layer_stack_with_oja():
             worst_out = max(worst_out, tu.row_rel_err(
                 outs[s][b, h * G:(h + 1) * G].double().cpu().numpy(), ref))
         del K, V, cache, outs
-    assert worst_P <= 1e-3, worst_P
+    # fp32 against float64 over 32,768 tokens and 128 QRs: a float32
+    # restatement of the loop drifts a few 1e-6 (tests/test_tolerances.py);
+    # 1e-4 leaves more than an order of magnitude for the GPU's summation order
+    print(f"28-layer stack: worst basis deviation {worst_P:.3e}, worst output {worst_out:.3e}")
+    assert worst_P <= TOL_P_STACK, worst_P
     assert worst_out < tu.TOL["bf16"], worst_out

@@ -61,6 +61,8 @@ def test_llama_layer_anchors_small(lrkv):
     dict(T=300, H_q=64, H_kv=8),                 # G = 8
     dict(T=250, r_k=48, r_v=96),                 # uneven ranks
     dict(T=250, r_k=128, r_v=8),
+    dict(T=400, r_k=40, r_v=24),                 # ranks not multiples of 16
+    dict(B=37, T=150, window=16),                # more sequences than a warp's lanes
 ])
 def test_edge_cases(lrkv, case):
     kw = dict(B=2, n_decode=2, n_sink=0, window=0)

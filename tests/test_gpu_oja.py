@@ -81,3 +81,43 @@ def test_oja_strided_streams(lrkv):
     lrkv.oja_update(P, Xd[:, :n], 2e-3, 128, 0)
     ref = orc.oja_update_streams(P0.astype(np.float64), X[:, :n].float().numpy(), 2e-3, 128, 0)
     assert _rel(P.cpu().double().numpy(), ref) <= 1e-4
+
+
+def _blocked_ref(P0, X, eta, qr_every, seen, chunk):
+    return np.stack([orc.oja_update_blocked(P0[s].astype(np.float64), X[s].float().numpy(), eta,
+                                            qr_every, seen, chunk) for s in range(P0.shape[0])])
+
+
+@pytest.mark.parametrize("r,dtype,qr_every,seen,chunk", [
+    (48, "bf16", 256, 100, 64), (32, "f32", 64, 0, 16), (8, "bf16", 0, 0, 64),
+    (64, "bf16", 128, 5, 64), (56, "f32", 100, 3, 7), (48, "bf16", 256, 0, 1)])
+def test_chunked_oja_matches_oracle(lrkv, r, dtype, qr_every, seen, chunk):
+    """lrkv_oja_update_chunked against the oracle's chunked rule (fp32 bar);
+    chunk 7 and QR every 100 make chunks end early at QR points."""
+    S, n, eta = 5, 700, 1e-3
+    P0, X = _setup(S, r, n, dtype, seed=3)
+    P = torch.from_numpy(P0).cuda()
+    lrkv.oja_update_chunked(P, X.cuda(), eta, qr_every, seen, chunk)
+    ref = _blocked_ref(P0, X, eta, qr_every, seen, chunk)
+    assert _rel(P.cpu().double().numpy(), ref) <= 1e-4
+
+
+def test_chunked_oja_split_calls_equal_one_call(lrkv):
+    """Splitting the tokens at a chunk boundary changes nothing."""
+    S, r, n = 3, 48, 640
+    P0, X = _setup(S, r, n, "bf16", seed=4)
+    Xd = X.cuda()
+    one = torch.from_numpy(P0).cuda()
+    lrkv.oja_update_chunked(one, Xd, 1e-3, 256, 0, 64)
+    two = torch.from_numpy(P0).cuda()
+    lrkv.oja_update_chunked(two, Xd[:, :256].contiguous(), 1e-3, 256, 0, 64)
+    lrkv.oja_update_chunked(two, Xd[:, 256:].contiguous(), 1e-3, 256, 256, 64)
+    assert torch.equal(one, two)
+
+
+def test_chunked_oja_rejects_wide_ranks(lrkv):
+    P = torch.zeros(1, 128, 96, device="cuda")
+    x = torch.zeros(1, 64, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lrkv.LrkvError) as e:
+        lrkv.oja_update_chunked(P, x, 1e-3, 0, 0, 64)
+    assert e.value.status == -2

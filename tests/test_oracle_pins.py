@@ -497,3 +497,189 @@ def test_decode_from_parts_equals_cache_attend(G):
     o = orc.decode_from_parts(q, Pk, Pv, Ck, Cv, Ka, Va, G, 0.15)
     ref = c.attend(q, Pk, Pv, 0.15)
     assert np.max(np.abs(o - ref)) < 1e-13 * np.max(np.abs(ref))
+
+
+# ------------------------------------------------------------ quantised codes
+
+def test_quantize_codes_worked_example():
+    """By hand: the largest magnitude maps to 127 and sets the scale; the
+    rest round half to even."""
+    C = np.array([[0.5, -1.27, 0.01, 0.005],
+                  [0.0, 0.0, 0.0, 0.0],
+                  [2.0, 1.0, -0.5, 0.25]])
+    q, s = orc.quantize_codes(C, 8)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert np.isclose(s[0], 0.01, rtol=1e-6) and s[1] == 0 and np.isclose(s[2], 2.0 / 127, rtol=1e-6)
+    assert q[0].tolist() == [50, -127, 1, 0]          # 0.5 -> 0 (half to even)
+    assert q[1].tolist() == [0, 0, 0, 0]
+    assert q[2].tolist() == [127, 64, -32, 16]        # 63.5 -> 64, 15.875 -> 16
+
+
+def test_quantize_codes_round_trip_bound_and_extremes():
+    """Every row: |c - q s| <= s / 2 (plus fp32 rounding of c), the largest
+    entry is reproduced to fp32 precision, and |q| <= 127."""
+    rng = np.random.default_rng(400)
+    C = rng.standard_normal((200, 24)) * np.exp(-np.arange(24) / 8.0)[None, :]
+    C[7] *= 1e-30                       # tiny row: still its own scale
+    q, s = orc.quantize_codes(C, 8)
+    Ch = orc.dequantize_codes(q, s)
+    err = np.abs(Ch - C)
+    assert np.all(err <= s[:, None] / 2 * (1 + 1e-6) + np.abs(C) * 2 ** -23)
+    assert np.all(np.abs(q.astype(int)) <= 127)
+    j = np.argmax(np.abs(C), axis=1)
+    assert np.all(np.abs(q[np.arange(200), j].astype(int)) == 127)
+    assert np.allclose(Ch[np.arange(200), j], C[np.arange(200), j], rtol=1e-6, atol=0)
+
+
+def test_quantised_cache_attends_over_dequantised_codes():
+    """The quantised cache keeps each code row as its dequantised int8 form;
+    attention reads those rows, anchors stay exact."""
+    rng = np.random.default_rng(401)
+    P = rng.standard_normal((1, 1, D, 16)) * 0.2
+    k, v = rng.standard_normal((1, 1, 40, D)), rng.standard_normal((1, 1, 40, D))
+    cq = orc.LatentCacheOracle(1, 1, 16, 16, n_sink=1, window=4, quant_bits=8)
+    cq.append(k, v, P, P)
+    lat = list(range(1, 36))
+    ref_k = orc.dequantize_codes(*orc.quantize_codes(k[0, 0, lat] @ P[0, 0], 8))
+    assert np.array_equal(cq.codes_k[0][0], ref_k)
+    Ka, _ = cq.anchors(0, 0)
+    assert np.array_equal(Ka, k[0, 0, [0, 36, 37, 38, 39]])
+    q = rng.standard_normal((1, 1, D))
+    o = cq.attend(q, P, P, 0.1)
+    o_ref = orc.latent_attention(q[0, 0], P[0, 0], P[0, 0], ref_k, cq.codes_v[0][0], Ka,
+                                 cq.anchors(0, 0)[1], 0.1)
+    assert np.max(np.abs(o[0, 0] - o_ref)) < 1e-14 * np.max(np.abs(o_ref))
+    # close to the unquantised cache (8-bit codes: well inside the bf16 bar)
+    c = orc.LatentCacheOracle(1, 1, 16, 16, n_sink=1, window=4)
+    c.append(k, v, P, P)
+    o_full = c.attend(q, P, P, 0.1)
+    assert np.max(np.abs(o - o_full)) < 2e-2 * np.max(np.abs(o_full))
+
+
+# ------------------------------------------------------------ chunked Oja
+
+def test_blocked_oja_with_chunk_one_is_the_sequential_rule():
+    rng = np.random.default_rng(500)
+    P0 = _orth(rng, D, 12)
+    X = rng.standard_normal((300, D)) * np.exp(-np.arange(D) / 16.0)[None, :]
+    a = orc.oja_update_blocked(P0, X, 0.01, 64, tokens_seen=30, chunk=1)
+    b = orc.oja_update(P0, X, 0.01, 64, tokens_seen=30)
+    assert np.max(np.abs(a - b)) < 1e-13
+
+
+def test_blocked_oja_one_chunk_is_the_covariance_form():
+    """One chunk, written through the chunk's second moment C = X^T X:
+    P + eta (C P - P P^T C P) -- the frozen-basis sum of Oja's per-token
+    updates, spelled without Y or Z."""
+    rng = np.random.default_rng(501)
+    P0 = rng.standard_normal((D, 8)) * 0.1
+    X = rng.standard_normal((40, D))
+    C = X.T @ X
+    ref = P0 + 0.003 * (C @ P0 - P0 @ (P0.T @ C @ P0))
+    got = orc.oja_update_blocked(P0, X, 0.003, 0, chunk=64)
+    assert np.max(np.abs(got - ref)) < 1e-12 * np.max(np.abs(ref))
+
+
+def test_blocked_oja_chunks_stop_at_qr_points():
+    """tokens_seen = 50, QR every 64: chunks of 64 end at tokens 14, 78, ...,
+    so the result equals explicit calls on those pieces with a QR after each
+    piece that reaches a multiple of 64."""
+    rng = np.random.default_rng(502)
+    P0 = _orth(rng, D, 8)
+    X = rng.standard_normal((200, D)) * 0.3
+    got = orc.oja_update_blocked(P0, X, 0.02, 64, tokens_seen=50, chunk=64)
+    P = P0.copy()
+    for lo, hi in [(0, 14), (14, 78), (78, 142), (142, 200)]:
+        P = orc.oja_update_blocked(P, X[lo:hi], 0.02, 0, chunk=64)
+        if (50 + hi) % 64 == 0:
+            P = orc.qr_positive(P)
+    assert np.max(np.abs(got - P)) < 1e-13
+
+
+def test_blocked_oja_span_is_a_fixed_point_and_tracks_a_planted_subspace():
+    rng = np.random.default_rng(503)
+    P = _orth(rng, D, 6)
+    X = rng.standard_normal((50, 6)) @ P.T           # rows inside span(P)
+    assert np.max(np.abs(orc.oja_update_blocked(P, X, 0.05, 0) - P)) < 1e-13
+    U = _orth(rng, D, 6)                              # planted subspace
+    Xs = rng.standard_normal((4000, 6)) * 3.0 @ U.T + 0.05 * rng.standard_normal((4000, D))
+    P1 = orc.oja_update_blocked(_orth(rng, D, 6), Xs, 2e-3, 256, chunk=32)
+    s = np.linalg.svd(U.T @ P1, compute_uv=False)
+    assert np.min(s) > 0.99                           # cosines of the principal angles
+
+
+def test_blocked_oja_departs_from_sequential_in_proportion_to_the_chunk():
+    """Freezing P over a chunk of b tokens changes each chunk's update by a
+    term of order eta^2 b: over the same tokens the distance to the
+    sequential rule grows in proportion to b (chunk 1 is the rule itself)."""
+    rng = np.random.default_rng(504)
+    P0 = _orth(rng, D, 16)
+    X = rng.standard_normal((2048, D)) * np.exp(-np.arange(D) / 16.0)[None, :]
+    seq = orc.oja_update(P0, X, 1e-3, 256)
+    d = {b: np.max(np.abs(orc.oja_update_blocked(P0, X, 1e-3, 256, chunk=b) - seq))
+         for b in (1, 8, 64)}
+    assert d[1] < 1e-13
+    assert 5 < d[64] / d[8] < 11
+    assert d[8] < 1e-3
+
+
+# ------------------------------------------------------------ value amortisation
+
+def test_value_predictor_residual_is_orthogonal_to_the_key_codes():
+    """Least squares, checked through its normal equations: C_k^T (C_k A - C_v) = 0."""
+    rng = np.random.default_rng(600)
+    Ck, Cv = rng.standard_normal((300, 16)), rng.standard_normal((300, 8))
+    A = orc.fit_value_predictor(Ck, Cv)
+    assert A.shape == (16, 8)
+    assert np.max(np.abs(Ck.T @ (Ck @ A - Cv))) < 1e-10 * np.max(np.abs(Ck.T @ Cv))
+
+
+def test_value_predictor_recovers_an_exact_linear_map():
+    rng = np.random.default_rng(601)
+    Ck = rng.standard_normal((200, 12))
+    A_true = rng.standard_normal((12, 6))
+    A = orc.fit_value_predictor(Ck, Ck @ A_true)
+    assert np.max(np.abs(A - A_true)) < 1e-12
+    vals, kept = orc.amortised_value_codes(Ck, Ck @ A_true, A, keep=0)
+    assert np.max(np.abs(vals - Ck @ A_true)) < 1e-12 and not kept.any()
+
+
+def test_amortised_selection_worked_example():
+    """Pages of 4 tokens, keep 2: residual norms (by hand) 3, 1, 5, 1 | 2, 2, 0;
+    page one keeps tokens 2 and 0, page two keeps 4 and 5 (tie: earlier)."""
+    Ck = np.zeros((7, 1))
+    Cv = np.array([[3.0], [1.0], [-5.0], [1.0], [2.0], [-2.0], [0.0]])
+    A = np.zeros((1, 1))
+    vals, kept = orc.amortised_value_codes(Ck, Cv, A, keep=2, page=4)
+    assert kept.tolist() == [True, False, True, False, True, True, False]
+    assert vals[:, 0].tolist() == [3.0, 0.0, -5.0, 0.0, 2.0, -2.0, 0.0]
+
+
+def test_amortised_values_with_every_residual_kept_are_the_value_codes():
+    rng = np.random.default_rng(602)
+    Ck, Cv = rng.standard_normal((150, 16)), rng.standard_normal((150, 8))
+    A = orc.fit_value_predictor(Ck, Cv)
+    vals, kept = orc.amortised_value_codes(Ck, Cv, A, keep=64)
+    assert kept.all() and np.max(np.abs(vals - Cv)) < 1e-12
+
+
+def test_amortised_cache_attends_over_predicted_values_plus_kept_residuals():
+    """An amortised cache reads the value code A^T c_k + kept residual; the
+    predictor is fitted over the prompt and applies to later evictions."""
+    rng = np.random.default_rng(603)
+    P = rng.standard_normal((1, 1, D, 16)) * 0.2
+    k, v = rng.standard_normal((1, 1, 200, D)), rng.standard_normal((1, 1, 200, D))
+    c = orc.LatentCacheOracle(1, 1, 16, 16, n_sink=1, window=8, value_keep=16)
+    c.append(k[:, :, :150], v[:, :, :150], P, P)
+    c.amortise()
+    n0 = c.codes_k[0][0].shape[0]
+    A = orc.fit_value_predictor(c.codes_k[0][0], c.codes_v[0][0])
+    c.append(k[:, :, 150:], v[:, :, 150:], P, P)          # evictions after the fit
+    assert np.array_equal(c.A[0][0], A) and c.codes_k[0][0].shape[0] > n0
+    vals, kept = orc.amortised_value_codes(c.codes_k[0][0], c.codes_v[0][0], A, 16)
+    q = rng.standard_normal((1, 1, D))
+    Ka, Va = c.anchors(0, 0)
+    ref = orc.latent_attention(q[0, 0], P[0, 0], P[0, 0], c.codes_k[0][0], vals, Ka, Va, 0.1)
+    assert np.max(np.abs(c.attend(q, P, P, 0.1)[0, 0] - ref)) < 1e-14 * np.max(np.abs(ref))
+    assert kept.sum() == sum(min(16, len(range(p, min(p + 64, len(kept)))))
+                             for p in range(0, len(kept), 64))
