@@ -255,6 +255,74 @@ def time_layer_decode(lrkv, dev, wl, steps, calls, world, clk, seed):
             "attn_GBs": round(nbytes / (attn_ms * 1e-3) / 1e9, 1), "context": L}
 
 
+def time_code_variants(lrkv, dev, world, clk, hbm, wl, calls):
+    """Decode attention over the same Llama-3.1-8B-shaped layer with per-token
+    int8 codes and with value amortisation (key codes + 16 residual slots per
+    page, predictors fitted over the prompt): microseconds per call, the
+    bytes one call streams, and the fraction of the measured copy peak."""
+    import torch
+    from rank_kv_cache_lrkv_b200 import replicas
+    g = torch.Generator(device=dev)
+    g.manual_seed(99)
+    n = wl.T + 2
+    Kd, Vd = device_kv(dev, g, wl.B, wl.H_kv, n, torch.bfloat16)
+    Pk, Pv = device_basis(dev, g, (wl.H_kv,), wl.r_k), device_basis(dev, g, (wl.H_kv,), wl.r_v)
+    q = (torch.randn((wl.B, wl.H_q, HEAD_DIM), device=dev, generator=g) / HEAD_DIM ** 0.5).to(
+        torch.bfloat16)
+    o = torch.empty_like(q)
+    L = wl.T + 1
+    sink = min(L, wl.n_sink)
+    win = min(L - sink, wl.window)
+    lat = L - sink - win
+    units = wl.B * wl.H_kv
+    pages = -(-lat // 64)
+    anchors = units * (sink + win) * 2 * HEAD_DIM * 2 + 2 * wl.B * wl.H_q * HEAD_DIM * 2
+    out = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name in ("int8_codes", "amortised_values"):
+        cache = lrkv.LatentCache(wl.B, wl.H_kv, wl.r_k, wl.r_v, n, wl.n_sink, wl.window,
+                                 device=dev, **{name: True})
+        lrkv.compress(cache, Kd[:, :, :wl.T], Vd[:, :, :wl.T], Pk, Pv)
+        ws = lrkv.decode_workspace(cache, wl.H_q, device=dev)
+        if name == "amortised_values":
+            A = torch.zeros(wl.B, wl.H_kv, wl.r_k, wl.r_v, device=dev)
+            lrkv.amortise(cache, Vd[:, :, :wl.T], Pv, A)
+            lrkv.compress_amortised(cache, Kd[:, :, wl.T:L], Vd[:, :, wl.T:L], Pk, Pv, A)
+            call = lambda: lrkv.decode_attn_amortised(cache, q, Pk, Pv, A, wl.scale, o, ws)
+            slab = 64 * wl.r_k * 2 + 16 * wl.r_v * 2 + 128
+        else:
+            lrkv.compress(cache, Kd[:, :, wl.T:L], Vd[:, :, wl.T:L], Pk, Pv)
+            call = lambda: lrkv.decode_attn(cache, q, Pk, Pv, wl.scale, o, ws)
+            slab = 64 * (wl.r_k + wl.r_v) + 512
+        call()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, capture_error_mode="relaxed"):
+            for _ in range(calls):
+                call()
+        gr.replay()
+        torch.cuda.synchronize()
+        with clk.region():
+            e0.record()
+            gr.replay()
+            e1.record()
+            torch.cuda.synchronize()
+        us = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) * 1e3 / calls
+        assert lrkv.workspace_error(ws) == 0
+        nbytes = units * pages * slab + anchors
+        out[name] = {"attn_us": round(us, 3), "bytes_per_call": nbytes,
+                     "attn_GBs": round(nbytes / (us * 1e-6) / 1e9, 1),
+                     "frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
+                     "page_slab_bytes": slab,
+                     "bf16_page_slab_bytes": 64 * (wl.r_k + wl.r_v) * 2}
+        del gr, cache
+    del Kd, Vd
+    torch.cuda.empty_cache()
+    out["workload"] = wl.name
+    out["inputs"] = "device draws with the recipe's spectra; random orthonormal bases"
+    return out
+
+
 def time_sweep(lrkv, dev, world, clk, hbm, steps, calls):
     """Rank x batch sweep on the Qwen3-1.7B-shaped layer at T=16384: decode
     tokens/s and the roofline fraction of decode attention per point."""
@@ -780,6 +848,7 @@ def run_ours(args, rank, world):
                         "frac": round(res["attn_GBs"] / hbm, 4)})
             extra[key] = res
         out["workloads"] = extra
+        out["code_variants"] = time_code_variants(lrkv, dev, world, clk, hbm, base, C2)
         out["sweep"] = time_sweep(lrkv, dev, world, clk, hbm, S2, C2)
         out["stack"] = time_stack(lrkv, dev, world, clk, min(max(K, 4), 16))
     clk.__exit__()

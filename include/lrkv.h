@@ -151,6 +151,42 @@ int lrkv_compress(const lrkv_cache *cache, const void *k, const void *v,
                   const float *P_k, const float *P_v,
                   int64_t basis_batch_stride, void *stream);
 
+/* The same append for a value-amortised cache (LRKV_BF16_VA) whose
+ * predictors A [batch][num_kv_heads][rank_k][rank_v] (fp32, 16-byte
+ * aligned, as lrkv_amortise wrote them) exist: key codes are stored as by
+ * lrkv_compress, and the value residual e = P_v^T v - A^T c_k of each token
+ * that becomes latent enters its page's residual slots when it is among the
+ * page's LRKV_VA_KEEP largest so far (ties: the earlier token; a token that
+ * starts a page clears the page's slots first).  lrkv_compress on such a
+ * cache stores the key codes only (use it for the prompt, before
+ * lrkv_amortise).  LRKV_ERR_UNSUPPORTED for other caches. */
+int lrkv_compress_amortised(const lrkv_cache *cache, const void *k, const void *v,
+                            int32_t n_tokens, const int32_t *n_new, int64_t seq_stride,
+                            int64_t head_stride, const float *P_k, const float *P_v,
+                            int64_t basis_batch_stride, const float *A, void *stream);
+
+/* Fit the value predictors of a value-amortised cache right after its
+ * prompt was appended with lrkv_compress, and fill the residual slots of the
+ * prompt's pages (LowRAM abstract: a per-head predictor fitted at test
+ * time; residuals kept for the tokens it reconstructs worst).
+ *   v : the same prompt value rows (bf16, layout and strides as given to
+ *       lrkv_compress; n_tokens rows per sequence, read from token 0).
+ *   A : output [batch][num_kv_heads][rank_k][rank_v] fp32: per unit the
+ *       least-squares solution of C_k A = C_v over the prompt's latent
+ *       tokens (normal equations by Cholesky in fp64 with a ridge of
+ *       1e-12 trace(C_k^T C_k) / rank_k), C_k the stored key codes and
+ *       C_v = V P_v computed from v (value codes are never stored).
+ *   workspace : at least lrkv_amortise_workspace_bytes, 16-byte aligned;
+ *       the first 4 bytes are an error word (2 = a block-table entry out of
+ *       range).
+ * Three stream-ordered launches (partial Gram matrices, solve, residual
+ * slots).  LRKV_ERR_UNSUPPORTED for other caches. */
+size_t lrkv_amortise_workspace_bytes(const lrkv_cache *cache);
+int lrkv_amortise(const lrkv_cache *cache, const void *v, int32_t n_tokens,
+                  int64_t seq_stride, int64_t head_stride, const float *P_v,
+                  int64_t basis_batch_stride, float *A, void *workspace,
+                  size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace lrkv_decode_attn needs on the current device.  It
  * holds the folded queries, the split-K partial records and (first 4 bytes)
  * an error word; zero the error word when the workspace is allocated. */
@@ -174,6 +210,19 @@ int lrkv_decode_attn(const lrkv_cache *cache, const void *q, int32_t num_q_heads
                      const float *P_k, const float *P_v,
                      int64_t basis_batch_stride, float scale, void *o,
                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* Decode attention over a value-amortised cache: as lrkv_decode_attn, with
+ * each latent token's value code read as A^T c_k plus its kept residual.
+ * The split-K pass sums p c_k over the key codes and p e over the residual
+ * slots; the merge applies A once per unit, o = P_v (A^T sum p c_k +
+ * sum p e) / l + anchors.  A as for lrkv_compress_amortised;
+ * rank_k + rank_v <= 128.  lrkv_decode_attn refuses these caches
+ * (LRKV_ERR_UNSUPPORTED) and this call refuses other caches. */
+int lrkv_decode_attn_amortised(const lrkv_cache *cache, const void *q, int32_t num_q_heads,
+                               const float *P_k, const float *P_v,
+                               int64_t basis_batch_stride, const float *A, float scale,
+                               void *o, void *workspace, size_t workspace_bytes,
+                               void *stream);
 
 /* Decode attention that allocates nothing and takes no workspace.  The
  * pages have no counterpart to this entry point: it exists for callers that

@@ -22,13 +22,16 @@ int check_rank(int r, int dtype) {
 
 int check_cache(const lrkv_cache* c) {
   if (!c) return LRKV_ERR_ARG;
-  if (c->dtype != LRKV_BF16 && c->dtype != LRKV_F32 && c->dtype != LRKV_BF16_Q8)
+  if (c->dtype != LRKV_BF16 && c->dtype != LRKV_F32 && c->dtype != LRKV_BF16_Q8 &&
+      c->dtype != LRKV_BF16_VA)
     return LRKV_ERR_UNSUPPORTED;
   if (c->head_dim != kHeadDim) return LRKV_ERR_UNSUPPORTED;
   if (c->batch < 1 || c->batch > LRKV_MAX_BATCH || c->num_kv_heads < 1) return LRKV_ERR_ARG;
   int rc = check_rank(c->rank_k, c->dtype);
   if (rc == LRKV_OK) rc = check_rank(c->rank_v, c->dtype);
   if (rc != LRKV_OK) return rc;
+  // value-amortised records hold rank_k + rank_v sums per head
+  if (c->dtype == LRKV_BF16_VA && c->rank_k + c->rank_v > kHeadDim) return LRKV_ERR_UNSUPPORTED;
   if (c->n_sink < 0 || c->n_sink > 1 || c->window < 0 || c->window > (1 << 20)) return LRKV_ERR_ARG;
   if (c->num_pages < 1 || c->max_pages_per_seq < 1) return LRKV_ERR_ARG;
   if (!c->codes || !c->block_table || !c->seq_len || !c->append_counter) return LRKV_ERR_ARG;
@@ -87,9 +90,11 @@ const char* lrkv_status_string(int s) {
   }
 }
 
-int lrkv_compress(const lrkv_cache* cache, const void* k, const void* v, int32_t n_tokens,
-                  const int32_t* n_new, int64_t seq_stride, int64_t head_stride, const float* P_k,
-                  const float* P_v, int64_t basis_batch_stride, void* stream) {
+// The checks of lrkv_compress and lrkv_compress_amortised, then the launch.
+static int compress_checked(const lrkv_cache* cache, const void* k, const void* v,
+                            int32_t n_tokens, const int32_t* n_new, int64_t seq_stride,
+                            int64_t head_stride, const float* P_k, const float* P_v,
+                            int64_t basis_batch_stride, const float* A, void* stream) {
   int rc = check_cache(cache);
   if (rc != LRKV_OK) return rc;
   if (n_tokens < 0) return LRKV_ERR_ARG;
@@ -103,7 +108,45 @@ int lrkv_compress(const lrkv_cache* cache, const void* k, const void* v, int32_t
   const long long cap = (long long)cache->max_pages_per_seq * kLatPage + cache->n_sink + cache->window;
   if (n_tokens > cap) return LRKV_ERR_CAPACITY;
   return compress_launch(*cache, k, v, n_tokens, n_new, seq_stride, head_stride, P_k, P_v,
-                         basis_batch_stride, static_cast<cudaStream_t>(stream));
+                         basis_batch_stride, static_cast<cudaStream_t>(stream), A);
+}
+
+int lrkv_compress(const lrkv_cache* cache, const void* k, const void* v, int32_t n_tokens,
+                  const int32_t* n_new, int64_t seq_stride, int64_t head_stride, const float* P_k,
+                  const float* P_v, int64_t basis_batch_stride, void* stream) {
+  return compress_checked(cache, k, v, n_tokens, n_new, seq_stride, head_stride, P_k, P_v,
+                          basis_batch_stride, nullptr, stream);
+}
+
+int lrkv_compress_amortised(const lrkv_cache* cache, const void* k, const void* v,
+                            int32_t n_tokens, const int32_t* n_new, int64_t seq_stride,
+                            int64_t head_stride, const float* P_k, const float* P_v,
+                            int64_t basis_batch_stride, const float* A, void* stream) {
+  if (!cache || cache->dtype != LRKV_BF16_VA) return cache ? LRKV_ERR_UNSUPPORTED : LRKV_ERR_ARG;
+  if (!A) return LRKV_ERR_ARG;
+  return compress_checked(cache, k, v, n_tokens, n_new, seq_stride, head_stride, P_k, P_v,
+                          basis_batch_stride, A, stream);
+}
+
+size_t lrkv_amortise_workspace_bytes(const lrkv_cache* cache) {
+  if (check_cache(cache) != LRKV_OK || cache->dtype != LRKV_BF16_VA) return 0;
+  return amortise_workspace_bytes(cache->batch, cache->num_kv_heads, cache->rank_k,
+                                  cache->rank_v);
+}
+
+int lrkv_amortise(const lrkv_cache* cache, const void* v, int32_t n_tokens, int64_t seq_stride,
+                  int64_t head_stride, const float* P_v, int64_t basis_batch_stride, float* A,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_cache(cache);
+  if (rc != LRKV_OK) return rc;
+  if (cache->dtype != LRKV_BF16_VA) return LRKV_ERR_UNSUPPORTED;
+  if (!v || !P_v || !A || !workspace || n_tokens < 1 || basis_batch_stride < 0 ||
+      !aligned16(v) || !aligned16(P_v) || !aligned16(A) || !aligned16(workspace) ||
+      seq_stride % 8 != 0 || head_stride % 8 != 0 || basis_batch_stride % 4 != 0)
+    return LRKV_ERR_ARG;
+  if (workspace_bytes < lrkv_amortise_workspace_bytes(cache)) return LRKV_ERR_WORKSPACE;
+  return amortise_launch(*cache, v, n_tokens, seq_stride, head_stride, P_v, basis_batch_stride,
+                         A, workspace, static_cast<cudaStream_t>(stream));
 }
 
 size_t lrkv_decode_workspace_bytes(const lrkv_cache* cache, int32_t num_q_heads) {
@@ -114,11 +157,14 @@ size_t lrkv_decode_workspace_bytes(const lrkv_cache* cache, int32_t num_q_heads)
                                 cache->dtype);
 }
 
-int lrkv_decode_attn(const lrkv_cache* cache, const void* q, int32_t num_q_heads,
-                     const float* P_k, const float* P_v, int64_t basis_batch_stride, float scale,
-                     void* o, void* workspace, size_t workspace_bytes, void* stream) {
+static int decode_checked(const lrkv_cache* cache, const void* q, int32_t num_q_heads,
+                          const float* P_k, const float* P_v, int64_t basis_batch_stride,
+                          const float* A, float scale, void* o, void* workspace,
+                          size_t workspace_bytes, void* stream) {
   int rc = check_cache(cache);
   if (rc != LRKV_OK) return rc;
+  if ((cache->dtype == LRKV_BF16_VA) != (A != nullptr)) return LRKV_ERR_UNSUPPORTED;
+  if (A && !aligned16(A)) return LRKV_ERR_ARG;
   rc = check_heads(cache->num_kv_heads, num_q_heads);
   if (rc != LRKV_OK) return rc;
   if (!q || !o || !P_k || !P_v || !workspace || basis_batch_stride < 0) return LRKV_ERR_ARG;
@@ -136,8 +182,24 @@ int lrkv_decode_attn(const lrkv_cache* cache, const void* q, int32_t num_q_heads
   L.maxp_fr = (cache->n_sink + cache->window + kFrTile - 1) / kFrTile;
   L.num_pages_fr = 0;
   L.q = q; L.P_k = P_k; L.P_v = P_v; L.basis_bs = basis_batch_stride; L.scale = scale;
-  L.o = o; L.ws = workspace; L.ws_bytes = workspace_bytes;
+  L.o = o; L.ws = workspace; L.ws_bytes = workspace_bytes; L.A = A;
   return decode_launch(L, static_cast<cudaStream_t>(stream));
+}
+
+int lrkv_decode_attn(const lrkv_cache* cache, const void* q, int32_t num_q_heads,
+                     const float* P_k, const float* P_v, int64_t basis_batch_stride, float scale,
+                     void* o, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_checked(cache, q, num_q_heads, P_k, P_v, basis_batch_stride, nullptr, scale, o,
+                        workspace, workspace_bytes, stream);
+}
+
+int lrkv_decode_attn_amortised(const lrkv_cache* cache, const void* q, int32_t num_q_heads,
+                               const float* P_k, const float* P_v, int64_t basis_batch_stride,
+                               const float* A, float scale, void* o, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (!A) return LRKV_ERR_ARG;
+  return decode_checked(cache, q, num_q_heads, P_k, P_v, basis_batch_stride, A, scale, o,
+                        workspace, workspace_bytes, stream);
 }
 
 int lrkv_oja_update(float* P, int32_t num_streams, int32_t rank, int64_t basis_stride,
@@ -194,7 +256,7 @@ int lrkv_rebase(const lrkv_cache* cache, const float* P_k_old, const float* P_k_
       !aligned16(P_v_old) || !aligned16(P_v_new))
     return LRKV_ERR_ARG;
   if (workspace_bytes < lrkv_rebase_workspace_bytes(cache)) return LRKV_ERR_WORKSPACE;
-  if (cache->dtype == LRKV_BF16_Q8) return LRKV_ERR_UNSUPPORTED;
+  if (cache->dtype == LRKV_BF16_Q8 || cache->dtype == LRKV_BF16_VA) return LRKV_ERR_UNSUPPORTED;
   if (!P_k_old && !P_v_old) return LRKV_OK;
   return rebase_launch(*cache, P_k_old, P_k_new, P_v_old, P_v_new, basis_batch_stride, workspace,
                        static_cast<cudaStream_t>(stream));

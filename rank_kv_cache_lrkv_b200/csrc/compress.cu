@@ -29,10 +29,11 @@ constexpr int kBulkRows = 64;     // tokens per bulk_compress CTA
 constexpr int kRowBatch = 16;  // token rows projected per pass
 // Dynamic shared memory of append_kernel: the unit's basis [128][r_k + r_v]
 // fp32, rows [kRowBatch][k, v][128] fp32, partial sums [256], and a page per row.
-// (+ one row of codes [256] and two scales for int8 codes)
+// (+ one row of codes [256] and two scales for int8 codes, a value residual
+// [128] and its slot for value-amortised slabs)
 inline size_t append_smem_bytes(int rk, int rv) {
   return ((size_t)kHeadDim * (rk + rv) + (size_t)kRowBatch * 2 * kHeadDim + 256 + kRowBatch +
-          256 + 4) * 4;
+          256 + 4 + kHeadDim + 4) * 4;
 }
 
 // One CTA per (KV head, sequence).  Latency matters here (a decode step
@@ -54,6 +55,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
   int* pg = reinterpret_cast<int*>(red + 256);                         // [row]
   float* crow = red + 256 + kRowBatch;                                 // [NJ] one row's codes
   float* qscale = crow + 256;                                          // [2] its scales
+  float* ev = qscale + 4;                                              // [rv] value residual
+  int* vslot = reinterpret_cast<int*>(ev + kHeadDim);                  // its slot
   const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
 
   // Launched with programmatic dependent launch: wait for the previous grid
@@ -188,6 +191,64 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
               static_cast<uint8_t>(static_cast<int8_t>(q8_code(crow[tid], qscale[isv])));
           if (jj == 0)
             *reinterpret_cast<float*>(cb + q8_scale_off(a, pg[rr], kvh, j, isv)) = qscale[isv];
+        }
+      } else if (a.va) {
+        // value-amortised slab: the key code is stored; the value residual
+        // against the fitted predictor, e = c_v - A^T c_k, enters the page's
+        // slots when it is among the page's LRKV_VA_KEEP largest so far
+        const int j = token_of(r0 + rr) - a.n_sink;
+        if (tid < NJ) {
+          float c = 0.f;
+          for (int seg = 0; seg < nseg; ++seg) c += red[seg * NJ + tid];
+          crow[tid] = c;
+          if (tid < a.rk && pg[rr] >= 0) codes[code_off_in<T>(a, pg[rr], kvh, j, tid, 0)] = from_f<T>(c);
+        }
+        if (a.A && pg[rr] >= 0) {
+          __syncthreads();
+          const float* Am = a.A + ((size_t)b * a.H_kv + kvh) * a.rk * a.rv;
+          if (tid < a.rv) {
+            float pr = 0.f;
+            for (int k = 0; k < a.rk; ++k) pr = fmaf(__ldg(Am + (size_t)k * a.rv + tid), crow[k], pr);
+            ev[tid] = crow[a.rk + tid] - pr;
+          }
+          __syncthreads();
+          uint8_t* slab = static_cast<uint8_t*>(a.codes) +
+                          ((size_t)pg[rr] * a.H_kv + kvh) * va_slab_bytes(a.rk, a.rv);
+          int* sidx = reinterpret_cast<int*>(slab + (size_t)kLatPage * a.rk * 2 + kVaKeep * a.rv * 2);
+          float* snrm = reinterpret_cast<float*>(sidx + kVaKeep);
+          if (tid < 32) {
+            float ss = 0.f;
+            for (int n = tid; n < a.rv; n += 32) ss = fmaf(ev[n], ev[n], ss);
+            ss = warp_sum(ss);
+            if (tid == 0) {
+              const int row = j % kLatPage;
+              if (row == 0)  // a fresh page: no slot used yet
+                for (int q = 0; q < kVaKeep; ++q) { sidx[q] = -1; snrm[q] = -1.f; }
+              int best = -1;
+              for (int q = 0; q < kVaKeep && best < 0; ++q)
+                if (sidx[q] < 0) best = q;
+              if (best < 0) {
+                // the smallest kept norm (ties: the later row) gives way to a
+                // strictly larger one, so the earlier token wins ties
+                best = 0;
+                for (int q = 1; q < kVaKeep; ++q)
+                  if (snrm[q] < snrm[best] || (snrm[q] == snrm[best] && sidx[q] > sidx[best]))
+                    best = q;
+                if (!(ss > snrm[best])) best = -1;
+              }
+              if (best >= 0) {
+                sidx[best] = row;
+                snrm[best] = ss;
+              }
+              *vslot = best;
+            }
+          }
+          __syncthreads();
+          const int sl = *vslot;
+          if (sl >= 0 && tid < a.rv) {
+            __nv_bfloat16* res = reinterpret_cast<__nv_bfloat16*>(slab + (size_t)kLatPage * a.rk * 2);
+            res[((tid >> 3) * kVaKeep + sl) * 8 + (tid & 7)] = __float2bfloat16_rn(ev[tid]);
+          }
         }
       } else if (tid < NJ && pg[rr] >= 0) {
         float c = 0.f;
@@ -480,7 +541,7 @@ static int bulk_launch(const AppendArgs& a, cudaStream_t st) {
     if (rc != LRKV_OK) return rc;
     const int sms = info.sms, optin = info.optin;
     rc = bulk_compress_tc_launch(a, sms, optin, st);
-    if (rc != LRKV_ERR_UNSUPPORTED || a.q8) return rc;
+    if (rc != LRKV_ERR_UNSUPPORTED || a.q8 || a.va) return rc;
     // persistent: one CTA per SM; 128-token tiles (8 warps) when they fit
     const bool big = bulk_mma_smem_bytes(a.rk, a.rv, 128, a.B) <= (size_t)optin;
     const size_t smem = bulk_mma_smem_bytes(a.rk, a.rv, big ? 128 : 64, a.B);
@@ -533,12 +594,14 @@ static int compress_t(const AppendArgs& a, cudaStream_t st) {
 
 int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, const int* n_new,
                     long long seq_stride, long long head_stride, const float* P_k,
-                    const float* P_v, long long basis_bs, cudaStream_t st) {
+                    const float* P_v, long long basis_bs, cudaStream_t st, const float* A) {
   AppendArgs a;
   a.B = c.batch; a.H_kv = c.num_kv_heads; a.rk = c.rank_k; a.rv = c.rank_v;
   a.n_sink = c.n_sink; a.W = c.window; a.maxp = c.max_pages_per_seq; a.num_pages = c.num_pages;
   a.n = n; a.anchor_tiles = (c.n_sink + c.window + kFrTile - 1) / kFrTile;
   a.q8 = c.dtype == LRKV_BF16_Q8 ? 1 : 0;
+  a.va = c.dtype == LRKV_BF16_VA ? 1 : 0;
+  a.A = A;
   a.codes = c.codes; a.anchors = c.anchors;
   a.bt = c.block_table; a.seq_len = c.seq_len; a.counter = c.append_counter; a.n_new = n_new;
   a.k = k; a.v = v; a.seq_stride = seq_stride; a.head_stride = head_stride;

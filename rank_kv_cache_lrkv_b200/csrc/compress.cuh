@@ -16,6 +16,8 @@ __device__ inline int appended(const int* n_new, int n, int b) {
 struct AppendArgs {
   int B, H_kv, rk, rv, n_sink, W, maxp, num_pages, n, anchor_tiles;
   int q8;            // codes stored as per-token int8 + fp32 scales (bf16 inputs)
+  int va;            // value-amortised slabs: key codes + residual slots
+  const float* A;    // value predictors [B][H_kv][rk][rv] (va; NULL: not fitted yet)
   void *codes, *anchors;
   const int* bt;
   int* seq_len;
@@ -64,9 +66,12 @@ template <typename T>
 __device__ inline long long code_off_in(const AppendArgs& a, int page, int kvh, int j, int jj,
                                         int isv) {
   constexpr int CE = Elem<T>::CE;
-  const int nch = (a.rk + a.rv) / CE;
+  // elements per slab: key and value codes, or (value-amortised) the key
+  // codes followed by the residual slots
+  const long long slab = a.va ? va_slab_bytes(a.rk, a.rv) / (long long)sizeof(T)
+                              : (long long)kLatPage * (a.rk + a.rv);
   const int chunk = isv * (a.rk / CE) + jj / CE;
-  return ((((long long)page * a.H_kv + kvh) * nch + chunk) * kLatPage + j % kLatPage) * CE +
+  return ((long long)page * a.H_kv + kvh) * slab + ((long long)chunk * kLatPage + j % kLatPage) * CE +
          jj % CE;
 }
 

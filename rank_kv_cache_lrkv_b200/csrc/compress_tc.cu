@@ -111,6 +111,23 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
                  "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
                  "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])::"memory");
 }
+// The same load without the wait: several may be in flight; tmem_wait_tie
+// then waits for all of them and ties one group's registers to the wait.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_tie(uint32_t (&v)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])::"memory");
+}
 // Generic-proxy writes to shared memory become visible to the async proxy.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -255,7 +272,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int lo = bulk_range_lo(blockIdx.x, total, gridDim.x);
   const int hi = bulk_range_lo(blockIdx.x + 1, total, gridDim.x);
   if (lo >= hi) return;  // uniform across the CTA
-  const int njobs = 2 * (hi - lo);
+  // jobs: (tile, side) pairs; value-amortised caches store key codes only
+  const int sides = a.va ? 1 : 2;
+  const int njobs = sides * (hi - lo);
 
   if (warp == 1) {
     tmem_alloc(taddr_slot, kTcTmemCols);
@@ -331,10 +350,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int s = j % NS, n = j / NS;
         if (n > 0 && !tc_wait(&empty[s], (n - 1) & 1, fail)) break;
         int b, kvh, i;
-        locate(lo + (j >> 1), b, kvh, i);
+        locate(lo + j / sides, b, kvh, i);
         const int t0 = srlo[b] + i * kTcRows;
         uint8_t* dst = sm + pl.stages + (size_t)s * kTcStageBytes;
-        const CUtensorMap* tm = (j & 1) ? &tmV : &tmK;
+        const CUtensorMap* tm = (j % sides) ? &tmV : &tmK;
         mbar_arrive_expect_tx(&full[s], kTcStageBytes);
         tma_load_4d(dst, tm, 0, t0, kvh, b, &full[s], pol);
         tma_load_4d(dst + kTcHalfBytes, tm, 64, t0, kvh, b, &full[s], pol);
@@ -357,10 +376,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int cur_unit = -1, m = -1;
     for (int j = 0; j < njobs; ++j) {
       if (__shfl_sync(0xffffffffu, *fail, 0)) break;
-      const int side = j & 1;
+      const int side = j % sides;
       if (side == 0) {
         int b, kvh, i;
-        locate(lo + (j >> 1), b, kvh, i);
+        locate(lo + j / sides, b, kvh, i);
         const int unit = b * a.H_kv + kvh;
         if (unit != cur_unit) {
           // the unit before is done once its MMAs complete: its buffer may refill
@@ -433,67 +452,73 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int page = -1, jlat = 0, kvh = 0, npage = -1, njlat = 0, nkvh = 0;
     row_of(lo, nkvh, njlat, npage);
     for (int j = 0; j < njobs; ++j) {
-      const int side = j & 1, buf = j % kTcAcc, u = j / kTcAcc;
+      const int side = j % sides, buf = j % kTcAcc, u = j / kTcAcc;
       if (side == 0) {
         page = npage;
         jlat = njlat;
         kvh = nkvh;
-        if (lo + (j >> 1) + 1 < hi) row_of(lo + (j >> 1) + 1, nkvh, njlat, npage);
+        if (lo + j / sides + 1 < hi) row_of(lo + j / sides + 1, nkvh, njlat, npage);
       }
       if (!tc_wait_warp(&accf[buf], u & 1, fail, lane)) break;
       tc_fence_after();
       const int r = side ? a.rv : a.rk;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kTcAccCols;
+      // every column group of the row in flight at once, then one wait
+      uint32_t v[8][16];
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (16 * c < r) tmem_ld16_async(tbase + 16 * c, v[c]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (16 * c < r) tmem_wait_tie(v[c]);
       if (a.q8) {
         // per-token int8 (r is a multiple of 16): the row's max |c| sets the
-        // scale, then a second pass over TMEM writes the codes under it
-        float m = 0.f;
-        for (int c0 = 0; c0 < r; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(tbase + c0, v);
+        // scale, the codes follow under it
+        float mx = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(__uint_as_float(v[e])));
-        }
-        const float sc = __fdiv_rn(m, 127.f);
+        for (int c = 0; c < 8; ++c)
+          if (16 * c < r)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(__uint_as_float(v[c][e])));
+        const float sc = __fdiv_rn(mx, 127.f);
         uint8_t* cb = static_cast<uint8_t*>(a.codes);
-        for (int c0 = 0; c0 < r; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(tbase + c0, v);
-          if (page >= 0) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e4 = 0; e4 < 4; ++e4) {
-              uint32_t x = 0;
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                x |= (static_cast<uint32_t>(q8_code(__uint_as_float(v[4 * e4 + e]), sc)) & 0xffu)
-                     << (8 * e);
-              w[e4] = x;
-            }
-            *reinterpret_cast<uint4*>(cb + q8_code_off(a, page, kvh, jlat, c0, side)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-        if (page >= 0) *reinterpret_cast<float*>(cb + q8_scale_off(a, page, kvh, jlat, side)) = sc;
-      } else
-      for (int c0 = 0; c0 < r; c0 += 16) {  // r is a multiple of 8
-        uint32_t v[16];
-        tmem_ld16(tbase + c0, v);
         if (page >= 0) {
 #pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (16 * c < r) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e4 = 0; e4 < 4; ++e4) {
+                uint32_t x = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  x |= (static_cast<uint32_t>(q8_code(__uint_as_float(v[c][4 * e4 + e]), sc)) &
+                        0xffu)
+                       << (8 * e);
+                w[e4] = x;
+              }
+              *reinterpret_cast<uint4*>(cb + q8_code_off(a, page, kvh, jlat, 16 * c, side)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+          *reinterpret_cast<float*>(cb + q8_scale_off(a, page, kvh, jlat, side)) = sc;
+        }
+      } else if (page >= 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (c0 + 8 * h < r) {
+            const int c8 = 16 * c + 8 * h;  // r is a multiple of 8
+            if (c8 < r) {
               const uint4 w = make_uint4(
-                  pack_bf16x2(__uint_as_float(v[8 * h + 0]), __uint_as_float(v[8 * h + 1])),
-                  pack_bf16x2(__uint_as_float(v[8 * h + 2]), __uint_as_float(v[8 * h + 3])),
-                  pack_bf16x2(__uint_as_float(v[8 * h + 4]), __uint_as_float(v[8 * h + 5])),
-                  pack_bf16x2(__uint_as_float(v[8 * h + 6]), __uint_as_float(v[8 * h + 7])));
-              *reinterpret_cast<uint4*>(codes +
-                                        code_off_in<bf16>(a, page, kvh, jlat, c0 + 8 * h, side)) =
+                  pack_bf16x2(__uint_as_float(v[c][8 * h + 0]), __uint_as_float(v[c][8 * h + 1])),
+                  pack_bf16x2(__uint_as_float(v[c][8 * h + 2]), __uint_as_float(v[c][8 * h + 3])),
+                  pack_bf16x2(__uint_as_float(v[c][8 * h + 4]), __uint_as_float(v[c][8 * h + 5])),
+                  pack_bf16x2(__uint_as_float(v[c][8 * h + 6]), __uint_as_float(v[c][8 * h + 7])));
+              *reinterpret_cast<uint4*>(codes + code_off_in<bf16>(a, page, kvh, jlat, c8, side)) =
                   w;
             }
           }
-        }
       }
       tc_fence_before();
       __syncwarp();

@@ -75,8 +75,15 @@ struct DecodeArgs {
   int C;               // CTAs of the split grid
   int NS;              // ring stages
   int stage_bytes;
-  int dq_bytes;        // int8 codes: per-consumer dequantised half page (bytes)
+  int dq_bytes;        // int8 codes: per-consumer dequantised half page (bytes);
+                       // value-amortised slabs: per-consumer page weights
+  const float* A;      // value-amortised slabs: predictors [B][H_kv][rk][rv]
+  int rw;              // latent record width per head: rv, or rk + rv (amortised)
 };
+
+constexpr int kModePlain = 0;  // bf16 / fp32 latent codes
+constexpr int kModeQ8 = 1;     // per-token int8 codes + scales
+constexpr int kModeVA = 2;     // key codes + value residual slots
 
 __host__ __device__ inline int hdr_floats(int G) { return ((2 * G + 3) / 4) * 4; }
 
@@ -478,6 +485,188 @@ __device__ inline void write_record_mma(float* rec, int rvd, const float (&m)[2]
     }
 }
 
+// One value-amortised page (64 tokens): the scores and the online softmax as
+// in process_tile_mma; then acck += p c_k over the key codes (the value
+// prediction A^T c_k is linear, so the merge applies A to the sum once), and
+// acce += p e over the page's residual slots, whose token rows come from the
+// slab (a slot with row -1, or at or past n_valid, weighs 0).  pw: this
+// warp's [64][8] fp32 page weights, so a slot can find its token's weight.
+template <int KS, int VB>
+__device__ __forceinline__ void process_tile_va(const uint4* kch, int n_valid, int nck, int ncv,
+                                                const QFrag<KS>& qf, float (&m)[2], float (&l)[2],
+                                                float (&acck)[2][KS][4], float (&acce)[VB][4],
+                                                float* pw, int lane) {
+  constexpr int TT = kLatPage, MB = TT / 16;
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t kbase = smem_u32(kch);
+  const uint32_t rbase = kbase + (uint32_t)(TT * nck * 16);  // residual rows [ncv][16][8]
+  const int* sidx = reinterpret_cast<const int*>(reinterpret_cast<const uint8_t*>(kch) +
+                                                 TT * nck * 16 + kVaKeep * ncv * 16);
+  const int nks = (nck + 1) >> 1, nvb = (ncv + 1) >> 1;
+  const bool partial = n_valid < TT;
+
+  float sc[MB][4], sl[MB][4];
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[mb][i] = sl[mb][i] = 0.f;
+  const int arow = lane & 15, ahalf = lane >> 4;
+#pragma unroll
+  for (int s = 0; s < KS; ++s) {
+    if (s < nks) {
+      const int c = min(2 * s + ahalf, nck - 1);
+      uint32_t a[MB][4];
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb)
+        ldsm_x4(kbase + (uint32_t)((c * TT + mb * 16 + arow) * 16), a[mb]);
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) mma_bf16_16816(sc[mb], a[mb], qf.hi[s][0], qf.hi[s][1]);
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) mma_bf16_16816(sl[mb], a[mb], qf.lo[s][0], qf.lo[s][1]);
+    }
+  }
+  float mt0 = -INFINITY, mt1 = -INFINITY;
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[mb][i] += sl[mb][i];
+    if (partial) {
+      if (mb * 16 + g >= n_valid) sc[mb][0] = sc[mb][1] = -INFINITY;
+      if (mb * 16 + g + 8 >= n_valid) sc[mb][2] = sc[mb][3] = -INFINITY;
+    }
+    mt0 = fmaxf(mt0, fmaxf(sc[mb][0], sc[mb][2]));
+    mt1 = fmaxf(mt1, fmaxf(sc[mb][1], sc[mb][3]));
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, o));
+    mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
+  }
+  const float mn0 = fmaxf(m[0], mt0), mn1 = fmaxf(m[1], mt1);
+  const float al0 = ex2_approx(m[0] - mn0), al1 = ex2_approx(m[1] - mn1);
+  m[0] = mn0;
+  m[1] = mn1;
+  float ps0 = 0.f, ps1 = 0.f;
+  uint32_t ph[MB][2], pl[MB][2];
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+    const float p0 = ex2_approx(sc[mb][0] - mn0), p1 = ex2_approx(sc[mb][1] - mn1);
+    const float p2 = ex2_approx(sc[mb][2] - mn0), p3 = ex2_approx(sc[mb][3] - mn1);
+    ps0 += p0 + p2;
+    ps1 += p1 + p3;
+    // weights by (token row, head) for the residual slots
+    pw[(mb * 16 + g) * 8 + 2 * t] = p0;
+    pw[(mb * 16 + g) * 8 + 2 * t + 1] = p1;
+    pw[(mb * 16 + g + 8) * 8 + 2 * t] = p2;
+    pw[(mb * 16 + g + 8) * 8 + 2 * t + 1] = p3;
+    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+    ph[mb][0] = movmatrix_trans(h01);
+    ph[mb][1] = movmatrix_trans(h23);
+    pl[mb][0] = movmatrix_trans(pack_bf16x2(p0 - bf_lo(h01), p1 - bf_hi(h01)));
+    pl[mb][1] = movmatrix_trans(pack_bf16x2(p2 - bf_lo(h23), p3 - bf_hi(h23)));
+  }
+  l[0] = fmaf(l[0], al0, ps0);
+  l[1] = fmaf(l[1], al1, ps1);
+#pragma unroll
+  for (int kb = 0; kb < KS; ++kb)
+#pragma unroll
+    for (int hl = 0; hl < 2; ++hl) {
+      acck[hl][kb][0] *= al0;
+      acck[hl][kb][1] *= al1;
+      acck[hl][kb][2] *= al0;
+      acck[hl][kb][3] *= al1;
+    }
+#pragma unroll
+  for (int vb = 0; vb < VB; ++vb) {
+    acce[vb][0] *= al0;
+    acce[vb][1] *= al1;
+    acce[vb][2] *= al0;
+    acce[vb][3] *= al1;
+  }
+  // acck^T (key dim x head) += C_k^T . P^T over the page's tokens
+  const int vrow = ((lane >> 4) << 3) + (lane & 7), vhalf = (lane >> 3) & 1;
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+    if (mb * 16 < n_valid) {
+#pragma unroll
+      for (int kb = 0; kb < KS; ++kb) {
+        if (kb < nks) {
+          const int c = min(2 * kb + vhalf, nck - 1);
+          uint32_t a[4];
+          ldsm_x4_trans(kbase + (uint32_t)((c * TT + mb * 16 + vrow) * 16), a);
+          if (partial) {
+            const int k0 = mb * 16 + 2 * t;
+            a[0] = mask_tokens(a[0], k0, n_valid);
+            a[1] = mask_tokens(a[1], k0, n_valid);
+            a[2] = mask_tokens(a[2], k0 + 8, n_valid);
+            a[3] = mask_tokens(a[3], k0 + 8, n_valid);
+          }
+          mma_bf16_16816(acck[0][kb], a, ph[mb][0], ph[mb][1]);
+          mma_bf16_16816(acck[1][kb], a, pl[mb][0], pl[mb][1]);
+        }
+      }
+    }
+  }
+  __syncwarp();  // pw is complete
+  // acce^T (value dim x head) += E^T . P_slots^T over the 16 residual slots
+  auto slot_p = [&](int sl) {
+    const int r = sidx[sl];
+    return (r >= 0 && r < n_valid) ? pw[r * 8 + g] : 0.f;
+  };
+  const uint32_t b0 = pack_bf16x2(slot_p(2 * t), slot_p(2 * t + 1));
+  const uint32_t b1 = pack_bf16x2(slot_p(2 * t + 8), slot_p(2 * t + 9));
+#pragma unroll
+  for (int vb = 0; vb < VB; ++vb) {
+    if (vb < nvb) {
+      const int c = min(2 * vb + vhalf, ncv - 1);
+      uint32_t a[4];
+      ldsm_x4_trans(rbase + (uint32_t)((c * kVaKeep + vrow) * 16), a);
+      mma_bf16_16816(acce[vb], a, b0, b1);
+    }
+  }
+  __syncwarp();  // pw may be rewritten by the next page
+}
+
+// The warp's (m, l, acck, acce) of the value-amortised path -> record
+// (m[G], l[G], then per head [rk] key-code sums and [rv] residual sums).
+template <int G, int KS, int VB>
+__device__ inline void write_record_va(float* rec, int rk, int rv, const float (&m)[2],
+                                       const float (&l)[2], const float (&acck)[2][KS][4],
+                                       const float (&acce)[VB][4], int lane) {
+  const int g = lane >> 2, t = lane & 3, H = hdr_floats(G), rw = rk + rv;
+  float l0 = l[0], l1 = l[1];
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  const int h0 = 2 * t, h1 = 2 * t + 1;
+  if (g == 0) {
+    if (h0 < G) { rec[h0] = m[0]; rec[G + h0] = l0; }
+    if (h1 < G) { rec[h1] = m[1]; rec[G + h1] = l1; }
+  }
+#pragma unroll
+  for (int kb = 0; kb < KS; ++kb)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int d = kb * 16 + g + 8 * r;
+      if (d < rk) {
+        if (h0 < G) rec[H + h0 * rw + d] = acck[0][kb][2 * r] + acck[1][kb][2 * r];
+        if (h1 < G) rec[H + h1 * rw + d] = acck[0][kb][2 * r + 1] + acck[1][kb][2 * r + 1];
+      }
+    }
+#pragma unroll
+  for (int vb = 0; vb < VB; ++vb)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int d = vb * 16 + g + 8 * r;
+      if (d < rv) {
+        if (h0 < G) rec[H + h0 * rw + rk + d] = acce[vb][2 * r];
+        if (h1 < G) rec[H + h1 * rw + rk + d] = acce[vb][2 * r + 1];
+      }
+    }
+}
+
 // ------------------------------------------------------------ q-fold kernel
 constexpr int kFoldThreads = 128;  // small, so q-fold CTAs fit beside split CTAs
 constexpr int kFoldSplit = 2;      // CTAs per unit, each folding a share of the columns
@@ -751,10 +940,11 @@ __device__ __forceinline__ void dequant_half(const uint4* slab, int half, int rk
 // 168 registers: ten warps, three on two of the SM's four sub-partitions
 // (16K registers each).  More consumer warps hide more of each warp's
 // dependent latency; fewer registers spill in the wider rank classes.
-// kQ8: the latent pages hold per-token int8 codes and fp32 scales; each
-// consumer dequantises a page half by half into its own bf16 buffer and
-// runs the bf16 tensor-core tile on it.
-template <typename T, int G, bool kDense, int KS, int VB, bool kQ8 = false>
+// kMode: kModeQ8, the latent pages hold per-token int8 codes and fp32
+// scales, and each consumer dequantises a page half by half into its own
+// bf16 buffer and runs the bf16 tensor-core tile on it; kModeVA, the pages
+// hold key codes and value residual slots (process_tile_va).
+template <typename T, int G, bool kDense, int KS, int VB, int kMode = kModePlain>
 __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   constexpr int CE = Elem<T>::CE;
   constexpr int NP = CE / 2;
@@ -924,7 +1114,7 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   const int w = warp - kFirstConsumer;
   const int nck = rsp == 0 ? a.rk / CE : kHeadDim / CE;  // (int8 pages: of the bf16 buffer)
   const int ncv = rsp == 0 ? a.rv / CE : kHeadDim / CE;
-  const int rvd = rsp == 0 ? a.rv : kHeadDim;
+  const int rvd = rsp == 0 ? a.rw : kHeadDim;
   const int qdim = rsp == 0 ? a.rk : kHeadDim;
   int TS = 1;
   while (TS * 2 * ncv <= 32) TS *= 2;
@@ -965,7 +1155,33 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
         for (int vb = 0; vb < VB; ++vb)
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[hl][vb][i] = 0.f;
-      if constexpr (kQ8 && !kDense) {
+      if constexpr (kMode == kModeVA && !kDense) {
+        // value-amortised pages: sum p c_k over the key codes and p e over
+        // the kept residuals; the merge applies the predictor
+        float* pw = reinterpret_cast<float*>(smem + sp_.dq + (size_t)w * a.dq_bytes);
+        float acck[2][KS][4], acce[VB][4];
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kb = 0; kb < KS; ++kb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acck[hl][kb][i] = 0.f;
+#pragma unroll
+        for (int vb = 0; vb < VB; ++vb)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acce[vb][i] = 0.f;
+        for (int tt = first; tt < ce; tt += kConsumers) {
+          const uint4* st = acquire(tt);
+          if (!st) break;
+          process_tile_va<KS, VB>(st, min(TT, ntok - (tt - ustart) * TT), nck, a.rv / 8, qf, m,
+                                  l, acck, acce, pw, lane);
+          release(tt);
+        }
+        write_record_va<G, KS, VB>(rec, a.rk, a.rv, m, l, acck, acce, lane);
+        t = ce;
+        if (*fail) break;
+        continue;
+      } else if constexpr (kMode == kModeQ8 && !kDense) {
         // int8 pages: each half of 32 tokens is dequantised into this warp's
         // buffer, then run on the tensor cores as a 32-token tile
         uint4* dq = reinterpret_cast<uint4*>(smem + sp_.dq + (size_t)w * a.dq_bytes);
@@ -1021,10 +1237,12 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
 // ------------------------------------------------------------ merge kernel
 // Shared-memory plan of the merge kernel (byte offsets from the base).
 struct MergePlan {
-  int pv, recb, wts, latf, frf, lf, starts, bars, total;
+  int pv, recb, wts, latf, frf, lf, starts, bars, am, uf, total;
 };
 __host__ __device__ inline int pv_row(int rv) { return rv + 4; }  // padded row of P_v
-__host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B) {
+// rk_va > 0: value-amortised records (key-code sums then residual sums, rw =
+// rk_va + rv per head) and the unit's predictor staged beside P_v.
+__host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B, int rk_va = 0) {
   MergePlan p;
   int off = 0;
   auto take = [&](int bytes, int align) {
@@ -1036,11 +1254,13 @@ __host__ __device__ inline MergePlan merge_plan(int rv, bool lat, int G, int B) 
   p.pv = take(lat ? kHeadDim * pv_row(rv) * 4 : 0, 16);
   p.recb = take(kMergeBuf, 128);
   p.wts = take(kMergeWarps * (kMergeMaxRec + 4) * 4, 16);
-  p.latf = take(G * (lat ? rv : 0) * 4, 16);
+  p.latf = take(G * (lat ? rv + rk_va : 0) * 4, 16);
   p.frf = take(G * kHeadDim * 4, 16);
   p.lf = take(G * 4, 16);
   p.starts = take(2 * (B + 1) * 4, 8);
   p.bars = take(8, 8);
+  p.am = take(lat ? rk_va * rv * 4 : 0, 16);
+  p.uf = take(lat && rk_va ? G * rv * 4 : 0, 16);
   p.total = off;
   return p;
 }
@@ -1084,7 +1304,8 @@ __device__ __forceinline__ float weighted_sum(const float* col, int S, const flo
 template <typename T, int G>
 __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const MergePlan mp = merge_plan(a.rv, a.codes != nullptr, G, a.B);
+  const int rk_va = a.A ? a.rk : 0;
+  const MergePlan mp = merge_plan(a.rv, a.codes != nullptr, G, a.B, rk_va);
   float* pv = reinterpret_cast<float*>(smem + mp.pv);      // [128][r_v + 4]
   float* recb = reinterpret_cast<float*>(smem + mp.recb);  // records of one chunk
   float* latf = reinterpret_cast<float*>(smem + mp.latf);  // [G][r_v]
@@ -1098,6 +1319,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
   const int unit = blockIdx.x, b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int rv = a.codes ? a.rv : 0, PR = pv_row(a.rv);
+  const int rw = a.codes ? a.rw : 0;  // latent record width per head
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_fence_init();
@@ -1110,6 +1332,11 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     for (int x = tid; x < kHeadDim * n4; x += kMergeThreads) {
       const int d = x / n4, j4 = x - d * n4;
       *reinterpret_cast<float4*>(pv + d * PR + 4 * j4) = ldg_f4_hint(P + x, pol);
+    }
+    if (rk_va) {  // the unit's value predictor A [rk][rv]
+      const float4* Ag = reinterpret_cast<const float4*>(a.A + (size_t)unit * rk_va * rv);
+      float4* am = reinterpret_cast<float4*>(smem + mp.am);
+      for (int x = tid; x < rk_va * rv / 4; x += kMergeThreads) am[x] = __ldg(Ag + x);
     }
   }
   // seq_len was final before the q-fold started (an ordinary launch).
@@ -1131,7 +1358,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     ncta[sp] = cta_of(us + tiles - 1, total[sp], Ce) - c0[sp] + 1;
   }
   const int per0 = kConsumers, per1 = anchors ? 1 : kConsumers;
-  const int S0 = H + G * a.rv, S1 = H + G * kHeadDim;  // floats per record
+  const int S0 = H + G * a.rw, S1 = H + G * kHeadDim;  // floats per record
   const int n0 = ncta[0] * per0, n1 = ncta[1] * per1;
   const float* src0 = a.part_lat + (size_t)(unit + c0[0]) * per0 * S0;
   const float* src1 = a.part_fr + (size_t)(unit + c0[1]) * per1 * S1;
@@ -1141,7 +1368,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
   // the full-rank sums; lane owns columns j0 + lane + 32 i and d0 + lane + 32 i
   constexpr int kParts = kMergeWarps / G;
   const int g = warp % G, part = warp / G;
-  const int jn = (rv + kParts - 1) / kParts, j0 = min(rv, part * jn), j1 = min(rv, j0 + jn);
+  const int jn = (rw + kParts - 1) / kParts, j0 = min(rw, part * jn), j1 = min(rw, j0 + jn);
   constexpr int dn = kHeadDim / kParts, kD = (dn + 31) / 32;
   const int d0 = part * dn;
   float* wts = reinterpret_cast<float*>(smem + mp.wts) + warp * (kMergeMaxRec + 4);
@@ -1223,7 +1450,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = j0 + lane + 32 * i;
-      if (j < j1) lat[i] = fmaf(lat[i], al, weighted_sum(recb + H + g * a.rv + j, S0, wts, nl));
+      if (j < j1) lat[i] = fmaf(lat[i], al, weighted_sum(recb + H + g * a.rw + j, S0, wts, nl));
     }
 #pragma unroll
     for (int i = 0; i < kD; ++i) {
@@ -1245,7 +1472,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = j0 + lane + 32 * i;
-      if (j < j1) latf[g * rv + j] = lat[i];
+      if (j < j1) latf[g * rw + j] = lat[i];
     }
 #pragma unroll
     for (int i = 0; i < kD; ++i)
@@ -1253,6 +1480,20 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     if (part == 0 && lane == 0) Lf[g] = L;
   }
   __syncthreads();
+  // value-amortised: u[g][n] = sum_k A[k][n] keysum[g][k] + ressum[g][n]
+  const float* uf = latf;
+  if (rk_va && rv) {
+    float* u = reinterpret_cast<float*>(smem + mp.uf);
+    const float* am = reinterpret_cast<const float*>(smem + mp.am);
+    for (int x = tid; x < G * rv; x += kMergeThreads) {
+      const int gg = x / rv, n = x - gg * rv;
+      float acc = latf[gg * rw + rk_va + n];
+      for (int k = 0; k < rk_va; ++k) acc = fmaf(am[k * rv + n], latf[gg * rw + k], acc);
+      u[x] = acc;
+    }
+    __syncthreads();
+    uf = u;
+  }
   // o[g][d] = (sum_j P_v[d][j] lat[g][j] + fr[g][d]) / L_g: thread -> row d
   // and heads [h0, h0 + kHT)
   constexpr int kHT = (G * kHeadDim + kMergeThreads - 1) / kMergeThreads;
@@ -1267,7 +1508,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
 #pragma unroll
       for (int h = 0; h < kHT; ++h) {
         if (h0 + h < G) {
-          const float4 l4 = *reinterpret_cast<const float4*>(latf + (h0 + h) * rv + j);
+          const float4 l4 = *reinterpret_cast<const float4*>(uf + (h0 + h) * rv + j);
           out[h] = fmaf(p4.x, l4.x, fmaf(p4.y, l4.y, fmaf(p4.z, l4.z, fmaf(p4.w, l4.w, out[h]))));
         }
       }
@@ -1285,12 +1526,13 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
 
 // ------------------------------------------------------------ host side
 struct Plan {
-  int C, NS, stage_bytes, dq_bytes, smem, merge_smem;
+  int C, NS, stage_bytes, dq_bytes, rw, smem, merge_smem;
   size_t off_qlat, off_qfr, off_lat, off_fr, total;
 };
 
+// mode: kModePlain, kModeQ8 (int8 codes) or kModeVA (value-amortised slabs).
 static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, bool has_fr,
-                       bool anchors, int esize, Plan& p, bool q8 = false) {
+                       bool anchors, int esize, Plan& p, int mode = kModePlain) {
   int dev = 0;
   DevInfo info;
   const int rc = current_device_info(dev, info);
@@ -1300,10 +1542,17 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   // the ring holds latent pages, or dense full-rank pages (no latent space)
   p.stage_bytes = has_lat ? kLatPage * (rk + rv) * esize : 2 * kFrTile * kHeadDim * esize;
   p.dq_bytes = 0;
-  if (has_lat && q8) {  // int8 codes + scales; a bf16 half page per consumer
+  int rw = rv;          // latent record width per head
+  if (has_lat && mode == kModeQ8) {  // int8 codes + scales; a bf16 half page per consumer
     p.stage_bytes = kLatPage * (rk + rv) + 512;
     p.dq_bytes = kFrTile * (rk + rv) * 2;
   }
+  if (has_lat && mode == kModeVA) {  // key codes + residual slots; page weights per consumer
+    p.stage_bytes = va_slab_bytes(rk, rv);
+    p.dq_bytes = kLatPage * 8 * 4;
+    rw = rk + rv;
+  }
+  p.rw = rw;
   // Leave room for a q-fold CTA beside each split CTA.
   const int budget = optin - 8 * 1024;
   const bool tc = esize == 2;  // bf16: tensor-core consumers
@@ -1312,7 +1561,7 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   if (p.NS < 2) return LRKV_ERR_UNSUPPORTED;
   p.smem = smem_plan(p.NS, p.stage_bytes, B, G, tc, p.dq_bytes).total;
   p.C = sms;
-  p.merge_smem = merge_plan(rv, has_lat, G, B).total;
+  p.merge_smem = merge_plan(rv, has_lat, G, B, mode == kModeVA ? rk : 0).total;
   const int U = B * H_kv;
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   size_t off = 256;
@@ -1320,7 +1569,7 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   p.off_qfr = off;  off = al(off + (size_t)B * H_q * (has_fr ? kHeadDim : 0) * 4);
   const size_t slots = (size_t)(U + p.C - 1);
   p.off_lat = off;
-  off = al(off + (has_lat ? slots * kConsumers * (hdr_floats(G) + G * rv) * 4 : 0));
+  off = al(off + (has_lat ? slots * kConsumers * (hdr_floats(G) + G * rw) * 4 : 0));
   p.off_fr = off;
   off = al(off + (has_fr ? slots * (anchors ? 1 : kConsumers) * (hdr_floats(G) + G * kHeadDim) * 4
                          : 0));
@@ -1328,11 +1577,15 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   return LRKV_OK;
 }
 
+static int mode_of(int dtype) {
+  return dtype == LRKV_BF16_Q8 ? kModeQ8 : (dtype == LRKV_BF16_VA ? kModeVA : kModePlain);
+}
+
 int decode_plan_check(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, bool has_fr,
                       int dtype) {
   Plan p;
   return plan_decode(B, H_kv, H_q, rk, rv, has_lat, has_fr, has_lat && has_fr,
-                     dtype == LRKV_F32 ? 4 : 2, p, dtype == LRKV_BF16_Q8);
+                     dtype == LRKV_F32 ? 4 : 2, p, mode_of(dtype));
 }
 
 size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has_lat,
@@ -1340,7 +1593,7 @@ size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has
   Plan p;
   // anchors: full-rank space present next to a latent one (no block table)
   if (plan_decode(B, H_kv, H_q, rk, rv, has_lat, has_fr, has_lat && has_fr,
-                  dtype == LRKV_F32 ? 4 : 2, p, dtype == LRKV_BF16_Q8) != LRKV_OK)
+                  dtype == LRKV_F32 ? 4 : 2, p, mode_of(dtype)) != LRKV_OK)
     return 0;
   return p.total;
 }
@@ -1366,9 +1619,13 @@ template <typename T, int G>
 static const void* split_fn(const DecodeArgs& a) {
   if (!a.codes) return (const void*)split_kernel<T, G, true, 8, 8>;
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (a.A) {  // value-amortised slabs
+      if (a.rk <= 64 && a.rv <= 32) return (const void*)split_kernel<T, G, false, 4, 2, kModeVA>;
+      return (const void*)split_kernel<T, G, false, 8, 8, kModeVA>;
+    }
     if (a.dq_bytes) {  // int8 codes
-      if (a.rk <= 64 && a.rv <= 32) return (const void*)split_kernel<T, G, false, 4, 2, true>;
-      return (const void*)split_kernel<T, G, false, 8, 8, true>;
+      if (a.rk <= 64 && a.rv <= 32) return (const void*)split_kernel<T, G, false, 4, 2, kModeQ8>;
+      return (const void*)split_kernel<T, G, false, 8, 8, kModeQ8>;
     }
     if (a.rk <= 64 && a.rv <= 32) return (const void*)split_kernel<T, G, false, 4, 2>;
   }
@@ -1412,7 +1669,7 @@ int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
   const int es = L.dtype == LRKV_F32 ? 4 : 2;
   Plan p;
   int rc = plan_decode(L.B, L.H_kv, L.H_q, L.rk, L.rv, has_lat, has_fr,
-                       anchor_mode(L.fr, L.bt_fr), es, p, L.dtype == LRKV_BF16_Q8);
+                       anchor_mode(L.fr, L.bt_fr), es, p, mode_of(L.dtype));
   if (rc != LRKV_OK) return rc;
   if (L.ws_bytes < p.total) return LRKV_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(L.ws);
@@ -1431,6 +1688,8 @@ int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
   a.part_lat = reinterpret_cast<float*>(ws + p.off_lat);
   a.part_fr = reinterpret_cast<float*>(ws + p.off_fr);
   a.C = p.C; a.NS = p.NS; a.stage_bytes = p.stage_bytes; a.dq_bytes = p.dq_bytes;
+  a.rw = p.rw;
+  a.A = L.dtype == LRKV_BF16_VA ? L.A : nullptr;
   if (L.dtype == LRKV_F32) return launch_decode_g<float>(a, p, st);
   return launch_decode_g<__nv_bfloat16>(a, p, st);
 }

@@ -36,6 +36,7 @@ struct DecodeLaunch {
   void* o;
   void* ws;
   size_t ws_bytes;
+  const float* A = nullptr;  // value predictors of a value-amortised cache
 };
 
 size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has_lat,
@@ -49,7 +50,8 @@ int decode_launch(const DecodeLaunch& L, cudaStream_t st);
 
 int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, const int* n_new,
                     long long seq_stride, long long head_stride, const float* P_k,
-                    const float* P_v, long long basis_bs, cudaStream_t st);
+                    const float* P_v, long long basis_bs, cudaStream_t st,
+                    const float* A = nullptr);
 int dense_append_launch(const lrkv_dense_cache& c, const void* k, const void* v, int n,
                         const int* n_new,
                         long long seq_stride, long long head_stride, cudaStream_t st);

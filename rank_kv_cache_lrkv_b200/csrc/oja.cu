@@ -488,6 +488,342 @@ __global__ void __launch_bounds__(kOjaThreads) oja_blocked_kernel(
   for (int e = tid; e < kHeadDim * r; e += kOjaThreads) Pg[e] = Ps[(e / r) * ldp + e % r];
 }
 
+// ---- chunked Oja on the tensor cores (bf16 token rows)
+// One CTA of 256 threads (8 warps) per stream, r <= 64.  Per chunk of
+// nc <= 64 tokens, three warp-level bf16 MMA products (m16n8k16, fp32
+// accumulation) with every fp32 operand split into hi + lo bf16 halves (the
+// lo x lo term dropped), so each product keeps about 16 mantissa bits:
+//   Y = X P          warp -> m-block w % 4 (16 tokens), half the columns
+//   Z = X - Y P^T    warp -> m-block w % 4, half of the 128 dims
+//   P += eta Z^T Y   warp -> dims 16 w .. 16 w + 15, every column
+// X is exact in bf16.  P is kept in fp32 (the master the update and the QR
+// work on) and as hi/lo bf16 rows [128][ldp] that serve as the B operand of
+// the first product (ldmatrix.trans) and of the second (ldmatrix); Y and Z
+// are kept as hi/lo bf16 only.  Row strides are odd multiples of 16 bytes
+// (ldmatrix without bank conflicts).  Rows of the next chunk arrive by
+// cp.async (rows past the chunk zero-filled) while the current one runs.
+constexpr int kMmaOjaThreads = 256;
+constexpr int kLdX = kHeadDim + 8;  // bf16 row stride of X and Z (272 bytes)
+
+__host__ __device__ inline int oja_ld16(int r) { return (r / 8) % 2 == 0 ? r + 8 : r + 16; }
+
+struct OjaMmaPlan {
+  int pf, ph, pl, x, yh, yl, zh, zl, col, h, red, total;
+};
+__host__ __device__ inline OjaMmaPlan oja_mma_plan(int r) {
+  OjaMmaPlan p;
+  int off = 0;
+  auto take = [&](int bytes) {
+    off = (off + 15) / 16 * 16;
+    const int at = off;
+    off += bytes;
+    return at;
+  };
+  const int ldp = oja_ld16(r);
+  p.pf = take(kHeadDim * (r + 1) * 4);          // fp32 master [128][r + 1]
+  p.ph = take(kHeadDim * ldp * 2);              // [128][ldp] bf16
+  p.pl = take(kHeadDim * ldp * 2);
+  p.x = take(2 * kBlkRows * kLdX * 2);          // [2][64][kLdX] bf16
+  p.yh = take(kBlkRows * ldp * 2);              // [64][ldp]
+  p.yl = take(kBlkRows * ldp * 2);
+  p.zh = take(kBlkRows * kLdX * 2);             // [64][kLdX]
+  p.zl = take(kBlkRows * kLdX * 2);
+  p.col = take(kHeadDim * 4);
+  p.h = take(kHeadDim * 4);
+  p.red = take(8 * 4);
+  p.total = off;
+  return p;
+}
+
+// Q of QR(P), diag(R) > 0, on the fp32 tile [128][ld] with 256 threads
+// (threads < 128 own a row each; the others join the barriers).
+__device__ void qr_rows256(float* P, int r, int ld, float* col, float* h, float* red) {
+  const int i = threadIdx.x, lane = i & 31, w = i >> 5;
+  for (int j = 0; j < r; ++j) {
+    if (i < kHeadDim) col[i] = P[i * ld + j];
+    __syncthreads();
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int k = i; k < j; k += kMmaOjaThreads) {
+        float s0 = 0.f, s1 = 0.f;
+        for (int ii = 0; ii < kHeadDim; ii += 2) {
+          s0 = fmaf(P[ii * ld + k], col[ii], s0);
+          s1 = fmaf(P[(ii + 1) * ld + k], col[ii + 1], s1);
+        }
+        h[k] = s0 + s1;
+      }
+      __syncthreads();
+      float c = i < kHeadDim ? col[i] : 0.f;
+      if (i < kHeadDim)
+        for (int k = 0; k < j; ++k) c = fmaf(-h[k], P[i * ld + k], c);
+      __syncthreads();
+      if (i < kHeadDim) col[i] = c;
+      __syncthreads();
+    }
+    const float c = i < kHeadDim ? col[i] : 0.f;
+    const float ss = warp_sum(c * c);
+    if (lane == 0) red[w] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMmaOjaThreads / 32; ++k) tot += red[k];
+    if (i < kHeadDim) P[i * ld + j] = c / sqrtf(tot);
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kMmaOjaThreads, 1) oja_chunked_mma(
+    float* P, int r, long long bstride, const __nv_bfloat16* __restrict__ x, long long xstride,
+    int n, float eta, int qr_every, long long seen, int chunk) {
+  using bf16 = __nv_bfloat16;
+  extern __shared__ __align__(16) uint8_t osm[];
+  const OjaMmaPlan pl = oja_mma_plan(r);
+  const int ldp = oja_ld16(r), ldf = r + 1;
+  float* Pf = reinterpret_cast<float*>(osm + pl.pf);
+  bf16* Ph = reinterpret_cast<bf16*>(osm + pl.ph);
+  bf16* Pl = reinterpret_cast<bf16*>(osm + pl.pl);
+  bf16* Xs = reinterpret_cast<bf16*>(osm + pl.x);
+  bf16* Yh = reinterpret_cast<bf16*>(osm + pl.yh);
+  bf16* Yl = reinterpret_cast<bf16*>(osm + pl.yl);
+  bf16* Zh = reinterpret_cast<bf16*>(osm + pl.zh);
+  bf16* Zl = reinterpret_cast<bf16*>(osm + pl.zl);
+  float* col = reinterpret_cast<float*>(osm + pl.col);
+  float* hq = reinterpret_cast<float*>(osm + pl.h);
+  float* red = reinterpret_cast<float*>(osm + pl.red);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  float* Pg = P + (size_t)blockIdx.x * bstride;
+  const bf16* xg = x + (size_t)blockIdx.x * xstride;
+  const int NB = (r + 7) / 8, KSr = (r + 15) / 16;  // n-blocks of the columns, k-steps over r
+
+  // the fp32 master and its hi/lo rows (padding columns zero)
+  for (int e = tid; e < kHeadDim * ldp; e += kMmaOjaThreads) {
+    const int i = e / ldp, j = e - i * ldp;
+    const float v = j < r ? Pg[(size_t)i * r + j] : 0.f;
+    if (j < r) Pf[i * ldf + j] = v;
+    const bf16 hh = __float2bfloat16_rn(v);
+    Ph[e] = hh;
+    Pl[e] = __float2bfloat16_rn(v - __bfloat162float(hh));
+  }
+  for (int e = tid; e < kBlkRows * ldp; e += kMmaOjaThreads) {  // Y padding stays zero
+    Yh[e] = __float2bfloat16_rn(0.f);
+    Yl[e] = __float2bfloat16_rn(0.f);
+  }
+  auto refresh_rows = [&](int i0, int i1) {  // hi/lo rows from the master
+    for (int e = i0 * r + tid; e < i1 * r; e += kMmaOjaThreads) {
+      const int i = e / r, j = e - i * r;
+      const float v = Pf[i * ldf + j];
+      const bf16 hh = __float2bfloat16_rn(v);
+      Ph[i * ldp + j] = hh;
+      Pl[i * ldp + j] = __float2bfloat16_rn(v - __bfloat162float(hh));
+    }
+  };
+  auto chunk_len = [&](int j) {
+    int nc = min(min(chunk, kBlkRows), n - j);
+    if (qr_every > 0) {
+      const long long to_qr = qr_every - (seen + j) % qr_every;
+      if (to_qr < nc) nc = (int)to_qr;
+    }
+    return nc;
+  };
+  auto stage = [&](int j, int buf) {  // rows of the chunk at j; the rest zero-filled
+    const int nc = chunk_len(j);
+    bf16* dst = Xs + (size_t)buf * kBlkRows * kLdX;
+    for (int e = tid; e < kBlkRows * (kHeadDim / 8); e += kMmaOjaThreads) {
+      const int t = e >> 4, c = e & 15;
+      const bool ok = t < nc;
+      cp_async16(dst + t * kLdX + c * 8, xg + (size_t)(ok ? j + t : j) * kHeadDim + c * 8,
+                 ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  if (n > 0) stage(0, 0);
+  int buf = 0;
+  const int arow = lane & 15, ahalf = lane >> 4;                     // A, ldmatrix
+  const int brow = (lane & 7) + ((lane >> 4) << 3), bk = ((lane >> 3) & 1) * 8;  // B, ldmatrix
+  const int trow = (lane & 7) + ((lane >> 3) & 1) * 8, tcol = (lane >> 4) * 8;   // B, .trans
+  const int atrow = (lane & 7) + ((lane >> 4) << 3), atcol = ((lane >> 3) & 1) * 8;  // A, .trans
+  for (int j = 0; j < n;) {
+    const int nc = chunk_len(j);
+    cp_async_wait<0>();
+    __syncthreads();  // X of this chunk landed; the previous chunk's products are done
+    if (j + nc < n) stage(j + nc, buf ^ 1);
+    const bf16* X = Xs + (size_t)buf * kBlkRows * kLdX;
+    const uint32_t xb = smem_u32(X);
+    // ---- Y = X P : warp -> tokens 16 (w % 4) .., n-block pairs of its half
+    {
+      const int mb = warp & 3, half = warp >> 2, NP = (NB + 1) / 2;
+      const int p0 = half ? (NP + 1) / 2 : 0, p1 = half ? NP : (NP + 1) / 2;
+      float acc[4][2][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q][u][e] = 0.f;
+#pragma unroll 2
+      for (int ks = 0; ks < kHeadDim / 16; ++ks) {
+        uint32_t a[4];
+        ldsm_x4(xb + (uint32_t)(((mb * 16 + arow) * kLdX + ks * 16 + ahalf * 8) * 2), a);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int pr = p0 + q;
+          if (pr < p1) {
+            // B[k = dim][n = column] = P[dim][column]: rows k, so .trans
+            const uint32_t off =
+                (uint32_t)(((ks * 16 + trow) * ldp + pr * 16 + tcol) * 2);
+            uint32_t bh[4], bl[4];
+            ldsm_x4_trans(smem_u32(Ph) + off, bh);
+            ldsm_x4_trans(smem_u32(Pl) + off, bl);
+            mma_bf16_16816(acc[q][0], a, bh[0], bh[1]);
+            mma_bf16_16816(acc[q][1], a, bh[2], bh[3]);
+            mma_bf16_16816(acc[q][0], a, bl[0], bl[1]);
+            mma_bf16_16816(acc[q][1], a, bl[2], bl[3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int pr = p0 + q;
+        if (pr < p1) {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col0 = (2 * pr + u) * 8 + 2 * t4;
+            if (col0 < r) {
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int row = mb * 16 + g + 8 * h2;
+                const float y0 = acc[q][u][2 * h2], y1 = acc[q][u][2 * h2 + 1];
+                const uint32_t hh = pack_bf16x2(y0, y1);
+                *reinterpret_cast<uint32_t*>(Yh + row * ldp + col0) = hh;
+                *reinterpret_cast<uint32_t*>(Yl + row * ldp + col0) =
+                    pack_bf16x2(y0 - bf_lo(hh), y1 - bf_hi(hh));
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // ---- Z = X - Y P^T : warp -> tokens 16 (w % 4) .., dims 64 (w / 4) ..
+    {
+      const int mb = warp & 3, d0 = (warp >> 2) * 64;
+      float acc[4][2][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q][u][e] = 0.f;
+      for (int ks = 0; ks < KSr; ++ks) {
+        uint32_t ah[4], al[4];
+        const uint32_t aoff = (uint32_t)(((mb * 16 + arow) * ldp + ks * 16 + ahalf * 8) * 2);
+        ldsm_x4(smem_u32(Yh) + aoff, ah);
+        ldsm_x4(smem_u32(Yl) + aoff, al);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // B[k = column][n = dim] = P[dim][column]: rows n
+          const uint32_t off = (uint32_t)(((d0 + q * 16 + brow) * ldp + ks * 16 + bk) * 2);
+          uint32_t bh[4], bl[4];
+          ldsm_x4(smem_u32(Ph) + off, bh);
+          ldsm_x4(smem_u32(Pl) + off, bl);
+          mma_bf16_16816(acc[q][0], ah, bh[0], bh[1]);
+          mma_bf16_16816(acc[q][1], ah, bh[2], bh[3]);
+          mma_bf16_16816(acc[q][0], ah, bl[0], bl[1]);
+          mma_bf16_16816(acc[q][1], ah, bl[2], bl[3]);
+          mma_bf16_16816(acc[q][0], al, bh[0], bh[1]);
+          mma_bf16_16816(acc[q][1], al, bh[2], bh[3]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int row = mb * 16 + g + 8 * h2, d = d0 + q * 16 + u * 8 + 2 * t4;
+            const uint32_t xv = *reinterpret_cast<const uint32_t*>(X + row * kLdX + d);
+            const float z0 = bf_lo(xv) - acc[q][u][2 * h2], z1 = bf_hi(xv) - acc[q][u][2 * h2 + 1];
+            const uint32_t hh = pack_bf16x2(z0, z1);
+            *reinterpret_cast<uint32_t*>(Zh + row * kLdX + d) = hh;
+            *reinterpret_cast<uint32_t*>(Zl + row * kLdX + d) =
+                pack_bf16x2(z0 - bf_lo(hh), z1 - bf_hi(hh));
+          }
+    }
+    __syncthreads();
+    // ---- P += eta Z^T Y : warp -> dims 16 w .., every column
+    {
+      const int i0 = warp * 16;
+      float acc[4][2][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q][u][e] = 0.f;
+      const int NP = (NB + 1) / 2;
+#pragma unroll
+      for (int ks = 0; ks < kBlkRows / 16; ++ks) {
+        if (ks * 16 < nc) {
+          // A[m = dim][k = token] = Z[token][dim]: rows k, so .trans
+          const uint32_t aoff = (uint32_t)(((ks * 16 + atrow) * kLdX + i0 + atcol) * 2);
+          uint32_t ah[4], al[4];
+          ldsm_x4_trans(smem_u32(Zh) + aoff, ah);
+          ldsm_x4_trans(smem_u32(Zl) + aoff, al);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q < NP) {
+              // B[k = token][n = column] = Y[token][column]: rows k, so .trans
+              const uint32_t off = (uint32_t)(((ks * 16 + trow) * ldp + q * 16 + tcol) * 2);
+              uint32_t bh[4], bl[4];
+              ldsm_x4_trans(smem_u32(Yh) + off, bh);
+              ldsm_x4_trans(smem_u32(Yl) + off, bl);
+              mma_bf16_16816(acc[q][0], ah, bh[0], bh[1]);
+              mma_bf16_16816(acc[q][1], ah, bh[2], bh[3]);
+              mma_bf16_16816(acc[q][0], ah, bl[0], bl[1]);
+              mma_bf16_16816(acc[q][1], ah, bl[2], bl[3]);
+              mma_bf16_16816(acc[q][0], al, bh[0], bh[1]);
+              mma_bf16_16816(acc[q][1], al, bh[2], bh[3]);
+            }
+          }
+        }
+      }
+      // the warp owns rows i0 .. i0 + 15 of P: master and hi/lo updated here
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c0 = (2 * q + u) * 8 + 2 * t4;
+          if (q < NP && c0 < r) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int i = i0 + g + 8 * h2;
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                if (c0 + e < r) {
+                  float& pp = Pf[i * ldf + c0 + e];
+                  pp = fmaf(eta, acc[q][u][2 * h2 + e], pp);
+                  const bf16 hh = __float2bfloat16_rn(pp);
+                  Ph[i * ldp + c0 + e] = hh;
+                  Pl[i * ldp + c0 + e] = __float2bfloat16_rn(pp - __bfloat162float(hh));
+                }
+              }
+            }
+          }
+        }
+    }
+    j += nc;
+    buf ^= 1;
+    if (qr_every > 0 && (seen + j) % qr_every == 0) {
+      __syncthreads();
+      qr_rows256(Pf, r, ldf, col, hq, red);
+      refresh_rows(0, kHeadDim);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int e = tid; e < kHeadDim * r; e += kMmaOjaThreads) Pg[e] = Pf[(e / r) * ldf + e % r];
+}
+
 int oja_blocked_launch(float* P, int S, int r, long long basis_stride, const void* x,
                        int x_dtype, long long x_stride, int n, float eta, int qr_every,
                        long long tokens_seen, int chunk, cudaStream_t st) {
@@ -496,6 +832,14 @@ int oja_blocked_launch(float* P, int S, int r, long long basis_stride, const voi
   if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0 || (x_stride * es) % 16 != 0)
     return LRKV_ERR_ARG;
   if (r > 64 || r % 8 != 0) return LRKV_ERR_UNSUPPORTED;
+  if (x_dtype == LRKV_BF16) {  // token rows exact in bf16: the tensor-core kernel
+    const int rc = prepare_kernel((const void*)oja_chunked_mma, false);
+    if (rc != LRKV_OK) return rc;
+    oja_chunked_mma<<<S, kMmaOjaThreads, oja_mma_plan(r).total, st>>>(
+        P, r, basis_stride, static_cast<const __nv_bfloat16*>(x), x_stride, n, eta, qr_every,
+        tokens_seen, chunk);
+    return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+  }
   const size_t sm = oja_blocked_smem_bytes(r, es);
   const void* fn = x_dtype == LRKV_BF16 ? (const void*)oja_blocked_kernel<__nv_bfloat16>
                                         : (const void*)oja_blocked_kernel<float>;

@@ -17,7 +17,8 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblrkv.so")
 
-LRKV_BF16, LRKV_F32, LRKV_BF16_Q8 = 0, 1, 2
+LRKV_BF16, LRKV_F32, LRKV_BF16_Q8, LRKV_BF16_VA = 0, 1, 2, 3
+VA_KEEP = 16
 HEAD_DIM = 128
 PAGE_TOKENS = 64
 FULL_RANK_TILE = 32
@@ -56,7 +57,9 @@ EXPORTS = ["lrkv_compress", "lrkv_decode_workspace_bytes", "lrkv_decode_attn",
            "lrkv_oja_update", "lrkv_qr_orthonormalize", "lrkv_dense_append",
            "lrkv_dense_decode_workspace_bytes", "lrkv_dense_decode_attn",
            "lrkv_status_string", "lrkv_version", "lrkv_decode_attn_static",
-           "lrkv_rebase_workspace_bytes", "lrkv_rebase", "lrkv_oja_update_chunked"]
+           "lrkv_rebase_workspace_bytes", "lrkv_rebase", "lrkv_oja_update_chunked",
+           "lrkv_compress_amortised", "lrkv_amortise_workspace_bytes", "lrkv_amortise",
+           "lrkv_decode_attn_amortised"]
 
 
 def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
@@ -80,6 +83,11 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "lrkv_decode_attn_static": (ctypes.c_int, [P, P, I32, P, P, I64, F32, P, P]),
         "lrkv_rebase_workspace_bytes": (SZ, [P]),
         "lrkv_rebase": (ctypes.c_int, [P, P, P, P, P, I64, P, SZ, P]),
+        "lrkv_compress_amortised": (ctypes.c_int, [P, P, P, I32, P, I64, I64, P, P, I64, P, P]),
+        "lrkv_amortise_workspace_bytes": (SZ, [P]),
+        "lrkv_amortise": (ctypes.c_int, [P, P, I32, I64, I64, P, I64, P, P, SZ, P]),
+        "lrkv_decode_attn_amortised": (ctypes.c_int,
+                                       [P, P, I32, P, P, I64, P, F32, P, P, SZ, P]),
         "lrkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "lrkv_version": (ctypes.c_int, []),
     }
@@ -129,7 +137,7 @@ class LatentCache:
     def __init__(self, B: int, H_kv: int, r_k: int, r_v: int, max_tokens: int,
                  n_sink: int = 0, window: int = 0, dtype=torch.bfloat16,
                  device="cuda", page_perm: Optional[torch.Tensor] = None,
-                 int8_codes: bool = False):
+                 int8_codes: bool = False, amortised_values: bool = False):
         ce = chunk_elems(dtype)
         self.B, self.H_kv, self.r_k, self.r_v = B, H_kv, r_k, r_v
         self.n_sink, self.window, self.dtype = n_sink, window, dtype
@@ -137,7 +145,16 @@ class LatentCache:
         max_lat = max(1, max_tokens - n_sink - window)
         self.max_pages = math.ceil(max_lat / PAGE_TOKENS)
         self.num_pages = B * self.max_pages
-        if int8_codes:
+        self.amortised_values = amortised_values
+        if amortised_values:
+            # one slab per (page, kv head): key-code chunks, then the value
+            # residual slots [r_v / 8][16][8] bf16, slot rows int32 [16] and
+            # squared norms fp32 [16]
+            assert dtype == torch.bfloat16 and not int8_codes
+            self.codes = torch.zeros((self.num_pages, H_kv,
+                                      PAGE_TOKENS * r_k * 2 + VA_KEEP * r_v * 2 + VA_KEEP * 8),
+                                     dtype=torch.uint8, device=device)
+        elif int8_codes:
             # one slab per (page, kv head): int8 code chunks of 16, key codes
             # then value codes, then [64][2] fp32 scales (bf16 inputs)
             assert dtype == torch.bfloat16
@@ -156,7 +173,8 @@ class LatentCache:
                                    dtype=dtype, device=device)
         self.seq_len = torch.zeros(B, dtype=torch.int32, device=device)
         self.append_counter = torch.zeros(B, dtype=torch.int32, device=device)
-        code = LRKV_BF16_Q8 if int8_codes else _dtype_code(dtype)
+        code = LRKV_BF16_Q8 if int8_codes else (LRKV_BF16_VA if amortised_values
+                                                 else _dtype_code(dtype))
         self.desc = CacheDesc(B, H_kv, HEAD_DIM, r_k, r_v, code, n_sink, window,
                               self.num_pages, self.max_pages, self.codes.data_ptr(),
                               self.block_table.data_ptr(), self.anchors.data_ptr(),
@@ -185,6 +203,51 @@ def compress(cache: LatentCache, k: torch.Tensor, v: torch.Tensor, P_k: torch.Te
         ctypes.byref(cache.desc), _ptr(k), _ptr(v), k.shape[2], _ptr(n_new), ss, hs, _ptr(P_k),
         _ptr(P_v),
         basis_batch_stride, _stream(stream)))
+
+
+def compress_amortised(cache: LatentCache, k: torch.Tensor, v: torch.Tensor,
+                       P_k: torch.Tensor, P_v: torch.Tensor, A: torch.Tensor,
+                       basis_batch_stride: int = 0, n_new: Optional[torch.Tensor] = None,
+                       stream=None) -> None:
+    """lrkv_compress_amortised: append to a value-amortised cache whose
+    predictors A [B, H_kv, r_k, r_v] exist."""
+    assert k.dtype == cache.dtype and v.dtype == cache.dtype and k.shape == v.shape
+    assert A.dtype == torch.float32 and A.is_contiguous()
+    ss, hs = _kv_strides(k)
+    assert _kv_strides(v) == (ss, hs)
+    _check("lrkv_compress_amortised", _lib.lrkv_compress_amortised(
+        ctypes.byref(cache.desc), _ptr(k), _ptr(v), k.shape[2], _ptr(n_new), ss, hs, _ptr(P_k),
+        _ptr(P_v), basis_batch_stride, _ptr(A), _stream(stream)))
+
+
+def amortise(cache: LatentCache, v: torch.Tensor, P_v: torch.Tensor, A: torch.Tensor,
+             basis_batch_stride: int = 0, stream=None) -> None:
+    """lrkv_amortise: fit the value predictors A [B, H_kv, r_k, r_v] (fp32,
+    written) over the prompt v [B, H_kv, n, 128] and fill the prompt pages'
+    residual slots."""
+    assert v.dtype == torch.bfloat16 and A.dtype == torch.float32 and A.is_contiguous()
+    ss, hs = _kv_strides(v)
+    n = int(_lib.lrkv_amortise_workspace_bytes(ctypes.byref(cache.desc)))
+    if n == 0:
+        raise LrkvError("lrkv_amortise_workspace_bytes", -2)
+    ws = torch.zeros(n, dtype=torch.uint8, device=v.device)
+    _check("lrkv_amortise", _lib.lrkv_amortise(
+        ctypes.byref(cache.desc), _ptr(v), v.shape[2], ss, hs, _ptr(P_v), basis_batch_stride,
+        _ptr(A), _ptr(ws), n, _stream(stream)))
+    cache._amortise_ws = ws  # kept alive until the stream has used it
+
+
+def decode_attn_amortised(cache: LatentCache, q: torch.Tensor, P_k: torch.Tensor,
+                          P_v: torch.Tensor, A: torch.Tensor, scale: float, o: torch.Tensor,
+                          workspace: torch.Tensor, basis_batch_stride: int = 0,
+                          stream=None) -> torch.Tensor:
+    """lrkv_decode_attn_amortised: o [B, H_q, 128] from q over a
+    value-amortised cache with predictors A."""
+    assert q.is_contiguous() and o.is_contiguous() and q.dtype == cache.dtype
+    _check("lrkv_decode_attn_amortised", _lib.lrkv_decode_attn_amortised(
+        ctypes.byref(cache.desc), _ptr(q), q.shape[1], _ptr(P_k), _ptr(P_v), basis_batch_stride,
+        _ptr(A), float(scale), _ptr(o), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o
 
 
 def decode_workspace_bytes(cache: LatentCache, num_q_heads: int) -> int:
