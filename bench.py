@@ -629,10 +629,14 @@ def run_ours(args, rank, world):
     ws = lrkv.decode_workspace(cache, wl.H_q, device=dev)
     o = torch.empty_like(qs[0])
 
-    def step(s):
+    def step(s, fused=False):
         t = wl.T + s
-        lrkv.compress(cache, Kd[:, :, t:t + 1], Vd[:, :, t:t + 1], Pk, Pv)
-        lrkv.decode_attn(cache, qs[s], Pk, Pv, wl.scale, o, ws)
+        if fused:  # lrkv_decode_step: append + query fold, split-K, merge
+            lrkv.decode_step(cache, Kd[:, :, t:t + 1], Vd[:, :, t:t + 1], qs[s], Pk, Pv,
+                             wl.scale, o, ws)
+        else:      # two calls: append; q-fold, split-K, merge
+            lrkv.compress(cache, Kd[:, :, t:t + 1], Vd[:, :, t:t + 1], Pk, Pv)
+            lrkv.decode_attn(cache, qs[s], Pk, Pv, wl.scale, o, ws)
 
     if args.profile:
         for s in range(min(args.profile, wl.n_decode)):
@@ -685,6 +689,24 @@ def run_ours(args, rank, world):
     if world > 1:
         dist.barrier()
     assert lrkv.workspace_error(ws) == 0
+    # the same steps through lrkv_decode_step, for comparison
+    g1 = torch.cuda.CUDAGraph()
+    cache.seq_len.copy_(saved_len)
+    with torch.cuda.graph(g1, capture_error_mode="relaxed"):
+        for s in range(W, W + K):
+            step(s, fused=True)
+    cache.seq_len.copy_(saved_len)
+    g1.replay()
+    torch.cuda.synchronize()
+    cache.seq_len.copy_(saved_len)
+    torch.cuda.synchronize()
+    with clk.region():
+        e0.record()
+        g1.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    ms_two = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    del g1
 
     # roofline of lrkv_decode_attn alone: the same call replayed (state fixed)
     R = 200
@@ -741,8 +763,15 @@ def run_ours(args, rank, world):
         "ms_per_step": round(ms / K, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": dict(config_of(wl), parallelism=f"replicas{world}"),
+        "config": dict(config_of(wl), parallelism=f"replicas{world}",
+                       step="lrkv_compress then lrkv_decode_attn (append; q-fold, split-K, "
+                            "merge)"),
         "gpu_launches": 4 * K,
+        "decode_step_call": {"ms_per_step": round(ms_two / K, 5),
+                             "tokens_per_s": round(replicas.aggregate_tokens_per_s(
+                                 wl.B, K, world, ms_two), 2),
+                             "note": "the same steps through lrkv_decode_step (3 launches: "
+                                     "append + query fold, split-K, merge); e2e uses this call"},
         "roofline": {"kernel": "lrkv_decode_attn (qfold + split + merge)", "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "frac_of_8TBs": round(achieved / 8000, 4),
@@ -821,8 +850,7 @@ def run_ours(args, rank, world):
             e0.record()
             for s in range(E):
                 dev_in.copy_(host_in[s], non_blocking=True)
-                lrkv.compress(cache, kd, vd, Pk, Pv)
-                lrkv.decode_attn(cache, qd, Pk, Pv, wl.scale, o, ws)
+                lrkv.decode_step(cache, kd, vd, qd, Pk, Pv, wl.scale, o, ws)
                 oh[s].copy_(o, non_blocking=True)
             e1.record()
             torch.cuda.synchronize()

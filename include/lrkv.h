@@ -211,6 +211,24 @@ int lrkv_decode_attn(const lrkv_cache *cache, const void *q, int32_t num_q_heads
                      int64_t basis_batch_stride, float scale, void *o,
                      void *workspace, size_t workspace_bytes, void *stream);
 
+/* One decode step: append one token per sequence, then decode attention
+ * with the appended token in the cache.  The same results as
+ * lrkv_compress(cache, k, v, 1, NULL, ...) followed by lrkv_decode_attn
+ * (the folded queries agree up to fp32 rounding order), with one launch
+ * fewer: the append kernel, which stages each unit's basis anyway, also
+ * folds that unit's queries q~ = P_k^T q into the workspace.
+ *   k, v : [batch][num_kv_heads][1][128] post-RoPE (seq_stride, head_stride
+ *          in elements, as for lrkv_compress); q, o, scale, workspace as for
+ *          lrkv_decode_attn (the same workspace size).
+ *   Plain caches only (LRKV_BF16, LRKV_F32; LRKV_ERR_UNSUPPORTED otherwise).
+ *   Arguments are checked as by the two calls; on failure nothing is
+ *   launched. */
+int lrkv_decode_step(const lrkv_cache *cache, const void *k, const void *v,
+                     int64_t seq_stride, int64_t head_stride, const void *q,
+                     int32_t num_q_heads, const float *P_k, const float *P_v,
+                     int64_t basis_batch_stride, float scale, void *o,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
 /* Decode attention over a value-amortised cache: as lrkv_decode_attn, with
  * each latent token's value code read as A^T c_k plus its kept residual.
  * The split-K pass sums p c_k over the key codes and p e over the residual

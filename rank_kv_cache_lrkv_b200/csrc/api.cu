@@ -157,10 +157,11 @@ size_t lrkv_decode_workspace_bytes(const lrkv_cache* cache, int32_t num_q_heads)
                                 cache->dtype);
 }
 
-static int decode_checked(const lrkv_cache* cache, const void* q, int32_t num_q_heads,
-                          const float* P_k, const float* P_v, int64_t basis_batch_stride,
-                          const float* A, float scale, void* o, void* workspace,
-                          size_t workspace_bytes, void* stream) {
+// The checks of the decode entry points; fills the launch description.
+static int decode_setup(const lrkv_cache* cache, const void* q, int32_t num_q_heads,
+                        const float* P_k, const float* P_v, int64_t basis_batch_stride,
+                        const float* A, float scale, void* o, void* workspace,
+                        size_t workspace_bytes, DecodeLaunch& L) {
   int rc = check_cache(cache);
   if (rc != LRKV_OK) return rc;
   if ((cache->dtype == LRKV_BF16_VA) != (A != nullptr)) return LRKV_ERR_UNSUPPORTED;
@@ -170,7 +171,6 @@ static int decode_checked(const lrkv_cache* cache, const void* q, int32_t num_q_
   if (!q || !o || !P_k || !P_v || !workspace || basis_batch_stride < 0) return LRKV_ERR_ARG;
   // the value basis is read four floats at a time
   if (!aligned16(workspace) || !aligned16(P_v) || basis_batch_stride % 4 != 0) return LRKV_ERR_ARG;
-  DecodeLaunch L;
   L.B = cache->batch; L.H_kv = cache->num_kv_heads; L.H_q = num_q_heads; L.dtype = cache->dtype;
   L.seq_len = cache->seq_len; L.n_sink = cache->n_sink; L.W = cache->window;
   L.codes = cache->codes; L.bt_lat = cache->block_table;
@@ -183,7 +183,47 @@ static int decode_checked(const lrkv_cache* cache, const void* q, int32_t num_q_
   L.num_pages_fr = 0;
   L.q = q; L.P_k = P_k; L.P_v = P_v; L.basis_bs = basis_batch_stride; L.scale = scale;
   L.o = o; L.ws = workspace; L.ws_bytes = workspace_bytes; L.A = A;
+  return LRKV_OK;
+}
+
+static int decode_checked(const lrkv_cache* cache, const void* q, int32_t num_q_heads,
+                          const float* P_k, const float* P_v, int64_t basis_batch_stride,
+                          const float* A, float scale, void* o, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  DecodeLaunch L;
+  const int rc = decode_setup(cache, q, num_q_heads, P_k, P_v, basis_batch_stride, A, scale, o,
+                              workspace, workspace_bytes, L);
+  if (rc != LRKV_OK) return rc;
   return decode_launch(L, static_cast<cudaStream_t>(stream));
+}
+
+int lrkv_decode_step(const lrkv_cache* cache, const void* k, const void* v, int64_t seq_stride,
+                     int64_t head_stride, const void* q, int32_t num_q_heads, const float* P_k,
+                     const float* P_v, int64_t basis_batch_stride, float scale, void* o,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!cache) return LRKV_ERR_ARG;
+  int rc = check_cache(cache);
+  if (rc != LRKV_OK) return rc;
+  if (cache->dtype != LRKV_BF16 && cache->dtype != LRKV_F32) return LRKV_ERR_UNSUPPORTED;
+  DecodeLaunch L;
+  rc = decode_setup(cache, q, num_q_heads, P_k, P_v, basis_batch_stride, nullptr, scale, o,
+                    workspace, workspace_bytes, L);
+  if (rc != LRKV_OK) return rc;
+  // the append's arguments, as lrkv_compress checks them for one token
+  const int ce = chunk_elems(cache->dtype);
+  if (!k || !v || !aligned16(k) || !aligned16(v) || seq_stride % ce != 0 ||
+      head_stride % ce != 0 || !aligned16(P_k))
+    return LRKV_ERR_ARG;
+  StepFold f;
+  rc = decode_fold_targets(L, &f.qlat, &f.qfr, &f.qscale);
+  if (rc != LRKV_OK) return rc;
+  f.q = q;
+  f.H_q = num_q_heads;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = compress_launch(*cache, k, v, 1, nullptr, seq_stride, head_stride, P_k, P_v,
+                       basis_batch_stride, st, nullptr, &f);
+  if (rc != LRKV_OK) return rc;
+  return decode_launch(L, st, true);
 }
 
 int lrkv_decode_attn(const lrkv_cache* cache, const void* q, int32_t num_q_heads,

@@ -204,6 +204,18 @@ __device__ __forceinline__ void pdl_trigger() {
 __device__ __forceinline__ void named_bar(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Named barrier that also returns whether any of its threads passed
+// pred = true (the same answer in every thread).
+__device__ __forceinline__ bool named_bar_any(int id, int threads, bool pred) {
+  int r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n"
+      " bar.red.or.pred q, %2, %3, p;\n selp.s32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((int)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
 
 __device__ inline float warp_max(float v) {
 #pragma unroll

@@ -30,10 +30,11 @@ constexpr int kRowBatch = 16;  // token rows projected per pass
 // Dynamic shared memory of append_kernel: the unit's basis [128][r_k + r_v]
 // fp32, rows [kRowBatch][k, v][128] fp32, partial sums [256], and a page per row.
 // (+ one row of codes [256] and two scales for int8 codes, a value residual
-// [128] and its slot for value-amortised slabs)
+// [128] and its slot for value-amortised slabs, and the query rows [8][128]
+// of a decode step's fold)
 inline size_t append_smem_bytes(int rk, int rv) {
   return ((size_t)kHeadDim * (rk + rv) + (size_t)kRowBatch * 2 * kHeadDim + 256 + kRowBatch +
-          256 + 4 + kHeadDim + 4) * 4;
+          256 + 4 + kHeadDim + 4 + 8 * kHeadDim) * 4;
 }
 
 // One CTA per (KV head, sequence).  Latency matters here (a decode step
@@ -57,11 +58,25 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
   float* qscale = crow + 256;                                          // [2] its scales
   float* ev = qscale + 4;                                              // [rv] value residual
   int* vslot = reinterpret_cast<int*>(ev + kHeadDim);                  // its slot
+  float* qsm = reinterpret_cast<float*>(vslot + 4);                    // [G][128] fold input
   const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
 
   // Launched with programmatic dependent launch: wait for the previous grid
-  // before reading anything (only the launch latency is hidden).
+  // before reading anything (only the launch latency is hidden).  The next
+  // grid may be scheduled from here on; it waits for this one to finish
+  // before it reads what this one writes.
   pdl_wait();
+  pdl_trigger();
+  // 0. a decode step's query rows (G <= 8 heads, four values per thread),
+  // in flight together with the loads below
+  const int FG = a.fq ? a.fH_q / a.H_kv : 0;
+  const size_t fh0 = ((size_t)b * a.fH_q + (size_t)kvh * FG);
+  float fqv[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int x = tid + e * (int)blockDim.x;
+    fqv[e] = x < FG * kHeadDim ? to_f<T>(static_cast<const T*>(a.fq)[fh0 * kHeadDim + x]) : 0.f;
+  }
   // 1. seq_len, and the basis into shared memory ([i][o]: P_k columns then P_v),
   // sixteen 16-byte loads in flight per thread (one round at r_k + r_v <= 128)
   const int L0 = __ldcg(a.seq_len + b);
@@ -95,6 +110,30 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a, int do_input_
   // The arrive (release) comes after the basis loads, which are in flight
   // together with the seq_len load, so it costs no round trip of its own.
   if constexpr (kCluster) cluster_arrive();
+  // 1b. a decode step's query fold for unit (b, kvh): q~[g][j] =
+  // fqscale sum_i P_k[i][j] q[g][i] from the staged basis (thread -> output
+  // (g, j), four partial sums); the scaled rows for the anchors
+  if (FG) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int x = tid + e * (int)blockDim.x;
+      if (x < FG * kHeadDim) {
+        qsm[x] = fqv[e];
+        if (a.fqfr) a.fqfr[fh0 * kHeadDim + x] = fqv[e] * a.fqscale;
+      }
+    }
+    __syncthreads();
+    for (int x = tid; x < FG * a.rk; x += blockDim.x) {
+      const int g = x / a.rk, j = x - g * a.rk;
+      const float* qg = qsm + g * kHeadDim;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int i = 0; i < kHeadDim; i += 4)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) s4[u] = fmaf(Ps[(i + u) * NJ + j], qg[i + u], s4[u]);
+      a.fqlat[fh0 * a.rk + x] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * a.fqscale;
+    }
+  }
   const int L1 = L0 + appended(a.n_new, a.n, b);
   const Split s0 = split_tokens(L0, a.n_sink, a.W), s1 = split_tokens(L1, a.n_sink, a.W);
   const T* kin = static_cast<const T*>(a.k) + (size_t)b * a.seq_stride + (size_t)kvh * a.head_stride;
@@ -594,7 +633,8 @@ static int compress_t(const AppendArgs& a, cudaStream_t st) {
 
 int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, const int* n_new,
                     long long seq_stride, long long head_stride, const float* P_k,
-                    const float* P_v, long long basis_bs, cudaStream_t st, const float* A) {
+                    const float* P_v, long long basis_bs, cudaStream_t st, const float* A,
+                    const StepFold* fold) {
   AppendArgs a;
   a.B = c.batch; a.H_kv = c.num_kv_heads; a.rk = c.rank_k; a.rv = c.rank_v;
   a.n_sink = c.n_sink; a.W = c.window; a.maxp = c.max_pages_per_seq; a.num_pages = c.num_pages;
@@ -606,6 +646,11 @@ int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, co
   a.bt = c.block_table; a.seq_len = c.seq_len; a.counter = c.append_counter; a.n_new = n_new;
   a.k = k; a.v = v; a.seq_stride = seq_stride; a.head_stride = head_stride;
   a.P_k = P_k; a.P_v = P_v; a.basis_bs = basis_bs;
+  a.fq = fold ? fold->q : nullptr;
+  a.fH_q = fold ? fold->H_q : 0;
+  a.fqscale = fold ? fold->qscale : 0.f;
+  a.fqlat = fold ? fold->qlat : nullptr;
+  a.fqfr = fold ? fold->qfr : nullptr;
   return c.dtype == LRKV_F32 ? compress_t<float>(a, st) : compress_t<__nv_bfloat16>(a, st);
 }
 

@@ -27,6 +27,14 @@ struct AppendArgs {
   long long seq_stride, head_stride;
   const float *P_k, *P_v;
   long long basis_bs;
+  // Optional query fold of a decode step (fq != nullptr), done by the CTA of
+  // unit (b, kvh) from the basis it stages anyway: q [B][fH_q][128] ->
+  // fqlat [B][fH_q][rk] = fqscale P_k^T q and, when fqfr != nullptr,
+  // fqfr [B][fH_q][128] = fqscale q.
+  const void* fq;
+  int fH_q;
+  float fqscale;
+  float *fqlat, *fqfr;
 };
 
 // Element offset of (slot, dim d) of the key (isv = 0) or value (isv = 1)

@@ -46,6 +46,7 @@ constexpr int kMergeThreads = 256;
 constexpr int kMergeWarps = kMergeThreads / 32;
 constexpr int kMergeBuf = 64 * 1024;           // merge: bytes of records per chunk
 constexpr int kMergeMaxRec = 256;              // merge: records per chunk at most
+constexpr int kBarRecords = 1;                 // consumers: a unit's warp records are written
 
 struct DecodeArgs {
   int B, H_kv, G, H_q;
@@ -70,8 +71,8 @@ struct DecodeArgs {
   int* err;            // sticky error word
   float* qlat;         // [B][H_q][rk] folded queries (scaled)
   float* qfr;          // [B][H_q][128] scaled queries
-  float* part_lat;     // [(U + C - 1) * kConsumers] latent records
-  float* part_fr;      // anchors: [U + C - 1]; dense: [(U + C - 1) * kConsumers]
+  float* part_lat;     // [U + C - 1] latent records, one per (CTA, unit)
+  float* part_fr;      // [U + C - 1] full-rank records, one per (CTA, unit)
   int C;               // CTAs of the split grid
   int NS;              // ring stages
   int stage_bytes;
@@ -79,6 +80,7 @@ struct DecodeArgs {
                        // value-amortised slabs: per-consumer page weights
   const float* A;      // value-amortised slabs: predictors [B][H_kv][rk][rv]
   int rw;              // latent record width per head: rv, or rk + rv (amortised)
+  int wait_first;      // 1: the previous grid (a step's append) writes the cache
 };
 
 constexpr int kModePlain = 0;  // bf16 / fp32 latent codes
@@ -743,13 +745,14 @@ __host__ __device__ inline bool anchor_mode(const void* fr, const int* bt_fr) {
 
 // Shared-memory plan of the split kernel (byte offsets from the base).
 struct SmemPlan {
-  int ring, full, empty, tag, start_lat, start_fr, pbuf, qown, flags, dq, total;
+  int ring, full, empty, tag, start_lat, start_fr, pbuf, qown, wrec, flags, dq, total;
 };
 // tc: the consumers run on the tensor cores and keep their query fragments in
 // registers, so only the anchor warp needs probability and query slices.
 // dq_bytes: per consumer warp, the bf16 form of half an int8 page.
+// rvd: record width per head of the ring space (r_v, r_k + r_v, or 128).
 __host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, int G, bool tc,
-                                              int dq_bytes = 0) {
+                                              int dq_bytes, int rvd) {
   const int slots = tc ? 1 : kConsumers + 1;
   SmemPlan p;
   int off = 0;
@@ -769,6 +772,8 @@ __host__ __device__ inline SmemPlan smem_plan(int NS, int stage_bytes, int B, in
   // the unit's folded queries [G][128]
   p.pbuf = take(slots * kLatPage * G * 8, 16);
   p.qown = take(slots * G * kHeadDim * 4, 16);
+  // the consumer warps' records of one unit, combined into the CTA's record
+  p.wrec = take(kConsumers * (hdr_floats(G) + G * rvd) * 4, 16);
   p.flags = take(16, 16);
   p.dq = take(kConsumers * dq_bytes, 128);
   p.total = off;
@@ -934,6 +939,38 @@ __device__ __forceinline__ void dequant_half(const uint4* slab, int half, int rk
   __syncwarp();
 }
 
+// The consumer warps' records of one unit (shared memory wrec, kConsumers
+// rows of S floats: m[G], l[G], acc [G][rvd]) -> the CTA's record for the
+// unit (rec, global memory): M = max m, w = exp2(m - M), l = sum w l,
+// acc = sum w acc.  Run by the 32 * kConsumers consumer threads (ltid);
+// a warp without a tile of the unit holds m = -inf and weighs 0.
+template <int G>
+__device__ inline void combine_warp_records(const float* wrec, int S, int rvd, float* rec,
+                                            int ltid) {
+  const int H = hdr_floats(G);
+  for (int x = ltid; x < G * rvd + G; x += 32 * kConsumers) {
+    const bool hdr = x >= G * rvd;
+    const int g = hdr ? x - G * rvd : x / rvd, j = hdr ? 0 : x - g * rvd;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, wrec[w * S + g]);
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumers; ++w) {
+      const float m = wrec[w * S + g];
+      const float wt = m > -INFINITY ? exp2f(m - M) : 0.f;
+      const float v = hdr ? wrec[w * S + G + g] : wrec[w * S + H + g * rvd + j];
+      sum = fmaf(wt, wt > 0.f ? v : 0.f, sum);
+    }
+    if (hdr) {
+      rec[g] = M;
+      rec[G + g] = sum;
+    } else {
+      rec[H + g * rvd + j] = sum;
+    }
+  }
+}
+
 // ------------------------------------------------------------ split kernel
 // kDense: the ring carries full-rank pages (dense baseline) instead of latent
 // pages; KS / VB: rank class of the tensor-core tiles (bf16 only).
@@ -950,7 +987,8 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   constexpr int NP = CE / 2;
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr bool kTC = std::is_same<T, __nv_bfloat16>::value;
-  const SmemPlan sp_ = smem_plan(a.NS, a.stage_bytes, a.B, G, kTC, a.dq_bytes);
+  const SmemPlan sp_ = smem_plan(a.NS, a.stage_bytes, a.B, G, kTC, a.dq_bytes,
+                                 kDense ? kHeadDim : a.rw);
   uint8_t* ring = smem + sp_.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp_.full);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + sp_.empty);
@@ -967,6 +1005,10 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   pdl_trigger();  // the merge grid may be scheduled; it waits for this grid to finish
+  // After a step's append (which also folded the queries) nothing of the
+  // cache may be read before that grid is done; after a q-fold the cache was
+  // final before it started.
+  if (a.wait_first) pdl_wait();
   if (warp == 0) build_prefix(a, start_lat, start_fr);
   if (threadIdx.x == 32) {
     *fail = 0;
@@ -1112,6 +1154,7 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
   // ---------------- consumers (bf16 pages on the tensor cores, fp32 on SIMT)
   constexpr bool kTensorTiles = std::is_same<T, __nv_bfloat16>::value;
   const int w = warp - kFirstConsumer;
+  float* wrec = reinterpret_cast<float*>(smem + sp_.wrec);
   const int nck = rsp == 0 ? a.rk / CE : kHeadDim / CE;  // (int8 pages: of the bf16 buffer)
   const int ncv = rsp == 0 ? a.rv / CE : kHeadDim / CE;
   const int rvd = rsp == 0 ? a.rw : kHeadDim;
@@ -1142,7 +1185,7 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
     auto release = [&](int tt) {
       if (lane == 0) mbar_arrive(&empty[(tt - lo) % a.NS]);
     };
-    float* rec = part + ((size_t)(unit + c) * kConsumers + w) * rec_stride;
+    float* rec = wrec + w * rec_stride;  // this warp's record, combined below
     if constexpr (kTensorTiles) {
       constexpr int TT = kDense ? kFrTile : kLatPage;
       QFrag<KS> qf;
@@ -1178,9 +1221,6 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
           release(tt);
         }
         write_record_va<G, KS, VB>(rec, a.rk, a.rv, m, l, acck, acce, lane);
-        t = ce;
-        if (*fail) break;
-        continue;
       } else if constexpr (kMode == kModeQ8 && !kDense) {
         // int8 pages: each half of 32 tokens is dequantised into this warp's
         // buffer, then run on the tensor cores as a 32-token tile
@@ -1209,7 +1249,7 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
         }
       }
       // This warp's record for (unit, CTA); m = -inf when it had no tile.
-      write_record_mma<G, VB>(rec, rvd, m, l, acc, lane);
+      if constexpr (!(kMode == kModeVA && !kDense)) write_record_mma<G, VB>(rec, rvd, m, l, acc, lane);
     } else {
       float m[G], l[G];
       float2 acc[G][NP];
@@ -1229,8 +1269,14 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
       }
       write_record<T, G>(rec, rvd, TS, ncv, m, l, acc, lane);
     }
+    // The CTA's one record for (unit, space).  Every consumer warp passes
+    // here once per unit; a failure seen by any of them ends them all.
+    if (named_bar_any(kBarRecords, 32 * kConsumers, *fail != 0)) break;
+    combine_warp_records<G>(wrec, rec_stride, rvd, part + (size_t)(unit + c) * rec_stride,
+                            threadIdx.x - 32 * kFirstConsumer);
+    // a warp without tiles in the next unit writes its next record at once
+    named_bar(kBarRecords, 32 * kConsumers);
     t = ce;
-    if (*fail) break;
   }
 }
 
@@ -1357,7 +1403,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     c0[sp] = cta_of(us, total[sp], Ce);
     ncta[sp] = cta_of(us + tiles - 1, total[sp], Ce) - c0[sp] + 1;
   }
-  const int per0 = kConsumers, per1 = anchors ? 1 : kConsumers;
+  const int per0 = 1, per1 = 1;  // one record per (CTA, unit) in each space
   const int S0 = H + G * a.rw, S1 = H + G * kHeadDim;  // floats per record
   const int n0 = ncta[0] * per0, n1 = ncta[1] * per1;
   const float* src0 = a.part_lat + (size_t)(unit + c0[0]) * per0 * S0;
@@ -1556,10 +1602,11 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   // Leave room for a q-fold CTA beside each split CTA.
   const int budget = optin - 8 * 1024;
   const bool tc = esize == 2;  // bf16: tensor-core consumers
-  const int fixed = smem_plan(0, p.stage_bytes, B, G, tc, p.dq_bytes).total + 1024;
+  const int rvd = has_lat ? rw : kHeadDim;  // record width per head of the ring space
+  const int fixed = smem_plan(0, p.stage_bytes, B, G, tc, p.dq_bytes, rvd).total + 1024;
   p.NS = std::min(kMaxStages, (budget - fixed) / p.stage_bytes);
   if (p.NS < 2) return LRKV_ERR_UNSUPPORTED;
-  p.smem = smem_plan(p.NS, p.stage_bytes, B, G, tc, p.dq_bytes).total;
+  p.smem = smem_plan(p.NS, p.stage_bytes, B, G, tc, p.dq_bytes, rvd).total;
   p.C = sms;
   p.merge_smem = merge_plan(rv, has_lat, G, B, mode == kModeVA ? rk : 0).total;
   const int U = B * H_kv;
@@ -1569,10 +1616,9 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   p.off_qfr = off;  off = al(off + (size_t)B * H_q * (has_fr ? kHeadDim : 0) * 4);
   const size_t slots = (size_t)(U + p.C - 1);
   p.off_lat = off;
-  off = al(off + (has_lat ? slots * kConsumers * (hdr_floats(G) + G * rw) * 4 : 0));
+  off = al(off + (has_lat ? slots * (hdr_floats(G) + G * rw) * 4 : 0));
   p.off_fr = off;
-  off = al(off + (has_fr ? slots * (anchors ? 1 : kConsumers) * (hdr_floats(G) + G * kHeadDim) * 4
-                         : 0));
+  off = al(off + (has_fr ? slots * (hdr_floats(G) + G * kHeadDim) * 4 : 0));
   p.total = off;
   return LRKV_OK;
 }
@@ -1633,7 +1679,7 @@ static const void* split_fn(const DecodeArgs& a) {
 }
 
 template <typename T, int G>
-static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st) {
+static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st, bool folded) {
   // Keep SMs in the large-shared-memory configuration while the q-fold runs,
   // so the split kernel's CTAs can start beside it without a reconfiguration.
   // (Kernel attributes are set once per device; see prepare_kernel.)
@@ -1642,8 +1688,10 @@ static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st) {
   if (rc == LRKV_OK) rc = prepare_kernel(split, true);
   if (rc == LRKV_OK) rc = prepare_kernel((const void*)merge_kernel<T, G>, false);
   if (rc != LRKV_OK) return rc;
-  qfold_kernel<T, G><<<a.B * a.H_kv * kFoldSplit, kFoldThreads, 0, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
+  if (!folded) {
+    qfold_kernel<T, G><<<a.B * a.H_kv * kFoldSplit, kFoldThreads, 0, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
+  }
   void* args[] = {&a};
   if (launch_pdl(split, dim3(p.C), dim3(kThreads), p.smem, st, args) != cudaSuccess)
     return LRKV_ERR_CUDA;
@@ -1654,26 +1702,25 @@ static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st) {
 }
 
 template <typename T>
-static int launch_decode_g(const DecodeArgs& a, const Plan& p, cudaStream_t st) {
+static int launch_decode_g(const DecodeArgs& a, const Plan& p, cudaStream_t st, bool folded) {
   switch (a.G) {
-    case 1: return launch_decode_t<T, 1>(a, p, st);
-    case 2: return launch_decode_t<T, 2>(a, p, st);
-    case 4: return launch_decode_t<T, 4>(a, p, st);
-    case 8: return launch_decode_t<T, 8>(a, p, st);
+    case 1: return launch_decode_t<T, 1>(a, p, st, folded);
+    case 2: return launch_decode_t<T, 2>(a, p, st, folded);
+    case 4: return launch_decode_t<T, 4>(a, p, st, folded);
+    case 8: return launch_decode_t<T, 8>(a, p, st, folded);
     default: return LRKV_ERR_UNSUPPORTED;
   }
 }
 
-int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
+// Plan and workspace pointers of a decode call.
+static int decode_args(const DecodeLaunch& L, DecodeArgs& a, Plan& p) {
   const bool has_lat = L.codes != nullptr, has_fr = L.fr != nullptr;
   const int es = L.dtype == LRKV_F32 ? 4 : 2;
-  Plan p;
   int rc = plan_decode(L.B, L.H_kv, L.H_q, L.rk, L.rv, has_lat, has_fr,
                        anchor_mode(L.fr, L.bt_fr), es, p, mode_of(L.dtype));
   if (rc != LRKV_OK) return rc;
   if (L.ws_bytes < p.total) return LRKV_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(L.ws);
-  DecodeArgs a;
   a.B = L.B; a.H_kv = L.H_kv; a.G = L.H_q / L.H_kv; a.H_q = L.H_q;
   a.seq_len = L.seq_len; a.n_sink = L.n_sink; a.W = L.W;
   a.codes = L.codes; a.bt_lat = L.bt_lat; a.maxp_lat = L.maxp_lat;
@@ -1690,8 +1737,29 @@ int decode_launch(const DecodeLaunch& L, cudaStream_t st) {
   a.C = p.C; a.NS = p.NS; a.stage_bytes = p.stage_bytes; a.dq_bytes = p.dq_bytes;
   a.rw = p.rw;
   a.A = L.dtype == LRKV_BF16_VA ? L.A : nullptr;
-  if (L.dtype == LRKV_F32) return launch_decode_g<float>(a, p, st);
-  return launch_decode_g<__nv_bfloat16>(a, p, st);
+  a.wait_first = 0;
+  return LRKV_OK;
+}
+
+int decode_fold_targets(const DecodeLaunch& L, float** qlat, float** qfr, float* qscale) {
+  DecodeArgs a;
+  Plan p;
+  const int rc = decode_args(L, a, p);
+  if (rc != LRKV_OK) return rc;
+  *qlat = a.qlat;
+  *qfr = L.fr ? a.qfr : nullptr;
+  *qscale = a.qscale;
+  return LRKV_OK;
+}
+
+int decode_launch(const DecodeLaunch& L, cudaStream_t st, bool folded) {
+  DecodeArgs a;
+  Plan p;
+  const int rc = decode_args(L, a, p);
+  if (rc != LRKV_OK) return rc;
+  a.wait_first = folded ? 1 : 0;
+  if (L.dtype == LRKV_F32) return launch_decode_g<float>(a, p, st, folded);
+  return launch_decode_g<__nv_bfloat16>(a, p, st, folded);
 }
 
 }  // namespace lrkv

@@ -46,12 +46,27 @@ int decode_plan_check(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, bo
                       int dtype);
 // Status explaining a zero lrkv_decode_workspace_bytes for this cache.
 int decode_plan_status(const lrkv_cache* cache, int H_q);
-int decode_launch(const DecodeLaunch& L, cudaStream_t st);
+// The query fold of a decode step, done by the append kernel: q (cache
+// dtype, [B][H_q][128]) -> qlat [B][H_q][rk] = qscale P_k^T q and, when qfr
+// is set, qfr [B][H_q][128] = qscale q (qscale = scale log2 e).
+struct StepFold {
+  const void* q;
+  int H_q;
+  float qscale;
+  float *qlat, *qfr;
+};
+// folded == true: a decode step whose queries the append kernel just folded
+// into the workspace (decode_fold_targets); the q-fold launch is skipped and
+// the split kernel waits for the append before reading the cache.
+int decode_launch(const DecodeLaunch& L, cudaStream_t st, bool folded = false);
+// Workspace addresses the q-fold of L writes (qfr == nullptr: no full-rank
+// space); a status other than LRKV_OK when L cannot be planned.
+int decode_fold_targets(const DecodeLaunch& L, float** qlat, float** qfr, float* qscale);
 
 int compress_launch(const lrkv_cache& c, const void* k, const void* v, int n, const int* n_new,
                     long long seq_stride, long long head_stride, const float* P_k,
                     const float* P_v, long long basis_bs, cudaStream_t st,
-                    const float* A = nullptr);
+                    const float* A = nullptr, const StepFold* fold = nullptr);
 int dense_append_launch(const lrkv_dense_cache& c, const void* k, const void* v, int n,
                         const int* n_new,
                         long long seq_stride, long long head_stride, cudaStream_t st);

@@ -59,7 +59,7 @@ EXPORTS = ["lrkv_compress", "lrkv_decode_workspace_bytes", "lrkv_decode_attn",
            "lrkv_status_string", "lrkv_version", "lrkv_decode_attn_static",
            "lrkv_rebase_workspace_bytes", "lrkv_rebase", "lrkv_oja_update_chunked",
            "lrkv_compress_amortised", "lrkv_amortise_workspace_bytes", "lrkv_amortise",
-           "lrkv_decode_attn_amortised"]
+           "lrkv_decode_attn_amortised", "lrkv_decode_step"]
 
 
 def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
@@ -84,6 +84,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "lrkv_rebase_workspace_bytes": (SZ, [P]),
         "lrkv_rebase": (ctypes.c_int, [P, P, P, P, P, I64, P, SZ, P]),
         "lrkv_compress_amortised": (ctypes.c_int, [P, P, P, I32, P, I64, I64, P, P, I64, P, P]),
+        "lrkv_decode_step": (ctypes.c_int, [P, P, P, I64, I64, P, I32, P, P, I64, F32, P, P, SZ,
+                                            P]),
         "lrkv_amortise_workspace_bytes": (SZ, [P]),
         "lrkv_amortise": (ctypes.c_int, [P, P, I32, I64, I64, P, I64, P, P, SZ, P]),
         "lrkv_decode_attn_amortised": (ctypes.c_int,
@@ -247,6 +249,23 @@ def decode_attn_amortised(cache: LatentCache, q: torch.Tensor, P_k: torch.Tensor
     _check("lrkv_decode_attn_amortised", _lib.lrkv_decode_attn_amortised(
         ctypes.byref(cache.desc), _ptr(q), q.shape[1], _ptr(P_k), _ptr(P_v), basis_batch_stride,
         _ptr(A), float(scale), _ptr(o), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o
+
+
+def decode_step(cache: LatentCache, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
+                P_k: torch.Tensor, P_v: torch.Tensor, scale: float, o: torch.Tensor,
+                workspace: torch.Tensor, basis_batch_stride: int = 0,
+                stream=None) -> torch.Tensor:
+    """lrkv_decode_step: append k, v [B, H_kv, 1, 128] and attend with q
+    [B, H_q, 128] -> o."""
+    assert k.dtype == cache.dtype and v.dtype == cache.dtype and k.shape == v.shape
+    assert k.shape[2] == 1 and q.is_contiguous() and o.is_contiguous() and q.dtype == cache.dtype
+    ss, hs = _kv_strides(k)
+    assert _kv_strides(v) == (ss, hs)
+    _check("lrkv_decode_step", _lib.lrkv_decode_step(
+        ctypes.byref(cache.desc), _ptr(k), _ptr(v), ss, hs, _ptr(q), q.shape[1], _ptr(P_k),
+        _ptr(P_v), basis_batch_stride, float(scale), _ptr(o), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
     return o
 
 
