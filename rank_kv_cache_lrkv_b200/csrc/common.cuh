@@ -144,6 +144,30 @@ __device__ inline void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint
       : "memory");
 }
 
+// Bulk copy shared -> global through the async proxy, tracked in the
+// issuing thread's bulk groups (commit, then wait for reads or completion).
+__device__ inline void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ inline void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// At most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+__device__ inline void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// At most N of this thread's committed bulk groups are still in flight.
+template <int N>
+__device__ inline void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// Shared-memory writes of this thread (and, after a barrier, of the threads
+// it synchronised with) become visible to later async-proxy reads.
+__device__ inline void proxy_fence_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------ conversions
 // bf16 pair in one 32-bit word -> two floats (exact).
 __device__ inline float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -160,30 +160,33 @@ __global__ void __launch_bounds__(kRebaseThreads, 1) rebase_codes_kernel(RebaseA
 }
 
 // ---- bf16 codes on the tensor cores
-// rebase_codes_mma: persistent, several CTAs per SM.  The latent pages of
-// every (sequence, KV head) unit are laid end to end and each CTA takes an
-// equal contiguous range.  A producer warp streams one slab per page into a
-// ring of shared-memory stages with bulk copies (block-table entries
-// resolved a batch of 32 pages ahead).  Four consumer warps share each
-// page: warp w owns the 16 tokens of m-block w and every code column, and
-// computes c'[t][n] = sum_k c[t][k] R[n][k] with warp-level bf16 MMAs
-// (m16n8k16, fp32 accumulation), R split into hi + lo bf16 halves so the
-// products keep about 16 mantissa bits.  A fragments come by ldmatrix
-// straight from the chunk-major slab; a warp reads and rewrites only its own
-// rows, so it writes its new codes in place and copies its latent rows back
-// with 16-byte stores without waiting for the other warps; the stage is
-// released when all four have arrived.  R sits in padded rows [n][k] in
-// shared memory, rebuilt by the four warps together (a named barrier on
-// each side) when the range enters a new unit.
-constexpr int kRbConsumers = 4;
-constexpr int kRbThreads = 32 * (kRbConsumers + 1);
-constexpr int kRbMaxStages = 4;
+// rebase_codes_mma: persistent, one CTA per SM.  The latent pages of every
+// (sequence, KV head) unit are laid end to end and each CTA takes an equal
+// contiguous range.  A producer warp streams one slab per page into a ring
+// of shared-memory stages with bulk copies (block-table entries resolved a
+// batch of 32 pages ahead).  Three groups of four consumer warps take the
+// pages in turn; in a group, warp w owns the 16 tokens of m-block w and
+// every code column, and computes c'[t][n] = sum_k c[t][k] R[n][k] with
+// warp-level bf16 MMAs (m16n8k16, fp32 accumulation), R split into hi + lo
+// bf16 halves so the products keep about 16 mantissa bits.  A fragments
+// come by ldmatrix straight from the chunk-major slab and the new codes are
+// written in place.  A full page then goes back to its slab with one bulk
+// store, and its stage is released once that store has read it (one store
+// of the group kept in flight); a partial page goes back row by row.  Each
+// group keeps R of its current unit in its own padded rows [n][k], rebuilt
+// by its four warps when its pages enter a new unit.
+constexpr int kRbGroups = 3;
+constexpr int kRbGroupWarps = 4;
+constexpr int kRbGroupThreads = 32 * kRbGroupWarps;
+constexpr int kRbThreads = 32 * (1 + kRbGroups * kRbGroupWarps);
+constexpr int kRbMaxStages = 16;
 
 __host__ __device__ inline int rb_r16(int r) { return (r + 15) / 16 * 16; }
 __host__ __device__ inline int rb_row(int r) { return rb_r16(r) + 8; }  // padded R row (bf16)
 
 struct RbPlan {
-  int ring, rk_hi, rk_lo, rv_hi, rv_lo, full, empty, meta, start, flag, total;
+  int ring, R[kRbGroups], full, empty, meta, start, flag, total;
+  int rk_lo, rv_hi, rv_lo;  // offsets inside a group's R block (rk_hi at 0)
 };
 __host__ __device__ inline RbPlan rb_plan(int NS, int rk, int rv, int B) {
   RbPlan p;
@@ -196,10 +199,11 @@ __host__ __device__ inline RbPlan rb_plan(int NS, int rk, int rv, int B) {
   };
   const int slab = kLatPage * (rk + rv) * 2;
   p.ring = take(NS * slab, 128);
-  p.rk_hi = take(rb_r16(rk) * rb_row(rk) * 2, 16);
-  p.rk_lo = take(rb_r16(rk) * rb_row(rk) * 2, 16);
-  p.rv_hi = take(rb_r16(rv) * rb_row(rv) * 2, 16);
-  p.rv_lo = take(rb_r16(rv) * rb_row(rv) * 2, 16);
+  const int kb = rb_r16(rk) * rb_row(rk) * 2, vb = rb_r16(rv) * rb_row(rv) * 2;
+  p.rk_lo = kb;
+  p.rv_hi = 2 * kb;
+  p.rv_lo = 2 * kb + vb;
+  for (int gi = 0; gi < kRbGroups; ++gi) p.R[gi] = take(2 * kb + 2 * vb, 16);
   p.full = take(NS * 8, 8);
   p.empty = take(NS * 8, 8);
   p.meta = take(NS * 2 * 4, 4);      // per stage: page (-1 bad), latent rows
@@ -238,7 +242,7 @@ __device__ inline bool rb_wait_warp(uint64_t* bar, uint32_t parity, volatile int
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-__global__ void __launch_bounds__(kRbThreads) rebase_codes_mma(RebaseArgs a, int NS) {
+__global__ void __launch_bounds__(kRbThreads, 1) rebase_codes_mma(RebaseArgs a, int NS) {
   using bf16 = __nv_bfloat16;
   extern __shared__ __align__(128) uint8_t rsm[];
   const RbPlan pl = rb_plan(NS, a.rk, a.rv, a.B);
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(kRbThreads) rebase_codes_mma(RebaseArgs a, int
   if (tid == 32) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kRbConsumers);
+      mbar_init(&empty[s], 1);  // the consuming group's leader, once its store has read
     }
     *fail = 0;
     *cfail = 0;
@@ -354,23 +358,27 @@ __global__ void __launch_bounds__(kRbThreads) rebase_codes_mma(RebaseArgs a, int
     return;
   }
 
-  // ---------------- consumers: warp cw owns rows 16 cw .. 16 cw + 15
-  const int cw = warp - 1, ctid = tid - 32;
+  // ---------------- consumers: group gi takes pages gi, gi + 3, ...; its
+  // warp cw owns rows 16 cw .. 16 cw + 15
+  const int gi = (warp - 1) / kRbGroupWarps, cw = (warp - 1) % kRbGroupWarps;
+  const int gtid = cw * 32 + lane, gbar = 1 + gi;
+  const bool leader = cw == 0 && lane == 0;
   const int g = lane >> 2, t = lane & 3;
-  auto Rh = [&](int sd) { return reinterpret_cast<bf16*>(rsm + (sd ? pl.rv_hi : pl.rk_hi)); };
-  auto Rl = [&](int sd) { return reinterpret_cast<bf16*>(rsm + (sd ? pl.rv_lo : pl.rk_lo)); };
+  uint8_t* Rb = rsm + pl.R[gi];
+  auto Rh = [&](int sd) { return reinterpret_cast<bf16*>(Rb + (sd ? pl.rv_hi : 0)); };
+  auto Rl = [&](int sd) { return reinterpret_cast<bf16*>(Rb + (sd ? pl.rv_lo : pl.rk_lo)); };
   auto side_on = [&](int sd) { return (sd ? a.Pv_old : a.Pk_old) != nullptr; };
   int cur_unit = -1;
-  for (int k = 0; k < N; ++k) {
+  int pending = -1;  // leader: stage whose bulk store may still be reading it
+  for (int k = gi; k < N; k += kRbGroups) {
     const int s = k % NS;
     int b, kvh, p;
     locate(lo + k, b, kvh, p);
     const int unit = b * a.H_kv + kvh;
     if (unit != cur_unit) {
       // R of the new unit as padded [n][k] rows, hi + lo, zero past the rank.
-      // Every consumer takes this branch at the same page (the page order is
-      // fixed), so the barriers always meet, even after a failed wait.
-      named_bar(1, 32 * kRbConsumers);  // no warp still reads the old R
+      // Every warp of the group takes this branch at the same page.
+      named_bar(gbar, kRbGroupThreads);  // no warp still reads the old R
 #pragma unroll 1
       for (int sd = 0; sd < 2; ++sd) {
         if (!side_on(sd)) continue;
@@ -378,21 +386,40 @@ __global__ void __launch_bounds__(kRbThreads) rebase_codes_mma(RebaseArgs a, int
         const float* Rt = (sd ? a.Rv : a.Rk) + (size_t)unit * r * r;  // Rt[k][n] = R[n][k]
         bf16* rh = Rh(sd);
         bf16* rl = Rl(sd);
-        for (int x = ctid; x < R16 * R16; x += 32 * kRbConsumers) {
-          const int kk = x / R16, n = x - kk * R16;
-          const float v = (kk < r && n < r) ? __ldcg(Rt + (size_t)kk * r + n) : 0.f;
-          const bf16 h = __float2bfloat16_rn(v);
-          rh[n * RS + kk] = h;
-          rl[n * RS + kk] = __float2bfloat16_rn(v - __bfloat162float(h));
+        // thread -> (row kk of R^T, four columns n); eight float4 loads in
+        // flight per thread before any is stored (r is a multiple of 8)
+        const int n4 = R16 / 4;
+        for (int x0 = gtid; x0 < R16 * n4; x0 += 8 * kRbGroupThreads) {
+          float4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int x = x0 + u * kRbGroupThreads, kk = x / n4, n = 4 * (x - kk * n4);
+            v[u] = (x < R16 * n4 && kk < r && n < r)
+                       ? __ldcg(reinterpret_cast<const float4*>(Rt + (size_t)kk * r + n))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int x = x0 + u * kRbGroupThreads, kk = x / n4, n = 4 * (x - kk * n4);
+            if (x < R16 * n4) {
+              const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const bf16 h = __float2bfloat16_rn(e[i]);
+                rh[(n + i) * RS + kk] = h;
+                rl[(n + i) * RS + kk] = __float2bfloat16_rn(e[i] - __bfloat162float(h));
+              }
+            }
+          }
         }
       }
       cur_unit = unit;
-      named_bar(1, 32 * kRbConsumers);
+      named_bar(gbar, kRbGroupThreads);
     }
-    if (!rb_wait_warp(&full[s], (k / NS) & 1, cfail, lane)) continue;  // skip work, keep pace
+    const bool landed = rb_wait_warp(&full[s], (k / NS) & 1, cfail, lane);
     const int page = meta[2 * s], rows = meta[2 * s + 1];
     uint8_t* st = rsm + pl.ring + (size_t)s * slab_bytes;
-    if (page >= 0) {
+    if (landed && page >= 0) {
       const uint32_t sbase = smem_u32(st);
       bf16* sb = reinterpret_cast<bf16*>(st);
 #pragma unroll 1
@@ -439,19 +466,41 @@ __global__ void __launch_bounds__(kRbThreads) rebase_codes_mma(RebaseArgs a, int
           }
         }
       }
-      __syncwarp();  // the warp's new codes are in place
-      // this warp's latent rows of the re-based sides go back, 16 bytes at a time
-      const uint4* src = reinterpret_cast<const uint4*>(st);
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(a.codes) +
-                                            ((size_t)page * a.H_kv + kvh) * kLatPage * NJ);
-      const int c0 = side_on(0) ? 0 : a.rk / 8, c1 = side_on(1) ? NJ / 8 : a.rk / 8;
-      for (int x = lane; x < (c1 - c0) * 16; x += 32) {
-        const int c = c0 + x / 16, row = cw * 16 + (x & 15);
-        if (row < rows) dst[c * kLatPage + row] = src[c * kLatPage + row];
+      if (rows < kLatPage) {
+        // a partial page: only its latent rows go back, 16 bytes at a time
+        __syncwarp();
+        const uint4* src = reinterpret_cast<const uint4*>(st);
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(a.codes) +
+                                              ((size_t)page * a.H_kv + kvh) * kLatPage * NJ);
+        const int c0 = side_on(0) ? 0 : a.rk / 8, c1 = side_on(1) ? NJ / 8 : a.rk / 8;
+        for (int x = lane; x < (c1 - c0) * 16; x += 32) {
+          const int c = c0 + x / 16, row = cw * 16 + (x & 15);
+          if (row < rows) dst[c * kLatPage + row] = src[c * kLatPage + row];
+        }
       }
     }
-    __syncwarp();  // the warp is done with the stage
-    if (lane == 0) mbar_arrive(&empty[s]);
+    // the group's new codes are in place (and a partial page's rows read);
+    // each thread's shared-memory writes are ordered before the bulk store
+    proxy_fence_smem();
+    named_bar(gbar, kRbGroupThreads);
+    if (leader) {
+      if (landed && page >= 0 && rows >= kLatPage) {
+        // a full page: the whole slab back with one bulk store
+        bulk_s2g(static_cast<bf16*>(a.codes) + ((size_t)page * a.H_kv + kvh) * kLatPage * NJ,
+                 st, slab_bytes);
+        bulk_commit();
+        bulk_wait_read<1>();  // the group's previous store has read its stage
+        if (pending >= 0) mbar_arrive(&empty[pending]);
+        pending = s;
+      } else {
+        mbar_arrive(&empty[s]);  // nothing reads this stage any more
+      }
+    }
+  }
+  if (leader) {
+    bulk_wait_read<0>();
+    if (pending >= 0) mbar_arrive(&empty[pending]);
+    bulk_wait<0>();  // the stores are complete before the CTA exits
   }
 }
 
@@ -470,20 +519,15 @@ int launch_rebase_t(const RebaseArgs& a, cudaStream_t st) {
     DevInfo info;
     rc = current_device_info(dev, info);
     if (rc != LRKV_OK) return rc;
+    // one CTA per SM; each consumer group keeps one stage back for its
+    // store, so at least two stages per group
     int NS = kRbMaxStages;
-    while (NS >= 2 && rb_plan(NS, a.rk, a.rv, a.B).total > info.optin) --NS;
-    if (NS >= 2) {
+    while (NS >= 2 * kRbGroups && rb_plan(NS, a.rk, a.rv, a.B).total > info.optin) --NS;
+    if (NS >= 2 * kRbGroups) {
       rc = prepare_kernel((const void*)rebase_codes_mma, false);
       if (rc != LRKV_OK) return rc;
       const int smem = rb_plan(NS, a.rk, a.rv, a.B).total;
-      int per_sm = 1;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rebase_codes_mma, kRbThreads,
-                                                        smem) != cudaSuccess ||
-          per_sm < 1) {
-        cudaGetLastError();
-        per_sm = 1;
-      }
-      rebase_codes_mma<<<info.sms * per_sm, kRbThreads, smem, st>>>(a, NS);
+      rebase_codes_mma<<<info.sms, kRbThreads, smem, st>>>(a, NS);
       return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
     }
   }
