@@ -81,6 +81,7 @@ struct DecodeArgs {
   const float* A;      // value-amortised slabs: predictors [B][H_kv][rk][rv]
   int rw;              // latent record width per head: rv, or rk + rv (amortised)
   int wait_first;      // 1: the previous grid (a step's append) writes the cache
+  int fold_split;      // q-fold CTAs per unit (each folds at most 32 columns)
 };
 
 constexpr int kModePlain = 0;  // bf16 / fp32 latent codes
@@ -671,17 +672,38 @@ __device__ inline void write_record_va(float* rec, int rk, int rv, const float (
 
 // ------------------------------------------------------------ q-fold kernel
 constexpr int kFoldThreads = 128;  // small, so q-fold CTAs fit beside split CTAs
-constexpr int kFoldSplit = 2;      // CTAs per unit, each folding a share of the columns
+constexpr int kFoldSplit = 2;      // CTAs per unit at least, each folding a share of the columns
 
 template <typename T, int G>
 __global__ void __launch_bounds__(kFoldThreads) qfold_kernel(DecodeArgs a) {
   __shared__ float qs[G * kHeadDim];
   __shared__ float red[G * kFoldThreads];
   pdl_trigger();
-  const int unit = blockIdx.x / kFoldSplit, part = blockIdx.x % kFoldSplit;
+  const int unit = blockIdx.x / a.fold_split, part = blockIdx.x % a.fold_split;
   const int b = unit / a.H_kv, kvh = unit - b * a.H_kv, tid = threadIdx.x;
   const size_t h0 = (size_t)b * a.H_q + (size_t)kvh * G;
   const T* q = static_cast<const T*>(a.q) + h0 * kHeadDim;
+  // This CTA folds columns [c0, c1) (at most 32); thread -> (column j,
+  // segment of at most 32 rows).  Its P_k loads do not depend on q, so they
+  // are issued first and land together with the query rows (the split
+  // kernel's stream is already running, so every round trip here is long).
+  const int rk = a.codes ? a.rk : 0, cper = (rk + a.fold_split - 1) / a.fold_split;
+  const int c0 = part * cper, c1 = min(rk, c0 + cper), nc = max(0, c1 - c0);
+  const int nseg = nc > 0 ? max(1, kFoldThreads / nc) : 1, rows = (kHeadDim + nseg - 1) / nseg;
+  int j = 0, seg = 0, nrow = 0;
+  if (nc > 0 && tid < nseg * nc) {
+    j = c0 + tid % nc;
+    seg = tid / nc;
+    nrow = min(rows, kHeadDim - seg * rows);
+  }
+  float pij[32];  // rows <= 32 (at most 32 columns per CTA)
+  {
+    const float* P = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * rk + j;
+    const uint64_t pol = l2_evict_last_policy();
+#pragma unroll
+    for (int u = 0; u < 32; ++u)
+      pij[u] = u < nrow ? ldg_f_hint(P + (size_t)(seg * rows + u) * rk, pol) : 0.f;
+  }
   for (int x = tid; x < G * kHeadDim; x += kFoldThreads) qs[x] = to_f<T>(q[x]);
   __syncthreads();
   if (part == 0) {
@@ -689,31 +711,18 @@ __global__ void __launch_bounds__(kFoldThreads) qfold_kernel(DecodeArgs a) {
       for (int x = tid; x < G * kHeadDim; x += kFoldThreads)
         a.qfr[h0 * kHeadDim + x] = qs[x] * a.qscale;
   }
-  if (!a.codes) return;
-  // This CTA folds columns [c0, c1); thread -> (column, row segment) with at
-  // most 32 rows, all loads in flight at once.
-  const int rk = a.rk, cper = (rk + kFoldSplit - 1) / kFoldSplit;
-  const int c0 = part * cper, c1 = min(rk, c0 + cper), nc = c1 - c0;
-  if (nc <= 0) return;
-  const int nseg = max(1, kFoldThreads / nc), rows = (kHeadDim + nseg - 1) / nseg;
-  const float* P = a.P_k + (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * rk;
-  const uint64_t pol = l2_evict_last_policy();
-  for (int col = tid; col < nseg * nc; col += kFoldThreads) {
-    const int j = c0 + col % nc, seg = col / nc;
+  if (nc <= 0) return;  // no latent space, or no columns for this CTA (uniform)
+  if (nrow > 0) {
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = 0.f;
-    const int i0 = seg * rows, i1 = min(kHeadDim, i0 + rows);
-    for (int ib = i0; ib < i1; ib += 32) {
-      float pij[32];
+    const int i0 = seg * rows;
 #pragma unroll
-      for (int u = 0; u < 32; ++u) pij[u] = ib + u < i1 ? ldg_f_hint(P + (size_t)(ib + u) * rk + j, pol) : 0.f;
+    for (int u = 0; u < 32; ++u)
+      if (u < nrow)
 #pragma unroll
-      for (int u = 0; u < 32; ++u)
-        if (ib + u < i1)
+        for (int g = 0; g < G; ++g) acc[g] = fmaf(pij[u], qs[g * kHeadDim + i0 + u], acc[g]);
 #pragma unroll
-          for (int g = 0; g < G; ++g) acc[g] = fmaf(pij[u], qs[g * kHeadDim + ib + u], acc[g]);
-    }
     for (int g = 0; g < G; ++g) red[(seg * G + g) * nc + (j - c0)] = acc[g];
   }
   __syncthreads();
@@ -1689,7 +1698,7 @@ static int launch_decode_t(DecodeArgs a, const Plan& p, cudaStream_t st, bool fo
   if (rc == LRKV_OK) rc = prepare_kernel((const void*)merge_kernel<T, G>, false);
   if (rc != LRKV_OK) return rc;
   if (!folded) {
-    qfold_kernel<T, G><<<a.B * a.H_kv * kFoldSplit, kFoldThreads, 0, st>>>(a);
+    qfold_kernel<T, G><<<a.B * a.H_kv * a.fold_split, kFoldThreads, 0, st>>>(a);
     if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
   }
   void* args[] = {&a};
@@ -1738,6 +1747,7 @@ static int decode_args(const DecodeLaunch& L, DecodeArgs& a, Plan& p) {
   a.rw = p.rw;
   a.A = L.dtype == LRKV_BF16_VA ? L.A : nullptr;
   a.wait_first = 0;
+  a.fold_split = std::max(kFoldSplit, (L.rk + 31) / 32);
   return LRKV_OK;
 }
 
