@@ -87,17 +87,27 @@ def step_bytes(wl, L):
 # the decode sources hash to the recorded values; scaled to the bench's
 # context by the algorithmic bytes.
 TRAFFIC = {
+    # ncu --set full, one split_kernel launch (cold caches): DRAM read + write
     "llama3.1_8b_layer_T32768_anchors": {
-        "bytes": 205418240, "context": 32769,
-        "sources": {"decode.cu": "cc5a270849cb6a21b4cedf3f1521d198ecf782dd1f47affdbadfb09c4e090c42",
-                    "common.cuh": "8dce2af1220e3508e414de083472ec6f7a22e0e1c2b9d523c5e212a703323cbc"},
+        "bytes": 206988288, "context": 32771,
+        "sources": {"decode.cu": "3c6ffb5c05e8cf574c1e2e192f66c93132fe06c07bfffb5290964322e37cef51",
+                    "common.cuh": "867648f72ac4bef6638f39474ad2af8cef852d6f55e4d265fffd4c7212795edf"},
+    },
+}
+# The same kernel with caches left as the previous launch left them (ncu
+# --cache-control none, one pass): what a replayed call reads from DRAM.
+TRAFFIC_WARM = {
+    "llama3.1_8b_layer_T32768_anchors": {
+        "bytes": 199370000, "context": 32773,
+        "sources": {"decode.cu": "3c6ffb5c05e8cf574c1e2e192f66c93132fe06c07bfffb5290964322e37cef51",
+                    "common.cuh": "867648f72ac4bef6638f39474ad2af8cef852d6f55e4d265fffd4c7212795edf"},
     },
 }
 
 
-def measured_traffic(wl, L):
+def measured_traffic(wl, L, table=None):
     import hashlib
-    rec = TRAFFIC.get(wl.name)
+    rec = (TRAFFIC if table is None else table).get(wl.name)
     if rec is None:
         return None
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "rank_kv_cache_lrkv_b200", "csrc")
@@ -795,7 +805,8 @@ def run_ours(args, rank, world):
                      "frac": round(achieved / hbm, 4), "frac_of_8TBs": round(achieved / 8000, 4),
                      "peak_source": "MEASURED_PEAKS.json hbm_gbs" if pk else "fallback",
                      "bytes_per_call": abytes, "us_per_call": round(attn_ms * 1e3, 3),
-                     "context": L_now, "traffic": measured_traffic(wl, L_now)},
+                     "context": L_now, "traffic": measured_traffic(wl, L_now),
+                     "traffic_warm": measured_traffic(wl, L_now, TRAFFIC_WARM)},
         "prefill_compress": {"tokens": wl.T * wl.B, "ms": round(prefill_ms, 3),
                              "eager_ms": round(prefill_eager_ms, 3),
                              "timing": "CUDA-graph replay (device time); eager_ms adds the "
