@@ -11,18 +11,18 @@
 //  1. rebase_matrix_kernel: one CTA per (unit, side) stages P_old and P_new
 //     in shared memory and writes R^T (row j = column j of R) to the
 //     workspace in fp32.
-//  2. rebase_codes_kernel: one CTA per (page of a sequence, KV head).  It
-//     reads seq_len, skips pages past the sequence's latent tokens, brings
-//     the page's slab into shared memory as fp32 rows, multiplies each
-//     token's code by R for each side being re-based, rounds to the cache
-//     dtype once, and writes the slab back in place with 16-byte stores.
-//     The work is small next to a decode step's stream (every latent byte
-//     is read and written once, plus r multiply-adds per code element), so
-//     it runs on the CUDA cores.
+//  2. the codes, by the first of these that serves the cache:
+//     rebase_codes_tc (bf16 codes, re-based ranks multiples of 16: the
+//     fifth-generation tensor cores, two pages per MMA), rebase_codes_mma
+//     (bf16 codes: warp-level MMAs), rebase_codes_kernel (fp32 codes, or
+//     when neither plan fits: CUDA cores, one CTA per page).  Each reads
+//     every latent byte once and writes it back once, rounding to the cache
+//     dtype once.
 #include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace lrkv {
 
@@ -504,6 +504,435 @@ __global__ void __launch_bounds__(kRbThreads, 1) rebase_codes_mma(RebaseArgs a, 
   }
 }
 
+// ---- bf16 codes on the fifth-generation tensor cores
+// rebase_codes_tc: persistent, one CTA per SM.  The latent pages of every
+// unit are laid end to end and each CTA takes an equal contiguous range,
+// walked as jobs of one or two pages of one unit.  The chunk-major slab of a
+// page ([chunk of 8 codes][64 tokens][16 bytes]) is already the K-major
+// layout of 8 x 16-byte core matrices a tensor-memory MMA reads without
+// swizzle; the two pages of a job are interleaved chunk by chunk
+// ([chunk][page][64][16 B]) so that they form one M = 128 operand: core
+// matrices 128 bytes apart along the tokens (SBO) and 2 KB apart along the
+// codes (LBO).
+//  * warp 0, one lane: the producer.  Per job it copies each page's chunks
+//    (1 KB each) into a stage with bulk copies, completing on an mbarrier.
+//  * warp 1: the MMA issuer.  Per job and re-based side, c'^T = R c^T as
+//    tcgen05.mma (M 128 tokens, N = rank rounded up to 16, K 16) with R
+//    split into hi + lo bf16 halves (about 16 mantissa bits), both into the
+//    same fp32 accumulator in tensor memory (up to four in flight).
+//  * warps 2..5: the epilogue.  One token row per thread (tensor-memory lane
+//    = row), tcgen05.ld, rounded to bf16 once, 16-byte stores straight back
+//    into the row's page; rows past a page's latent tokens are not written.
+//  * warp 6: the R warp.  R^T of each unit of the range (fp32, from the
+//    first launch) as hi/lo bf16 rows [k chunk][n][16 B] into one of two
+//    buffers, once the MMAs of the unit before last are done.
+// Every wait is bounded; on a timeout the CTA raises a shared flag, every
+// role leaves its loop, the producer waits (bounded) for its copies in
+// flight, and tensor memory is freed before the CTA exits.
+constexpr int kRtThreads = 224;
+constexpr int kRtMaxStages = 10;
+constexpr int kRtWarp = 6;
+
+__host__ __device__ inline int rt_r16(int r) { return (r + 15) / 16 * 16; }
+// Tensor-memory columns of one accumulator (both sides), and of the allocation.
+__host__ __device__ inline int rt_acc_cols(int rk, int rv) { return rt_r16(rk) + rt_r16(rv); }
+// Accumulators in flight: as many as fit the 512 tensor-memory columns, at
+// most four (the MMA runs that many jobs ahead of the epilogue).
+__host__ __device__ inline int rt_nacc(int rk, int rv) {
+  return min(4, 512 / rt_acc_cols(rk, rv));
+}
+__host__ __device__ inline int rt_tmem_cols(int rk, int rv) {
+  int n = 32;
+  while (n < rt_nacc(rk, rv) * rt_acc_cols(rk, rv)) n *= 2;
+  return n;
+}
+// Job slots of the metadata ring: the producer runs at most NS + 4 jobs
+// ahead of the epilogue (NS stages, at most four accumulators), so NS + 5
+// slots are never overwritten before the epilogue has read them.
+__host__ __device__ inline int rt_slots(int NS) { return NS + 5; }
+struct RtPlan {
+  int ring, rbuf, rsize, rk_lo, rv_hi, rv_lo, bars, meta, start, misc, total;
+};
+// R buffer: R_k^T hi, lo ([rk/8][rk16][16 B] each), then R_v^T hi, lo.
+__host__ __device__ inline RtPlan rt_plan(int NS, int rk, int rv, int B) {
+  RtPlan p;
+  const int stage = 2 * kLatPage * (rk + rv) * 2;
+  p.ring = 0;
+  const int kb = (rk / 8) * rt_r16(rk) * 16, vb = (rv / 8) * rt_r16(rv) * 16;
+  p.rk_lo = kb;
+  p.rv_hi = 2 * kb;
+  p.rv_lo = 2 * kb + vb;
+  p.rsize = 2 * kb + 2 * vb;
+  p.rbuf = NS * stage;
+  p.bars = p.rbuf + 2 * p.rsize;
+  // full, empty, accf[4], acce[4], rfull, rfree, mdone, then mfull per job slot
+  p.meta = p.bars + (2 * NS + 8 + 4 + 1 + rt_slots(NS)) * 8;
+  p.start = p.meta + rt_slots(NS) * 8 * 4;      // per job slot: pages[2], rows[2], kvh
+  p.misc = p.start + ((B + 1 + 3) / 4 * 4) * 4;
+  p.total = p.misc + 16;
+  return p;
+}
+
+__global__ void __launch_bounds__(kRtThreads, 1) rebase_codes_tc(RebaseArgs a, int NS) {
+  using bf16 = __nv_bfloat16;
+  extern __shared__ __align__(1024) uint8_t rt_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(rt_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const RtPlan pl = rt_plan(NS, a.rk, a.rv, a.B);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + pl.bars);
+  uint64_t* empty = full + NS;
+  uint64_t* accf = empty + NS;   // [4]
+  uint64_t* acce = accf + 4;     // [4]
+  uint64_t* rfull = acce + 4;    // [2]
+  uint64_t* rfree = rfull + 2;   // [2]
+  uint64_t* mdone = rfree + 2;
+  uint64_t* mfull = mdone + 1;   // [NM] job metadata written
+  int* meta = reinterpret_cast<int*>(sm + pl.meta);  // [NM][8]
+  const int NM = rt_slots(NS);
+  int* start = reinterpret_cast<int*>(sm + pl.start);
+  uint32_t* taddr_slot = reinterpret_cast<uint32_t*>(sm + pl.misc);
+  volatile int* fail = reinterpret_cast<volatile int*>(sm + pl.misc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NJ = a.rk + a.rv, nch = NJ / 8, stage_bytes = 2 * kLatPage * NJ * 2;
+  const bool on_k = a.Pk_old != nullptr, on_v = a.Pv_old != nullptr;
+
+  // page prefix over sequences, one warp
+  if (warp == 0) {
+    const int per = (a.B + 31) / 32;
+    const int b0 = min(a.B, lane * per), b1 = min(a.B, b0 + per);
+    int own = 0;
+    for (int b = b0; b < b1; ++b) own += rb_pages(a, b) * a.H_kv;
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int e = incl - own;
+    for (int b = b0; b < b1; ++b) {
+      start[b] = e;
+      e += rb_pages(a, b) * a.H_kv;
+    }
+    if (lane == 31) start[a.B] = incl;
+  }
+  if (tid == 32) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&accf[i], 1);
+      mbar_init(&acce[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&rfull[i], 1);
+      mbar_init(&rfree[i], 1);
+    }
+    mbar_init(mdone, 1);
+    for (int i = 0; i < NM; ++i) mbar_init(&mfull[i], 1);
+    *fail = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  const int total = start[a.B];
+  const int q = total / (int)gridDim.x, rem = total - q * (int)gridDim.x;
+  const int lo = blockIdx.x * q + (blockIdx.x * rem) / gridDim.x;
+  const int hi = (blockIdx.x + 1) * q + ((blockIdx.x + 1) * rem) / gridDim.x;
+  if (lo >= hi) return;  // uniform across the CTA
+  auto locate = [&](int k, int& b, int& kvh, int& p, int& pages) {
+    int l = 0, h = a.B;
+    while (h - l > 1) {
+      const int mid = (l + h) >> 1;
+      if (start[mid] <= k) l = mid; else h = mid;
+    }
+    b = l;
+    pages = (start[b + 1] - start[b]) / a.H_kv;
+    const int r = k - start[b];
+    kvh = r / pages;
+    p = r - kvh * pages;
+  };
+  // job j starts at page k and holds two pages when the next page of the
+  // range is in the same unit; every role walks the jobs the same way
+  auto job_pages = [&](int k) {
+    int b, kvh, p, pages;
+    locate(k, b, kvh, p, pages);
+    return (k + 1 < hi && p + 1 < pages) ? 2 : 1;
+  };
+
+  const int tcols = rt_tmem_cols(a.rk, a.rv), acols = rt_acc_cols(a.rk, a.rv);
+  const int nacc = rt_nacc(a.rk, a.rv);
+  if (warp == 1) {
+    tmem_alloc(taddr_slot, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *taddr_slot;
+
+  // R^T of unit `unit` as hi/lo bf16 rows of the canonical layout: element
+  // (n, k) of side sd at chunk k / 8, row n, half-word k % 8
+  auto build_r = [&](int unit, int buf, int t, int nt) {
+    for (int sd = 0; sd < 2; ++sd) {
+      if (!(sd ? on_v : on_k)) continue;
+      const int r = sd ? a.rv : a.rk, R16 = rt_r16(r);
+      const float* Rt = (sd ? a.Rv : a.Rk) + (size_t)unit * r * r;  // Rt[k][n] = R[n][k]
+      uint8_t* hb = sm + pl.rbuf + buf * pl.rsize + (sd ? pl.rv_hi : 0);
+      uint8_t* lb = sm + pl.rbuf + buf * pl.rsize + (sd ? pl.rv_lo : pl.rk_lo);
+      // item = (k chunk kc, row n): 8 values R[n][8 kc .. 8 kc + 7]
+      for (int it = t; it < (r / 8) * R16; it += nt) {
+        const int kc = it / R16, n = it - kc * R16;
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = n < r ? __ldcg(Rt + (size_t)(8 * kc + e) * r + n) : 0.f;
+        uint32_t h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          h[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+          l[e] = pack_bf16x2(x[2 * e] - bf_lo(h[e]), x[2 * e + 1] - bf_hi(h[e]));
+        }
+        const size_t off = ((size_t)kc * R16 + n) * 16;
+        *reinterpret_cast<uint4*>(hb + off) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(lb + off) = make_uint4(l[0], l[1], l[2], l[3]);
+      }
+    }
+    fence_proxy_async_smem();
+  };
+  auto unit_of = [&](int k) {
+    int b, kvh, p, pages;
+    locate(k, b, kvh, p, pages);
+    return b * a.H_kv + kvh;
+  };
+  // the R of the range's first two units, built by every thread before the stream
+  int nfirst = 0;
+  {
+    int cur = -1;
+    for (int k = lo; k < hi && nfirst < 2; ++k) {
+      int b, kvh, p, pages;
+      locate(k, b, kvh, p, pages);
+      const int unit = b * a.H_kv + kvh;
+      if (unit == cur) continue;
+      cur = unit;
+      build_r(unit, nfirst, tid, kRtThreads);
+      ++nfirst;
+      k += pages - p - 1;  // to the unit's last page
+    }
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int m = 0; m < nfirst; ++m) mbar_arrive(&rfull[m]);
+
+  const bf16* codes_in = static_cast<const bf16*>(a.codes);
+  if (warp == 0) {
+    // ---------------- producer: the warp resolves pages 32 at a time (lane l
+    // holds the block-table entry, latent rows and KV head of page base + l;
+    // the next batch's loads are in flight while this one is issued); lane 0
+    // issues the copies and publishes each job's pages for the epilogue
+    const uint64_t pol = l2_evict_first_policy();
+    auto resolve = [&](int kk, int& pg, int& rw, int& kv) {
+      pg = -1;
+      rw = 0;
+      kv = 0;
+      if (kk >= hi) return;
+      int b, p, pages;
+      locate(kk, b, kv, p, pages);
+      const int L = max(0, __ldcg(a.seq_len + b));
+      rw = min(kLatPage, split_tokens(L, a.n_sink, a.W).lat - p * kLatPage);
+      const int page = __ldg(a.bt + (size_t)b * a.maxp + p);
+      pg = (page >= 0 && page < a.num_pages) ? page : -1;
+    };
+    int base = lo, cpg, crw, ckv, npg, nrw, nkv;
+    resolve(base + lane, cpg, crw, ckv);
+    resolve(base + 32 + lane, npg, nrw, nkv);
+    int issued = 0, j = 0;
+    for (int k = lo; k < hi; ++j) {
+      const int np = job_pages(k);
+      int pg[2] = {-1, -1}, rw[2] = {0, 0}, kvh = 0;
+      for (int i = 0; i < 2; ++i) {
+        const int o = k + i - base;  // < 64: k < base + 32
+        const int x = __shfl_sync(0xffffffffu, o < 32 ? cpg : npg, o & 31);
+        const int y = __shfl_sync(0xffffffffu, o < 32 ? crw : nrw, o & 31);
+        const int z = __shfl_sync(0xffffffffu, o < 32 ? ckv : nkv, o & 31);
+        if (i < np) {
+          pg[i] = x;
+          rw[i] = y;
+          kvh = i == 0 ? z : kvh;
+        }
+      }
+      const int s = j % NS, n = j / NS;
+      int ok = 1;
+      if (lane == 0) {
+        if (n > 0 && !tc_wait(&empty[s], (n - 1) & 1, fail)) {
+          ok = 0;
+        } else {
+          if (pg[0] < 0 || (np > 1 && pg[1] < 0)) *a.err = kErrBadPage;
+          const uint32_t bytes = (uint32_t)(((pg[0] >= 0) + (pg[1] >= 0)) * nch * 1024);
+          mbar_arrive_expect_tx(&full[s], bytes);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      // the job's 1 KB chunk copies, spread over the lanes
+      uint8_t* dst = sm + pl.ring + (size_t)s * stage_bytes;
+      for (int x = lane; x < np * nch; x += 32) {
+        const int i = x / nch, c = x - i * nch;
+        if (pg[i] >= 0)
+          bulk_g2s_hint(dst + (size_t)c * 2048 + i * 1024,
+                        codes_in + ((size_t)pg[i] * a.H_kv + kvh) * kLatPage * NJ +
+                            (size_t)c * kLatPage * 8,
+                        1024, &full[s], pol);
+      }
+      if (lane == 0) {
+        int* m = meta + (j % NM) * 8;
+        m[0] = pg[0];
+        m[1] = pg[1];
+        m[2] = rw[0];
+        m[3] = rw[1];
+        m[4] = kvh;
+        mbar_arrive(&mfull[j % NM]);
+      }
+      issued = j + 1;
+      k += np;
+      if (k >= base + 32) {
+        base += 32;
+        cpg = npg; crw = nrw; ckv = nkv;
+        resolve(base + 32 + lane, npg, nrw, nkv);
+      }
+    }
+    // no copy may still be landing when the CTA exits
+    if (lane == 0)
+      for (int s = 0; s < NS && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / NS) * NS;
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(&full[s], (last / NS) & 1) && global_ns() - t0 < kTcTimeoutNs) {
+        }
+      }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    const uint32_t ring0 = smem_u32(sm + pl.ring);
+    const uint32_t rb0 = smem_u32(sm + pl.rbuf);
+    int cur_unit = -1, m = -1, j = 0;
+    for (int k = lo; k < hi; ++j) {
+      if (__shfl_sync(0xffffffffu, *fail, 0)) break;
+      const int np = job_pages(k);
+      const int unit = unit_of(k);
+      if (unit != cur_unit) {
+        if (m >= 0 && lane == 0) tc_commit(&rfree[m & 1]);
+        ++m;
+        cur_unit = unit;
+        if (!tc_wait_warp(&rfull[m & 1], (m >> 1) & 1, fail, lane)) break;
+      }
+      const int s = j % NS, n = j / NS, buf = j % nacc, u = j / nacc;
+      if (!tc_wait_warp(&full[s], n & 1, fail, lane)) break;
+      if (u > 0 && !tc_wait_warp(&acce[buf], (u - 1) & 1, fail, lane)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sa = ring0 + s * stage_bytes;
+        const uint32_t rb = rb0 + (m & 1) * pl.rsize;
+        for (int sd = 0; sd < 2; ++sd) {
+          if (!(sd ? on_v : on_k)) continue;
+          const int r = sd ? a.rv : a.rk, R16 = rt_r16(r), cb = sd ? a.rk / 8 : 0;
+          const uint32_t d = tmem + buf * acols + (sd ? rt_r16(a.rk) : 0);
+          const uint32_t idesc = tc_idesc(R16);
+          const uint32_t hb = rb + (sd ? pl.rv_hi : 0), lb = rb + (sd ? pl.rv_lo : pl.rk_lo);
+          for (int ks = 0; ks < r / 16; ++ks) {
+            // A: codes chunks cb + 2 ks, + 1; B: R^T chunks 2 ks, + 1
+            const uint64_t ad = interleave_desc(sa + (cb + 2 * ks) * 2048, 2048, 128);
+            const uint32_t bo = (2 * ks) * R16 * 16;
+            tc_mma(d, ad, interleave_desc(hb + bo, R16 * 16, 128), idesc, ks > 0 ? 1u : 0u);
+            tc_mma(d, ad, interleave_desc(lb + bo, R16 * 16, 128), idesc, 1u);
+          }
+        }
+        tc_commit(&empty[s]);
+        tc_commit(&accf[buf]);
+      }
+      __syncwarp();
+      k += np;
+    }
+    // every MMA issued has completed before tensor memory is freed
+    if (lane == 0) {
+      tc_commit(mdone);
+      const uint64_t t0 = global_ns();
+      while (!mbar_try_wait(mdone, 0) && global_ns() - t0 < kTcTimeoutNs) {
+      }
+    }
+    __syncwarp();
+  } else if (warp == kRtWarp) {
+    // ---------------- R warp: units 2, 3, ... of the range, in order
+    int cur_unit = -1, m = -1;
+    for (int k = lo; k < hi; ++k) {
+      int b, kvh, p, pages;
+      locate(k, b, kvh, p, pages);
+      const int unit = b * a.H_kv + kvh;
+      k += pages - p - 1;  // to the unit's last page
+      if (unit == cur_unit) continue;
+      cur_unit = unit;
+      if (++m < nfirst) continue;  // built by the whole CTA
+      if (!tc_wait_warp(&rfree[m & 1], ((m - 2) >> 1) & 1, fail, lane)) break;
+      build_r(unit, m & 1, lane, 32);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfull[m & 1]);
+    }
+  } else {
+    // ---------------- epilogue: tensor-memory lanes 32 qd .. 32 qd + 31 = token rows
+    const int qd = warp & 3, row = 32 * qd + lane, pi = row >> 6, t = row & 63;
+    bf16* codes = static_cast<bf16*>(a.codes);
+    int j = 0;
+    for (int k = lo; k < hi; ++j) {
+      const int np = job_pages(k);
+      const int buf = j % nacc, u = j / nacc;
+      // the job's pages, as the producer resolved them
+      if (!tc_wait_warp(&mfull[j % NM], (j / NM) & 1, fail, lane)) break;
+      __syncwarp();  // lane 0's acquire orders the other lanes' reads too
+      const int* m = meta + (j % NM) * 8;
+      const int page = pi < np ? m[pi] : -1, rows = m[2 + pi], kvh = m[4];
+      if (!tc_wait_warp(&accf[buf], u & 1, fail, lane)) break;
+      tc_fence_after();
+      const bool write = page >= 0 && t < rows;
+      bf16* dst = codes + ((size_t)(page >= 0 ? page : 0) * a.H_kv + kvh) * kLatPage * NJ;
+      for (int sd = 0; sd < 2; ++sd) {
+        if (!(sd ? on_v : on_k)) continue;
+        const int r = sd ? a.rv : a.rk, cb = sd ? a.rk / 8 : 0;
+        const uint32_t tb = tmem + ((uint32_t)(32 * qd) << 16) + buf * acols +
+                            (sd ? rt_r16(a.rk) : 0);
+        uint32_t v[8][16];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (16 * c < r) tmem_ld16_async(tb + 16 * c, v[c]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (16 * c < r) tmem_wait_tie(v[c]);
+        if (write) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int c8 = 16 * c + 8 * h;  // r is a multiple of 8
+              if (c8 < r) {
+                const uint4 w = make_uint4(
+                    pack_bf16x2(__uint_as_float(v[c][8 * h + 0]), __uint_as_float(v[c][8 * h + 1])),
+                    pack_bf16x2(__uint_as_float(v[c][8 * h + 2]), __uint_as_float(v[c][8 * h + 3])),
+                    pack_bf16x2(__uint_as_float(v[c][8 * h + 4]), __uint_as_float(v[c][8 * h + 5])),
+                    pack_bf16x2(__uint_as_float(v[c][8 * h + 6]), __uint_as_float(v[c][8 * h + 7])));
+                *reinterpret_cast<uint4*>(dst + ((size_t)(cb + c8 / 8) * kLatPage + t) * 8) = w;
+              }
+            }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[buf]);
+      k += np;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
+  }
+}
+
 template <typename T>
 int launch_rebase_t(const RebaseArgs& a, cudaStream_t st) {
   const int rmax = a.rk > a.rv ? a.rk : a.rv;
@@ -519,8 +948,23 @@ int launch_rebase_t(const RebaseArgs& a, cudaStream_t st) {
     DevInfo info;
     rc = current_device_info(dev, info);
     if (rc != LRKV_OK) return rc;
-    // one CTA per SM; each consumer group keeps one stage back for its
-    // store, so at least two stages per group
+    // tensor-memory kernel when both re-based ranks are multiples of 16 and
+    // its plan fits: one CTA per SM, as many stages as fit
+    const bool k16 = !a.Pk_old || a.rk % 16 == 0, v16 = !a.Pv_old || a.rv % 16 == 0;
+    if (k16 && v16) {
+      int NT = kRtMaxStages;
+      while (NT >= 2 && (size_t)rt_plan(NT, a.rk, a.rv, a.B).total + 1024 > (size_t)info.optin)
+        --NT;
+      if (NT >= 2) {
+        rc = prepare_kernel((const void*)rebase_codes_tc, false);
+        if (rc != LRKV_OK) return rc;
+        const size_t smem = (size_t)rt_plan(NT, a.rk, a.rv, a.B).total + 1024;
+        rebase_codes_tc<<<info.sms, kRtThreads, smem, st>>>(a, NT);
+        return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+      }
+    }
+    // otherwise warp-level MMAs: one CTA per SM; each consumer group keeps
+    // one stage back for its store, so at least two stages per group
     int NS = kRbMaxStages;
     while (NS >= 2 * kRbGroups && rb_plan(NS, a.rk, a.rv, a.B).total > info.optin) --NS;
     if (NS >= 2 * kRbGroups) {
