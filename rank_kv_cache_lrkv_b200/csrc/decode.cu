@@ -82,6 +82,8 @@ struct DecodeArgs {
   int rw;              // latent record width per head: rv, or rk + rv (amortised)
   int wait_first;      // 1: the previous grid (a step's append) writes the cache
   int fold_split;      // q-fold CTAs per unit (each folds at most 32 columns)
+  int combine;         // 1: one ring-space record per (CTA, unit), the consumer
+                       // warps' records combined in shared memory; 0: one per warp
 };
 
 constexpr int kModePlain = 0;  // bf16 / fp32 latent codes
@@ -1194,7 +1196,9 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
     auto release = [&](int tt) {
       if (lane == 0) mbar_arrive(&empty[(tt - lo) % a.NS]);
     };
-    float* rec = wrec + w * rec_stride;  // this warp's record, combined below
+    // this warp's record: combined below into the CTA's, or written as is
+    float* rec = a.combine ? wrec + w * rec_stride
+                           : part + ((size_t)(unit + c) * kConsumers + w) * rec_stride;
     if constexpr (kTensorTiles) {
       constexpr int TT = kDense ? kFrTile : kLatPage;
       QFrag<KS> qf;
@@ -1278,13 +1282,17 @@ __global__ void __maxnreg__(168) split_kernel(DecodeArgs a) {
       }
       write_record<T, G>(rec, rvd, TS, ncv, m, l, acc, lane);
     }
-    // The CTA's one record for (unit, space).  Every consumer warp passes
-    // here once per unit; a failure seen by any of them ends them all.
-    if (named_bar_any(kBarRecords, 32 * kConsumers, *fail != 0)) break;
-    combine_warp_records<G>(wrec, rec_stride, rvd, part + (size_t)(unit + c) * rec_stride,
-                            threadIdx.x - 32 * kFirstConsumer);
-    // a warp without tiles in the next unit writes its next record at once
-    named_bar(kBarRecords, 32 * kConsumers);
+    if (a.combine) {
+      // The CTA's one record for (unit, space).  Every consumer warp passes
+      // here once per unit; a failure seen by any of them ends them all.
+      if (named_bar_any(kBarRecords, 32 * kConsumers, *fail != 0)) break;
+      combine_warp_records<G>(wrec, rec_stride, rvd, part + (size_t)(unit + c) * rec_stride,
+                              threadIdx.x - 32 * kFirstConsumer);
+      // a warp without tiles in the next unit writes its next record at once
+      named_bar(kBarRecords, 32 * kConsumers);
+    } else if (*fail) {
+      break;
+    }
     t = ce;
   }
 }
@@ -1412,7 +1420,9 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(DecodeArgs a) {
     c0[sp] = cta_of(us, total[sp], Ce);
     ncta[sp] = cta_of(us + tiles - 1, total[sp], Ce) - c0[sp] + 1;
   }
-  const int per0 = 1, per1 = 1;  // one record per (CTA, unit) in each space
+  // records per (CTA, unit): the anchor warp writes one; the consumers one
+  // (combined) or one per warp
+  const int per0 = a.combine ? 1 : kConsumers, per1 = (anchors || a.combine) ? 1 : kConsumers;
   const int S0 = H + G * a.rw, S1 = H + G * kHeadDim;  // floats per record
   const int n0 = ncta[0] * per0, n1 = ncta[1] * per1;
   const float* src0 = a.part_lat + (size_t)(unit + c0[0]) * per0 * S0;
@@ -1625,9 +1635,10 @@ static int plan_decode(int B, int H_kv, int H_q, int rk, int rv, bool has_lat, b
   p.off_qfr = off;  off = al(off + (size_t)B * H_q * (has_fr ? kHeadDim : 0) * 4);
   const size_t slots = (size_t)(U + p.C - 1);
   p.off_lat = off;
-  off = al(off + (has_lat ? slots * (hdr_floats(G) + G * rw) * 4 : 0));
+  off = al(off + (has_lat ? slots * kConsumers * (hdr_floats(G) + G * rw) * 4 : 0));
   p.off_fr = off;
-  off = al(off + (has_fr ? slots * (hdr_floats(G) + G * kHeadDim) * 4 : 0));
+  off = al(off + (has_fr ? slots * (anchors ? 1 : kConsumers) * (hdr_floats(G) + G * kHeadDim) * 4
+                         : 0));
   p.total = off;
   return LRKV_OK;
 }
@@ -1748,6 +1759,12 @@ static int decode_args(const DecodeLaunch& L, DecodeArgs& a, Plan& p) {
   a.A = L.dtype == LRKV_BF16_VA ? L.A : nullptr;
   a.wait_first = 0;
   a.fold_split = std::max(kFoldSplit, (L.rk + 31) / 32);
+  // Combine the consumer warps' records inside each CTA when a unit spans
+  // at least eight CTAs: then the merge would otherwise fold 64 or more
+  // records per unit, and its latency chain grows with them (B = 1 at 16K:
+  // 20 -> 15 us per call); with fewer CTAs per unit the per-unit barriers
+  // cost more than they save.
+  a.combine = (long long)L.B * L.H_kv * 8 <= p.C ? 1 : 0;
   return LRKV_OK;
 }
 
