@@ -19,7 +19,8 @@
 //  * warp 0, one lane: the tensor-memory-access producer.  Per job it loads
 //    the tile's 128 rows of one side as two boxes of 64 dims (128-byte
 //    swizzle) through a tensor map over this GPU's own input (no cluster,
-//    no multicast) into a ring of 32 KB stages, completing on mbarriers.
+//    no multicast) into a ring of 32 KB stages, completing on mbarriers,
+//    and prefetches the rows of the jobs up to eight ahead into L2.
 //  * warp 6: the basis warp.  For each unit of the CTA's range, in order, it
 //    writes P^T of the unit (bf16) into one of two shared-memory buffers in
 //    the 128-byte-swizzled K-major layout, fences it for the async proxy
@@ -58,6 +59,7 @@ constexpr int kTcThreads = 224;                    // 7 warps
 constexpr int kTcHalfBytes = kTcRows * 128;        // one 64-dim box: 128 rows x 128 B
 constexpr int kTcStageBytes = 2 * kTcHalfBytes;    // one side of one tile
 constexpr int kTcMaxStages = 6;
+constexpr int kTcPrefetch = 8;                     // jobs whose rows are prefetched to L2
 constexpr int kBasisWarp = 6;
 constexpr int kTcAccCols = 128;                    // TMEM columns per accumulator
 constexpr int kTcAcc = 4;                          // accumulators in flight
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == 0) {
     // ---------------- producer
-    int issued = 0;
+    int issued = 0, pf = 0;
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
       for (int j = 0; j < njobs; ++j) {
@@ -247,6 +249,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_load_4d(dst, tm, 0, t0, kvh, b, &full[s], pol);
         tma_load_4d(dst + kTcHalfBytes, tm, 64, t0, kvh, b, &full[s], pol);
         issued = j + 1;
+        // the rows of the jobs up to kTcPrefetch ahead go to L2 now, so
+        // their loads land from L2 when a stage frees
+        for (; pf <= j + kTcPrefetch && pf < njobs; ++pf) {
+          if (pf < NS) continue;  // loaded right away
+          int pb, pk, pi;
+          locate(lo + pf / sides, pb, pk, pi);
+          const CUtensorMap* ptm = (pf % sides) ? &tmV : &tmK;
+          tma_prefetch_4d(ptm, 0, srlo[pb] + pi * kTcRows, pk, pb);
+          tma_prefetch_4d(ptm, 64, srlo[pb] + pi * kTcRows, pk, pb);
+        }
       }
       // no copy may still be landing when the CTA exits (immediate when the
       // MMA warp consumed them all)

@@ -1664,8 +1664,8 @@ size_t decode_workspace_bytes(int B, int H_kv, int H_q, int rk, int rv, bool has
   return p.total;
 }
 
-static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem,
-                              cudaStream_t st, void** args) {
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       void** args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;

@@ -19,6 +19,12 @@ int current_device_info(int& dev, DevInfo& info);
 // carveout.  Later calls return at once.
 int prepare_kernel(const void* fn, bool max_carveout);
 
+// Launch fn as the programmatic dependent of the stream's previous kernel
+// (it may start before that grid ends and waits for it with
+// griddepcontrol.wait before reading what that grid writes).
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       void** args);
+
 struct DecodeLaunch {
   int B, H_kv, H_q, dtype;
   const int* seq_len;

@@ -8,9 +8,9 @@
 // (sequence, KV head) unit and side).
 //
 // Two launches:
-//  1. rebase_matrix_kernel: one CTA per (unit, side) stages P_old and P_new
-//     in shared memory and writes R^T (row j = column j of R) to the
-//     workspace in fp32.
+//  1. rebase_matrix_kernel: eight CTAs per (unit, side), each staging P_new
+//     and its eighth of P_old's columns in shared memory, write R^T (row j =
+//     column j of R) to the workspace in fp32.
 //  2. the codes, by the first of these that serves the cache:
 //     rebase_codes_tc (bf16 codes, re-based ranks multiples of 16: the
 //     fifth-generation tensor cores, two pages per MMA), rebase_codes_mma
@@ -41,39 +41,52 @@ struct RebaseArgs {
   float *Rk, *Rv;  // [B][H_kv][r][r], R^T per unit
 };
 
-// Shared memory of rebase_matrix_kernel for rank r: both bases [128][r] fp32.
-inline size_t matrix_smem_bytes(int r) { return (size_t)2 * kHeadDim * r * 4; }
+// R^T rows are split over kRmSlices CTAs per (unit, side), so the small
+// products spread over the GPU instead of running as one long loop per unit.
+constexpr int kRmSlices = 8;
+__host__ __device__ inline int rm_rows(int r) { return (r + kRmSlices - 1) / kRmSlices; }
+// Shared memory of rebase_matrix_kernel for rank r: the new basis [128][r]
+// and the slice's columns of the old one [128][rm_rows(r)], fp32.
+inline size_t matrix_smem_bytes(int r) { return (size_t)kHeadDim * (r + rm_rows(r)) * 4; }
 
 // R^T[j][i] = sum_d P_new[d][i] P_old[d][j] for unit (blockIdx.y, blockIdx.x),
-// side blockIdx.z (0 keys, 1 values).
-__global__ void __launch_bounds__(kRebaseThreads, 1) rebase_matrix_kernel(RebaseArgs a) {
+// side blockIdx.z / kRmSlices (0 keys, 1 values), rows j of slice
+// blockIdx.z % kRmSlices.  The re-basing pass that follows is launched as its
+// programmatic dependent and waits for this grid before reading R.
+__global__ void __launch_bounds__(kRebaseThreads) rebase_matrix_kernel(RebaseArgs a) {
   extern __shared__ __align__(16) float msm[];
-  const int kvh = blockIdx.x, b = blockIdx.y, side = blockIdx.z, tid = threadIdx.x;
+  pdl_trigger();
+  const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int side = blockIdx.z / kRmSlices, slice = blockIdx.z - side * kRmSlices;
   const float* Po = side ? a.Pv_old : a.Pk_old;
   const float* Pn = side ? a.Pv_new : a.Pk_new;
   if (!Po) return;
-  const int r = side ? a.rv : a.rk;
+  const int r = side ? a.rv : a.rk, js = rm_rows(r);
+  const int j0 = slice * js, nj = min(r, j0 + js) - j0;
+  if (nj <= 0) return;
   const size_t base = (size_t)b * a.basis_bs + (size_t)kvh * kHeadDim * r;
-  float* so = msm;                  // [128][r] old basis
-  float* sn = msm + kHeadDim * r;   // [128][r] new basis
+  float* sn = msm;                  // [128][r] new basis
+  float* so = msm + kHeadDim * r;   // [128][js] old basis, columns j0 ..
   const int n4 = kHeadDim * r / 4;
-  for (int x = tid; x < n4; x += kRebaseThreads) {
-    reinterpret_cast<float4*>(so)[x] = __ldg(reinterpret_cast<const float4*>(Po + base) + x);
+  for (int x = tid; x < n4; x += kRebaseThreads)
     reinterpret_cast<float4*>(sn)[x] = __ldg(reinterpret_cast<const float4*>(Pn + base) + x);
+  for (int x = tid; x < kHeadDim * nj; x += kRebaseThreads) {
+    const int d = x / nj, jj = x - d * nj;
+    so[d * js + jj] = __ldg(Po + base + (size_t)d * r + j0 + jj);
   }
   __syncthreads();
   float* Rt = (side ? a.Rv : a.Rk) + ((size_t)b * a.H_kv + kvh) * r * r;
   // thread -> (row j, column i) of R^T; consecutive threads take consecutive
   // i, so the new basis is read along its rows and the old one broadcast
-  for (int x = tid; x < r * r; x += kRebaseThreads) {
-    const int j = x / r, i = x - j * r;
+  for (int x = tid; x < nj * r; x += kRebaseThreads) {
+    const int jj = x / r, i = x - jj * r;
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll 4
     for (int d = 0; d < kHeadDim; d += 2) {
-      s0 = fmaf(sn[d * r + i], so[d * r + j], s0);
-      s1 = fmaf(sn[(d + 1) * r + i], so[(d + 1) * r + j], s1);
+      s0 = fmaf(sn[d * r + i], so[d * js + jj], s0);
+      s1 = fmaf(sn[(d + 1) * r + i], so[(d + 1) * js + jj], s1);
     }
-    Rt[x] = s0 + s1;
+    Rt[(size_t)(j0 + jj) * r + i] = s0 + s1;
   }
 }
 
@@ -514,8 +527,10 @@ __global__ void __launch_bounds__(kRbThreads, 1) rebase_codes_mma(RebaseArgs a, 
 // ([chunk][page][64][16 B]) so that they form one M = 128 operand: core
 // matrices 128 bytes apart along the tokens (SBO) and 2 KB apart along the
 // codes (LBO).
-//  * warp 0, one lane: the producer.  Per job it copies each page's chunks
-//    (1 KB each) into a stage with bulk copies, completing on an mbarrier.
+//  * warp 0: the producer.  Per job its lanes copy each page's chunks (1 KB
+//    each) into a stage with bulk copies, completing on an mbarrier.  The
+//    kernel is the programmatic dependent of the R launch: the producer
+//    streams pages at once, every other warp waits for that grid first.
 //  * warp 1: the MMA issuer.  Per job and re-based side, c'^T = R c^T as
 //    tcgen05.mma (M 128 tokens, N = rank rounded up to 16, K 16) with R
 //    split into hi + lo bf16 halves (about 16 mantissa bits), both into the
@@ -703,9 +718,12 @@ __global__ void __launch_bounds__(kRtThreads, 1) rebase_codes_tc(RebaseArgs a, i
     locate(k, b, kvh, p, pages);
     return b * a.H_kv + kvh;
   };
-  // the R of the range's first two units, built by every thread before the stream
+  // The R of the range's first two units, built before the stream by every
+  // warp but the producer: R comes from the grid this one depends on, the
+  // codes do not, so the producer starts copying pages at once.
   int nfirst = 0;
-  {
+  if (warp != 0) {
+    pdl_wait();
     int cur = -1;
     for (int k = lo; k < hi && nfirst < 2; ++k) {
       int b, kvh, p, pages;
@@ -713,14 +731,14 @@ __global__ void __launch_bounds__(kRtThreads, 1) rebase_codes_tc(RebaseArgs a, i
       const int unit = b * a.H_kv + kvh;
       if (unit == cur) continue;
       cur = unit;
-      build_r(unit, nfirst, tid, kRtThreads);
+      build_r(unit, nfirst, tid - 32, kRtThreads - 32);
       ++nfirst;
       k += pages - p - 1;  // to the unit's last page
     }
+    named_bar(1, kRtThreads - 32);
+    if (tid == 32)
+      for (int m = 0; m < nfirst; ++m) mbar_arrive(&rfull[m]);
   }
-  __syncthreads();
-  if (tid == 0)
-    for (int m = 0; m < nfirst; ++m) mbar_arrive(&rfull[m]);
 
   const bf16* codes_in = static_cast<const bf16*>(a.codes);
   if (warp == 0) {
@@ -940,7 +958,7 @@ int launch_rebase_t(const RebaseArgs& a, cudaStream_t st) {
   int rc = prepare_kernel((const void*)rebase_matrix_kernel, false);
   if (rc == LRKV_OK) rc = prepare_kernel((const void*)rebase_codes_kernel<T>, false);
   if (rc != LRKV_OK) return rc;
-  rebase_matrix_kernel<<<dim3(a.H_kv, a.B, 2), kRebaseThreads, ms, st>>>(a);
+  rebase_matrix_kernel<<<dim3(a.H_kv, a.B, 2 * kRmSlices), kRebaseThreads, ms, st>>>(a);
   if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
     // tensor-core pass: as many ring stages as fit beside R and the prefix
@@ -959,8 +977,11 @@ int launch_rebase_t(const RebaseArgs& a, cudaStream_t st) {
         rc = prepare_kernel((const void*)rebase_codes_tc, false);
         if (rc != LRKV_OK) return rc;
         const size_t smem = (size_t)rt_plan(NT, a.rk, a.rv, a.B).total + 1024;
-        rebase_codes_tc<<<info.sms, kRtThreads, smem, st>>>(a, NT);
-        return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+        void* args[] = {const_cast<RebaseArgs*>(&a), &NT};
+        return launch_pdl((const void*)rebase_codes_tc, dim3(info.sms), dim3(kRtThreads), smem,
+                          st, args) == cudaSuccess
+                   ? LRKV_OK
+                   : LRKV_ERR_CUDA;
       }
     }
     // otherwise warp-level MMAs: one CTA per SM; each consumer group keeps
