@@ -465,6 +465,17 @@ bool encode_rows(CUtensorMap* tm, const void* base, int n, int H_kv, int B,
 
 }  // namespace
 
+bool encode_tiled(CUtensorMap* tm, CUtensorMapDataType dt, int rank, const void* base,
+                  const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(tm, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 size_t bulk_tc_smem_bytes(int rk, int rv, int NS, int B, int NB) {
   return (size_t)tc_plan(NS, round16(rk), round16(rv), B, NB).total + 1024;
 }

@@ -18,6 +18,7 @@
 //     when neither plan fits: CUDA cores, one CTA per page).  Each reads
 //     every latent byte once and writes it back once, rounding to the cache
 //     dtype once.
+#include <cstring>
 #include <type_traits>
 
 #include "common.cuh"
@@ -527,8 +528,11 @@ __global__ void __launch_bounds__(kRbThreads, 1) rebase_codes_mma(RebaseArgs a, 
 // ([chunk][page][64][16 B]) so that they form one M = 128 operand: core
 // matrices 128 bytes apart along the tokens (SBO) and 2 KB apart along the
 // codes (LBO).
-//  * warp 0: the producer.  Per job its lanes copy each page's chunks (1 KB
-//    each) into a stage with bulk copies, completing on an mbarrier.  The
+//  * warp 0: the producer.  Per job one tensor load brings two consecutive
+//    pages (a tensor map over the pool whose dimensions, innermost first,
+//    are the 1 KB chunk row, the page, the chunk and the KV head lands them
+//    interleaved); other jobs' lanes copy each page's chunks (1 KB each) with
+//    bulk copies; both complete on the stage's mbarrier.  The
 //    kernel is the programmatic dependent of the R launch: the producer
 //    streams pages at once, every other warp waits for that grid first.
 //  * warp 1: the MMA issuer.  Per job and re-based side, c'^T = R c^T as
@@ -588,7 +592,8 @@ __host__ __device__ inline RtPlan rt_plan(int NS, int rk, int rv, int B) {
   return p;
 }
 
-__global__ void __launch_bounds__(kRtThreads, 1) rebase_codes_tc(RebaseArgs a, int NS) {
+__global__ void __launch_bounds__(kRtThreads, 1)
+    rebase_codes_tc(RebaseArgs a, int NS, const __grid_constant__ CUtensorMap tmC, int pair_tm) {
   using bf16 = __nv_bfloat16;
   extern __shared__ __align__(1024) uint8_t rt_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
@@ -789,15 +794,21 @@ __global__ void __launch_bounds__(kRtThreads, 1) rebase_codes_tc(RebaseArgs a, i
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      // the job's 1 KB chunk copies, spread over the lanes
       uint8_t* dst = sm + pl.ring + (size_t)s * stage_bytes;
-      for (int x = lane; x < np * nch; x += 32) {
-        const int i = x / nch, c = x - i * nch;
-        if (pg[i] >= 0)
-          bulk_g2s_hint(dst + (size_t)c * 2048 + i * 1024,
-                        codes_in + ((size_t)pg[i] * a.H_kv + kvh) * kLatPage * NJ +
-                            (size_t)c * kLatPage * 8,
-                        1024, &full[s], pol);
+      if (pair_tm && np == 2 && pg[0] >= 0 && pg[1] == pg[0] + 1) {
+        // consecutive pages: one tensor load of the box (1 KB chunk, page
+        // pair, every chunk) lands them already interleaved
+        if (lane == 0) tma_load_4d(dst, &tmC, 0, pg[0], 0, kvh, &full[s], pol);
+      } else {
+        // the job's 1 KB chunk copies, spread over the lanes
+        for (int x = lane; x < np * nch; x += 32) {
+          const int i = x / nch, c = x - i * nch;
+          if (pg[i] >= 0)
+            bulk_g2s_hint(dst + (size_t)c * 2048 + i * 1024,
+                          codes_in + ((size_t)pg[i] * a.H_kv + kvh) * kLatPage * NJ +
+                              (size_t)c * kLatPage * 8,
+                          1024, &full[s], pol);
+        }
       }
       if (lane == 0) {
         int* m = meta + (j % NM) * 8;
@@ -977,7 +988,25 @@ int launch_rebase_t(const RebaseArgs& a, cudaStream_t st) {
         rc = prepare_kernel((const void*)rebase_codes_tc, false);
         if (rc != LRKV_OK) return rc;
         const size_t smem = (size_t)rt_plan(NT, a.rk, a.rv, a.B).total + 1024;
-        void* args[] = {const_cast<RebaseArgs*>(&a), &NT};
+        // the code pool as [H_kv][chunk][page][1 KB chunk row] (dimensions
+        // innermost first: chunk row as 256 words, page, chunk, KV head), so
+        // a box of two pages lands as [chunk][page][1 KB]
+        CUtensorMap tmC;
+        memset(&tmC, 0, sizeof(tmC));
+        int pair_tm = 0;
+        if (a.num_pages >= 2) {
+          const int nch = (a.rk + a.rv) / 8;
+          const cuuint64_t slab = (cuuint64_t)kLatPage * (a.rk + a.rv) * 2;
+          const cuuint64_t dims[4] = {(cuuint64_t)kLatPage * 4, (cuuint64_t)a.num_pages,
+                                      (cuuint64_t)nch, (cuuint64_t)a.H_kv};
+          const cuuint64_t strides[3] = {slab * a.H_kv, (cuuint64_t)kLatPage * 16, slab};
+          const cuuint32_t box[4] = {(cuuint32_t)kLatPage * 4, 2, (cuuint32_t)nch, 1};
+          pair_tm = encode_tiled(&tmC, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.codes, dims,
+                                 strides, box)
+                        ? 1
+                        : 0;
+        }
+        void* args[] = {const_cast<RebaseArgs*>(&a), &NT, &tmC, &pair_tm};
         return launch_pdl((const void*)rebase_codes_tc, dim3(info.sms), dim3(kRtThreads), smem,
                           st, args) == cudaSuccess
                    ? LRKV_OK

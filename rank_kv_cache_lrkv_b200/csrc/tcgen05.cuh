@@ -12,6 +12,12 @@ namespace lrkv {
 
 constexpr unsigned long long kTcTimeoutNs = 2000000000ull;
 
+// A tiled tensor map (no interleave, no swizzle, element strides 1) through
+// the runtime's driver entry point; false when the driver lacks the entry
+// point or refuses the map.  strides: bytes, dimensions 1 .. rank - 1.
+bool encode_tiled(CUtensorMap* tm, CUtensorMapDataType dt, int rank, const void* base,
+                  const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box);
+
 // ---- PTX of the fifth-generation tensor cores and the tensor-memory copies
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t cols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

@@ -50,11 +50,12 @@ def _row_err(a, b):
 
 
 def _case(lrkv, *, dtype, B, H_kv, G, rk, rv, n_sink, W, lens, per_seq, sides="kv",
-          same_span=False, seed=0):
+          same_span=False, seed=0, contiguous=False):
     gen = torch.Generator().manual_seed(seed)
     T = max(lens)
     perm = torch.randperm(B * math.ceil(max(1, T - n_sink - W) / 64), generator=gen)
-    cache = lrkv.LatentCache(B, H_kv, rk, rv, T, n_sink, W, dtype=dtype, page_perm=perm)
+    cache = lrkv.LatentCache(B, H_kv, rk, rv, T, n_sink, W, dtype=dtype,
+                             page_perm=None if contiguous else perm)
     K = torch.randn(B, H_kv, T, D, generator=gen).to(dtype).cuda()
     V = torch.randn(B, H_kv, T, D, generator=gen).to(dtype).cuda()
     Bp = B if per_seq else 1
@@ -151,3 +152,20 @@ def test_rebase_wide_ranks(lrkv):
     """r_k = r_v = 128 (the largest rank; one R per side staged at a time)."""
     _case(lrkv, dtype=torch.bfloat16, B=2, H_kv=1, G=8, rk=128, rv=128, n_sink=1, W=8,
           lens=[200, 75], per_seq=False, seed=5)
+
+
+def test_rebase_bf16_consecutive_pages(lrkv):
+    """bf16 codes at r 64/32 in a pool whose pages follow one another, so
+    page pairs arrive by one tensor load (about 4 pages per CTA); odd page
+    counts, partial last pages and range ends leave single-page jobs on the
+    chunk copies, and one sequence holds only anchors."""
+    _case(lrkv, dtype=torch.bfloat16, B=4, H_kv=4, G=4, rk=64, rv=32, n_sink=1, W=128,
+          lens=[4000, 64 * 5 + 129 + 7, 100, 64 * 40 + 129], per_seq=False, seed=6,
+          contiguous=True)
+
+
+def test_rebase_bf16_consecutive_pages_equal_ranks(lrkv):
+    """The same at r_k = r_v = 64 (16 chunks per page, a 32 KB box), about
+    3.5 pages per CTA."""
+    _case(lrkv, dtype=torch.bfloat16, B=2, H_kv=4, G=2, rk=64, rv=64, n_sink=1, W=8,
+          lens=[8000, 64 * 3 + 9 + 1], per_seq=False, seed=7, contiguous=True)
