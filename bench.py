@@ -91,7 +91,7 @@ TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum
     "llama3.1_8b_layer_T32768_anchors": {
         "bytes": 206470000, "context": 32771,
-        "sources": {"decode.cu": "6175b5086be0a15fe7a6b504c19bcbd86513a94ee6204801cf8df6087bc59efc",
+        "sources": {"decode.cu": "a5708206b9e5ec2d4f59d747935ec2f2276c7f63e0d2a388568107ff63295215",
                     "common.cuh": "867648f72ac4bef6638f39474ad2af8cef852d6f55e4d265fffd4c7212795edf"},
     },
 }
@@ -100,7 +100,7 @@ TRAFFIC = {
 TRAFFIC_WARM = {
     "llama3.1_8b_layer_T32768_anchors": {
         "bytes": 199030000, "context": 32773,
-        "sources": {"decode.cu": "6175b5086be0a15fe7a6b504c19bcbd86513a94ee6204801cf8df6087bc59efc",
+        "sources": {"decode.cu": "a5708206b9e5ec2d4f59d747935ec2f2276c7f63e0d2a388568107ff63295215",
                     "common.cuh": "867648f72ac4bef6638f39474ad2af8cef852d6f55e4d265fffd4c7212795edf"},
     },
 }
